@@ -36,7 +36,8 @@
  *  - a context of length 0 gives an all-zero output row;
  *  - FP8 values dequantise as code_value * scale[kv_head]; quantisation is
  *    code = nearest E4M3 value to (float)x / scale (IEEE single division), ties to the even code,
- *    magnitudes >= 448 (and infinities) saturate to +-448, NaN maps to the NaN code with its sign;
+ *    magnitudes >= 448 (and infinities) saturate to +-448, every NaN maps to the canonical NaN code
+ *    0x7F (the OCP spec does not fix the sign of a NaN produced by a conversion);
  *  - reshape_and_cache skips slots < 0 (padding) and slots past the pool.
  */
 #include <math.h>
@@ -105,11 +106,11 @@ double or_e4m3_to_double(uint8_t code) {
 }
 
 /* Encode a float to E4M3: the nearest finite E4M3 value, ties to the code with an even mantissa,
- * magnitudes at or above the largest finite value (448, including infinity) saturate to it, NaN maps
- * to the NaN code carrying the input's sign. The candidate set is searched directly: the 127
+ * magnitudes at or above the largest finite value (448, including infinity) saturate to it, and every
+ * NaN maps to the canonical NaN code 0x7F. The candidate set is searched directly: the 127
  * non-negative finite codes 0x00..0x7E have strictly increasing values. */
 uint8_t or_e4m3_from_float(float x) {
-  if (isnan(x)) return signbit(x) ? 0xFF : 0x7F;
+  if (isnan(x)) return 0x7F;
   uint8_t sign = signbit(x) ? 0x80 : 0x00;
   double a = fabs((double)x);
   if (a >= 448.0) return sign | 0x7E;

@@ -94,13 +94,13 @@ def test_e4m3_encode_is_nearest_by_brute_force():
         assert abs(oracle.e4m3_to_double([ci])[0] - xi) == best
 
 
-def test_e4m3_encode_saturates_and_keeps_nan():
+def test_e4m3_encode_saturates_and_maps_nan_to_canonical_nan():
     big = np.array([448.0, 449.0, 463.9, 464.0, 480.0, 1e6, 3.0e38, np.inf], np.float32)
     assert np.all(oracle.e4m3_from_float(big) == 0x7E)
     assert np.all(oracle.e4m3_from_float(-big) == 0xFE)
     nan = np.array([np.nan], np.float32)
     assert oracle.e4m3_from_float(nan)[0] == 0x7F
-    assert oracle.e4m3_from_float(-nan)[0] == 0xFF
+    assert oracle.e4m3_from_float(-nan)[0] == 0x7F   # reading: NaN of either sign -> canonical NaN
 
 
 def test_e4m3_encode_signed_zero_and_underflow():
