@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Benchmark of one paged decode step on B200: reshape_and_cache of each sequence's new token, then
+paged attention over the whole batch, on the 7B-shape decode workload (64 sequences, context lengths
+uniform in [512, 2048], 32 query / 32 kv heads, head size 128, block size 16, bf16, blocks shuffled
+across a 16384-block pool).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+Prints one JSON line (rank 0). `value` is the achieved KV-read bandwidth: the ideal bytes of every
+valid token's K and V row read once, divided by the device time of a step, summed over ranks and
+divided by the slowest rank's time. Multi-GPU runs shard independent sequences (one batch per rank,
+no collective on the data path; weak scaling). `--impl reference` times the CPU oracle instead.
+"""
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "paged decode attention: achieved KV-read HBM GB/s & % of peak; tokens/s"
+KERNEL_SOURCES = ("pa_attention.cuh", "pa_device.cuh", "pa_launch.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "paged_attention_main_7b_traffic.json")
+THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+                 0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+                 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+def bits16(t):
+    """Raw uint16 bits of a CPU fp16/bf16 tensor (how the oracle takes 16-bit arrays)."""
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def measured_peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except OSError:
+        return None
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "pagedattention_paged_kv_attention_b200", "csrc")
+    for name in KERNEL_SOURCES:
+        h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary, if it was taken
+    on the current kernel source and this workload; else None."""
+    try:
+        rec = json.load(open(TRAFFIC_FILE))
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_source_hash") != kernel_source_hash() or rec.get("workload") != workload:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while the timed region runs."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 3:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+                bits = int(parts[2], 16)
+            except ValueError:
+                continue
+            for b, name in THROTTLE_BITS.items():
+                if bits & b and name != "gpu_idle":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_selector(dev):
+    """nvidia-smi -i argument for the physical GPU behind a CUDA device (its UUID when known)."""
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    if uuid is not None:
+        u = str(uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    return str(dev.index)
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl" if args.impl != "reference" else "gloo",
+                                             timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def reduce_max(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def run_reference(args, cfg, world, rank):
+    """The CPU oracle timed on the machine's host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+    # pick a sample of sequences so that one step takes about 1 s
+    n, dt = 1, 0.0
+    while True:
+        w = W.make_workload(cfg, seed=cfg.seed, num_seqs=n, prefilled=True)
+        inp = dict(query_bits=bits16(w.query), q_dtype=cfg.dtype, key_cache=bits16(w.key_values),
+                   value_cache=bits16(w.value_values), kv_dtype=cfg.kv_dtype, block_tables=w.block_tables.numpy(),
+                   context_lens=w.context_lens.numpy(), scale=cfg.softmax_scale)
+        t0 = time.perf_counter()
+        oracle.paged_attention(**inp)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 or n >= cfg.num_seqs:
+            break
+        n = min(cfg.num_seqs, max(n * 2, int(n * 1.0 / max(dt, 1e-3))))
+    kv = W.ideal_bytes(w.context_lens.numpy(), cfg.num_kv_heads, cfg.head_size, 2, cfg.block_size,
+                       cfg.num_heads, 2)["kv"]
+    for _ in range(args.warmup):
+        oracle.paged_attention(**inp)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.paged_attention(**inp)
+        times.append(time.perf_counter() - t0)
+    t = float(np.mean(times))
+    value = kv / t / 1e9
+    sample = (f"{n} of {cfg.num_seqs} sequences of the workload ({int(w.context_lens.sum())} context tokens), "
+              f"fp64 oracle, one step = one pass over the sample")
+    cores = oracle.default_threads()
+    line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "impl": "reference", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.description, "name": cfg.name, "num_seqs_sampled": n},
+            "tokens_per_s": round(n / t, 3),
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="7b", choices=list(W.CONFIGS))
+    ap.add_argument("--partition-size", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    cfg = W.CONFIGS[args.workload]
+    world, rank, local = dist_setup(args)
+
+    if args.impl == "reference":
+        run_reference(args, cfg, world, rank)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    from pagedattention_paged_kv_attention_b200 import pagedattn as P
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = W.make_workload(cfg, seed=cfg.seed + 1000 * rank, device=dev)
+    S, H, d = w.query.shape
+    kv_bytes = 1 if cfg.kv_dtype == "fp8_e4m3" else 2
+    ks = vs = None
+    key_cache, value_cache = w.key_values, w.value_values
+    if cfg.kv_dtype == "fp8_e4m3":
+        # The product's own quantiser fills the FP8 pools from the drawn values.
+        NB, bs, Hkv, _ = key_cache.shape
+        ks, vs = w.k_scale.to(dev), w.v_scale.to(dev)
+        kq = torch.empty((NB, bs, Hkv, d), dtype=torch.uint8, device=dev)
+        vq = torch.empty_like(kq)
+        slots = torch.arange(NB * bs, dtype=torch.int64, device=dev)
+        P.reshape_and_cache(key_cache.view(NB * bs, Hkv, d), value_cache.view(NB * bs, Hkv, d), kq, vq, slots, ks, vs)
+        key_cache, value_cache = kq, vq
+        del slots
+    lens = w.context_lens.cpu().numpy()
+    mcl = int(lens.max())
+    ideal = W.ideal_bytes(lens, cfg.num_kv_heads, d, kv_bytes, cfg.block_size, H, 2)
+    ps = P.partition_size(S, H, cfg.num_kv_heads, mcl, args.partition_size)
+    parts = max(1, -(-mcl // ps))
+    ws = P.make_workspace(S, H, cfg.num_kv_heads, d, mcl, args.partition_size, device=dev)
+    out = torch.empty_like(w.query)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(q, nk, nv, slots, tables, clens, o, ev=None):
+        P.reshape_and_cache(nk, nv, key_cache, value_cache, slots, ks, vs)
+        if w.cow_mapping.shape[0]:
+            P.copy_blocks(key_cache, value_cache, w.cow_mapping)
+        if ev is not None:
+            ev[0].record(stream)
+        P.paged_attention(o, q, key_cache, value_cache, tables, clens, cfg.softmax_scale, mcl, ws, ks, vs,
+                          partition_size=args.partition_size)
+        if ev is not None:
+            ev[1].record(stream)
+
+    inputs = (w.query, w.new_key, w.new_value, w.slot_mapping, w.block_tables, w.context_lens)
+    launches_per_step = 2 + (1 if parts > 1 else 0) + (1 if w.cow_mapping.shape[0] else 0)
+
+    # ---- device-resident timing ----
+    for _ in range(args.warmup):
+        step(*inputs, out)
+    kernel_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_selector(dev)) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            step(*inputs, out, kernel_events[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = start.elapsed_time(stop) / args.steps
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in kernel_events]))
+    assert P.get_device_error(ws) == 0, "device error word set"
+    max_step_ms = reduce_max(step_ms, world, dev)
+    total_kv = reduce_sum(float(ideal["kv"]), world, dev)
+    total_seqs = reduce_sum(float(S), world, dev)
+    value = total_kv / (max_step_ms * 1e-3) / 1e9
+
+    # ---- end to end through the API: pinned host inputs in, output back to pinned host ----
+    host_in = [t.cpu().pin_memory() for t in inputs]
+    dev_in = [torch.empty_like(t) for t in inputs]
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for dst, src in zip(dev_in, host_in):
+            dst.copy_(src, non_blocking=True)
+        step(*dev_in, out)
+        host_out.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / args.steps, world, dev)
+    e2e_value = total_kv / (e2e_ms * 1e-3) / 1e9
+
+    if rank == 0:
+        peaks = measured_peaks()
+        peak = peaks["hbm_gbs"] if peaks else 6650.0
+        achieved = ideal["total"] / (attn_ms * 1e-3) / 1e9
+        workload = cfg.name
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(max_step_ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f16",
+            "data": "synthetic",
+            "config": {"workload": cfg.description, "name": cfg.name, "num_seqs": S, "num_heads": H,
+                       "num_kv_heads": cfg.num_kv_heads, "head_size": d, "block_size": cfg.block_size,
+                       "kv_dtype": cfg.kv_dtype, "context_tokens": int(lens.sum()), "max_context_len": mcl,
+                       "partition_size": ps, "partitions": parts, "seed": cfg.seed,
+                       "l2": "inputs larger than L2: %.2f GB of K/V read per step vs 126 MB L2" % (ideal["kv"] / 1e9),
+                       "parallelism": f"dp{world} (independent sequence batches)"},
+            "tokens_per_s": round(total_seqs / (max_step_ms * 1e-3), 1),
+            "pct_of_measured_hbm_peak": round(100 * value / peak, 2),
+            "pct_of_8tbs": round(100 * value / 8000.0, 2),
+            "roofline": {"kernel": "paged_attention (pa_paged_attention call: main kernel%s)" %
+                         (" + split-K reduce" if parts > 1 else ""),
+                         "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_source": "measured" if peaks else "fallback",
+                         "algorithmic_bytes_per_launch": ideal["total"], "avg_launch_ms": round(attn_ms, 4),
+                         "traffic": recorded_traffic(workload)},
+            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def cpu_baseline(cfg, seconds):
+    """The oracle (as it stands) on a bounded sample of the same workload, on the host cores."""
+    import oracle
+    n = 1
+    while True:
+        w = W.make_workload(cfg, seed=cfg.seed, num_seqs=n, prefilled=True)
+        inp = dict(query_bits=bits16(w.query), q_dtype=cfg.dtype, key_cache=bits16(w.key_values),
+                   value_cache=bits16(w.value_values), kv_dtype=cfg.kv_dtype, block_tables=w.block_tables.numpy(),
+                   context_lens=w.context_lens.numpy(), scale=cfg.softmax_scale)
+        t0 = time.perf_counter()
+        oracle.paged_attention(**inp)
+        dt = time.perf_counter() - t0
+        if dt >= seconds / 3 or n >= cfg.num_seqs:
+            break
+        n = min(cfg.num_seqs, max(n * 2, int(n * seconds / 3 / max(dt, 1e-3))))
+    reps, total = 0, 0.0
+    while total < seconds * 2 / 3 or reps == 0:
+        t0 = time.perf_counter()
+        oracle.paged_attention(**inp)
+        total += time.perf_counter() - t0
+        reps += 1
+    t = total / reps
+    kv = W.ideal_bytes(w.context_lens.numpy(), cfg.num_kv_heads, cfg.head_size, 2, cfg.block_size,
+                       cfg.num_heads, 2)["kv"]
+    return {"value": round(kv / t / 1e9, 4), "unit": "GB/s", "cores": oracle.default_threads(), "kind": "oracle",
+            "sample": f"{n} of {cfg.num_seqs} sequences ({int(w.context_lens.sum())} context tokens), "
+                      f"{reps} timed passes of {t:.2f} s, fp64",
+            "tokens_per_s": round(n / t, 3)}
+
+
+if __name__ == "__main__":
+    main()

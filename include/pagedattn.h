@@ -1,0 +1,194 @@
+/*
+ * pagedattn.h -- C ABI of libpagedattn.so: paged KV-cache decode attention on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow three web pages on PagedAttention, cited by title and section:
+ *  [T] "企业官网建设流程全解析" (the body is a PagedAttention tutorial; the title is unrelated):
+ *      sec. 2.1 "基本数据结构设计" -- KV stored in fixed-size blocks (16 tokens by default), a block table
+ *      mapping logical to physical blocks; sec. 2.2 "分块注意力计算过程" -- Attention(Q,K,V) =
+ *      softmax(QK^T/sqrt(d))V computed over the blocks; sec. 2.3 "显存共享机制" -- blocks shared by
+ *      reference count; sec. 3.2 "关键性能优化" -- preallocated block pool, asynchronous copies on CUDA
+ *      streams, FP8 storage of blocks.
+ *  [V] "vLLM的诞生背景：大模型推理的痛点与PagedAttention的破局": "PagedAttention的破局思路" -- blocks are
+ *      allocated on demand as a sequence grows; "PagedAttention的局限性" -- copy-on-write of shared
+ *      blocks, extra indexing cost of scattered blocks, block-size tuning.
+ *  [C] "PagedAttention 与连续批处理：LLM Serving 的底层架构拆解": "PagedAttention：把显存做成虚拟内存" --
+ *      attention finds each page through the page table; "对 agent 开发者的启示" -- decode is
+ *      memory-bound.
+ *
+ * Conventions for every entry point
+ *  - Ownership: the caller allocates every buffer (the block pool is preallocated, [T] sec. 3.2). The
+ *    library allocates nothing, keeps no per-call state and never frees caller memory.
+ *  - Pointers are DEVICE pointers unless a parameter says "host". Every device pointer must be 16-byte
+ *    aligned. Tensors are dense, row-major, in the layouts given below.
+ *  - Asynchrony: each call validates its arguments on the host, enqueues its kernels on `stream` and
+ *    returns without synchronising ([T] sec. 3.2). A NULL stream is the legacy default stream.
+ *  - Errors: invalid arguments are reported before anything is enqueued (nothing runs, no CUDA call is
+ *    made). Launch failures return PA_ERR_CUDA. The library never aborts, never throws across the ABI
+ *    and its kernels never trap; contract violations that only the device can see (a block id
+ *    outside the pool, a context length past the table or past max_context_len) are recorded in the
+ *    workspace's error word (see pa_get_device_error) and the affected output rows are set to NaN.
+ *
+ * Cache layout (shared by all calls): key_cache and value_cache are
+ *   [num_blocks][block_size][num_kv_heads][head_size]
+ * so element (blk, off, h, i) lives at ((blk*block_size + off)*num_kv_heads + h)*head_size + i.
+ * Token t of sequence s is stored in physical block block_tables[s][t / block_size] at offset
+ * t % block_size ([T] sec. 2.1; [V] "PagedAttention的破局思路").
+ *
+ * Supported set: head_size in {64, 128}; block_size in {8, 16, 32, 64}; num_heads % num_kv_heads == 0;
+ * query/output dtype PA_F16 or PA_BF16; cache dtype equal to the query dtype, or PA_FP8_E4M3 with
+ * head_size 128. Anything else returns PA_ERR_UNSUPPORTED.
+ */
+#ifndef PAGEDATTN_H_
+#define PAGEDATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+struct CUstream_st;                     /* cudaStream_t is `struct CUstream_st *` */
+typedef struct CUstream_st* pa_stream_t;
+
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARGUMENT = 1,          /* null/misaligned pointer, negative size, bad mapping, ... */
+  PA_ERR_UNSUPPORTED = 2,               /* valid but outside the supported set above */
+  PA_ERR_WORKSPACE_TOO_SMALL = 3,       /* workspace_bytes < pa_paged_attention_workspace_size(...) */
+  PA_ERR_CUDA = 4                       /* a CUDA runtime/driver call or a launch failed */
+} pa_status;
+
+typedef enum pa_dtype {
+  PA_F16 = 0,                           /* IEEE binary16 */
+  PA_BF16 = 1,                          /* bfloat16 */
+  PA_FP8_E4M3 = 2                       /* OCP FP8 E4M3 (bias 7, max 448, no infinities) */
+} pa_dtype;
+
+/* Bits of the device error word (pa_get_device_error). */
+#define PA_DEVERR_BLOCK_ID    0x1u      /* a needed block-table entry was outside [0, num_blocks) */
+#define PA_DEVERR_CONTEXT_LEN 0x2u      /* context_lens[s] < 0, > max_blocks_per_seq*block_size or
+                                           > max_context_len */
+#define PA_DEVERR_TIMEOUT     0x4u      /* a pipeline wait inside a kernel gave up (should not happen) */
+
+/* Bytes of the workspace header that holds the device error word (the workspace's first bytes). */
+#define PA_WORKSPACE_HEADER_BYTES 256
+
+/*
+ * Tokens per context partition that pa_paged_attention will use for these sizes.
+ * partition_size > 0 requests that size (it must be a multiple of 64); 0 lets the library choose from
+ * num_seqs, num_heads/num_kv_heads and max_context_len (the choice depends on nothing else).
+ * Returns the partition size, or -1 if the request is invalid. Host only; makes no CUDA call.
+ */
+PA_API int pa_paged_attention_partition_size(int num_seqs, int num_heads, int num_kv_heads,
+                                      int max_context_len, int partition_size);
+
+/*
+ * Workspace bytes pa_paged_attention needs for these sizes (same partition_size rule as above):
+ * PA_WORKSPACE_HEADER_BYTES for the error word plus, when the context is split into P > 1
+ * partitions, fp32 partial results num_seqs*num_heads*P*(head_size + 2)*4 bytes.
+ * Returns 0 if the arguments are invalid. Host only; makes no CUDA call.
+ */
+PA_API size_t pa_paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_size,
+                                         int max_context_len, int partition_size);
+
+/*
+ * Paged decode attention ([T] sec. 2.2 formula, normalised over the whole context; [C]
+ * "PagedAttention：把显存做成虚拟内存" for the page-table walk). For each sequence s and query head h,
+ * with G = num_heads / num_kv_heads and kv head h / G:
+ *     out[s][h][:] = sum_t softmax_t(scale * q[s][h] . k_t) * v_t,   t = 0 .. context_lens[s]-1,
+ * where k_t / v_t are read from block block_tables[s][t / block_size] at offset t % block_size.
+ * FP8 caches dequantise as code * k_scale[kv head] (resp. v_scale). A context of length 0 gives 0.
+ *
+ *  out            [num_seqs][num_heads][head_size], q_dtype; written.
+ *  query          [num_seqs][num_heads][head_size], q_dtype (PA_F16 or PA_BF16).
+ *  key_cache,
+ *  value_cache    [num_blocks][block_size][num_kv_heads][head_size], kv_dtype; read only.
+ *  k_scale,
+ *  v_scale        [num_kv_heads] fp32 dequantisation scales; required for PA_FP8_E4M3, else ignored.
+ *  block_tables   [num_seqs][max_blocks_per_seq] int32 physical block ids; entries past
+ *                 ceil(context_lens[s]/block_size) are never read.
+ *  context_lens   [num_seqs] int32.
+ *  max_context_len host int, >= every context_lens[s]; sizes the launch (partitions).
+ *  scale          the softmax scale (1/sqrt(head_size) in the pages' formula).
+ *  partition_size 0 = library's choice, else a multiple of 64 (tokens per split-K partition).
+ *  workspace      device scratch of workspace_bytes >= pa_paged_attention_workspace_size(...); its
+ *                 first PA_WORKSPACE_HEADER_BYTES hold the error word, which the caller zeroes once
+ *                 (e.g. with cudaMemset or pa_clear_device_error) and the kernels only OR into.
+ * Calls that share a workspace must be ordered on one stream. num_seqs == 0 is a no-op (pointers
+ * may then be NULL).
+ */
+PA_API pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dtype,
+                             const void* key_cache, const void* value_cache, pa_dtype kv_dtype,
+                             const float* k_scale, const float* v_scale,
+                             const int32_t* block_tables, int max_blocks_per_seq,
+                             const int32_t* context_lens, int num_seqs, int num_heads,
+                             int num_kv_heads, int head_size, int block_size, int num_blocks,
+                             int max_context_len, float scale, int partition_size,
+                             void* workspace, size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * Write new tokens into their physical slots ([V] "PagedAttention的破局思路": blocks are filled as the
+ * sequence grows). For token i with slot = slot_mapping[i] in [0, num_blocks*block_size):
+ *     key_cache[slot / block_size][slot % block_size][h][:] = key[i][h][:]   (same for value)
+ * slot < 0 marks padding and is skipped; slots past the pool are skipped too. For an FP8 cache each
+ * element stores the E4M3 code of (float)x / k_scale[h] (IEEE division, round to nearest even,
+ * magnitudes beyond 448 saturate, any NaN becomes the canonical NaN code 0x7F).
+ *
+ *  key, value     [num_tokens][num_kv_heads][head_size], in_dtype (PA_F16 or PA_BF16); read only.
+ *  key_cache,
+ *  value_cache    as above, kv_dtype = in_dtype or PA_FP8_E4M3; written at the given slots only.
+ *  k_scale,
+ *  v_scale        [num_kv_heads] fp32, required for PA_FP8_E4M3.
+ *  slot_mapping   [num_tokens] int64.
+ * Two tokens mapped to the same slot race (the result is one of them).
+ */
+PA_API pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dtype in_dtype,
+                               void* key_cache, void* value_cache, pa_dtype kv_dtype,
+                               const float* k_scale, const float* v_scale,
+                               const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                               int head_size, int block_size, int num_blocks, pa_stream_t stream);
+
+/*
+ * Copy-on-write of shared blocks ([V] "PagedAttention的局限性"; sharing by reference count in [T]
+ * sec. 2.3): for each pair p, copy the whole key block and the whole value block
+ * block_mapping[p][0] -> block_mapping[p][1].
+ *
+ *  block_mapping  [num_pairs][2] int64 (src, dst), device. Pairs with an id outside [0, num_blocks)
+ *                 are skipped. Destinations must be distinct and must not be a source of any pair
+ *                 (otherwise the copies race); pa_copy_blocks_check verifies this on a host copy.
+ */
+PA_API pa_status pa_copy_blocks(void* key_cache, void* value_cache, pa_dtype kv_dtype,
+                         const int64_t* block_mapping, int num_pairs, int num_kv_heads,
+                         int head_size, int block_size, int num_blocks, pa_stream_t stream);
+
+/*
+ * Host-side check of a copy_blocks mapping (host pointer, [num_pairs][2] int64): every id in
+ * [0, num_blocks), destinations distinct, no destination also a source. PA_OK or
+ * PA_ERR_INVALID_ARGUMENT. Makes no CUDA call.
+ */
+PA_API pa_status pa_copy_blocks_check(const int64_t* host_block_mapping, int num_pairs, int num_blocks);
+
+/*
+ * Read the device error word of a workspace into *err_out (host pointer). Synchronises `stream`.
+ * Returns PA_ERR_CUDA if the copy or the synchronisation fails.
+ */
+PA_API pa_status pa_get_device_error(const void* workspace, unsigned int* err_out, pa_stream_t stream);
+
+/* Zero the device error word of a workspace (enqueued on `stream`, asynchronous). */
+PA_API pa_status pa_clear_device_error(void* workspace, pa_stream_t stream);
+
+/* Static description of a status code. Never NULL. */
+PA_API const char* pa_status_string(pa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H_ */

@@ -1,0 +1,308 @@
+// pa_api.cu -- the C ABI of libpagedattn.so (declared and documented in include/pagedattn.h).
+//
+// Host side only: argument validation (before any CUDA call), launch planning (partition size, grid,
+// workspace layout), TMA descriptor encoding and dispatch to the kernels. Nothing here allocates
+// device memory; every buffer belongs to the caller (tutorial page "企业官网建设流程全解析", sec. 3.2
+// "关键性能优化": the block pool is preallocated at start-up; work is issued asynchronously on CUDA
+// streams).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+#include <unordered_set>
+
+#include "pa_cache_ops.cuh"
+#include "pa_launch.cuh"
+#include "pagedattn.h"
+
+namespace {
+
+constexpr int kPlanSMs = 148;            // B200 SM count; planning is a pure function of the sizes
+constexpr int kPlanCtasPerSm = 2;
+constexpr int kPlanWaves = 8;
+constexpr int kMinAutoPartition = 256;
+constexpr int kMaxAutoPartition = 1024;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Query heads handled per CTA (the kernel template's G) and CTAs per kv head.
+void group_tiling(int group, int* g_tile, int* subgroups) {
+  int g = 1;
+  while (g < group && g < 8) g *= 2;
+  *g_tile = g;
+  *subgroups = ceil_div(group, g);
+}
+
+int plan_partition(int num_seqs, int num_heads, int num_kv_heads, int max_context_len, int partition_size) {
+  if (partition_size < 0) return -1;
+  if (partition_size > 0) return (partition_size % pa::kStageTokens == 0) ? partition_size : -1;
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads || max_context_len < 0)
+    return -1;
+  int g_tile, subgroups;
+  group_tiling(num_heads / num_kv_heads, &g_tile, &subgroups);
+  const long items = std::max<long>(1, static_cast<long>(num_seqs) * num_kv_heads * subgroups);
+  const long target = static_cast<long>(kPlanSMs) * kPlanCtasPerSm * kPlanWaves;
+  const long splits = std::max<long>(1, (target + items - 1) / items);
+  long ps = (std::max(1, max_context_len) + splits - 1) / splits;
+  ps = round_up(static_cast<size_t>(ps), pa::kStageTokens);
+  ps = std::min<long>(std::max<long>(ps, kMinAutoPartition), kMaxAutoPartition);
+  return static_cast<int>(ps);
+}
+
+struct WorkspaceLayout {
+  size_t part_m, part_l, part_o, total;
+};
+
+WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_size, int partitions) {
+  WorkspaceLayout w{};
+  w.total = PA_WORKSPACE_HEADER_BYTES;
+  if (partitions > 1) {
+    const size_t rows = static_cast<size_t>(num_seqs) * num_heads * partitions;
+    w.part_m = w.total;
+    w.part_l = w.part_m + round_up(rows * 4, 256);
+    w.part_o = w.part_l + round_up(rows * 4, 256);
+    w.total = w.part_o + round_up(rows * head_size * 4, 256);
+  }
+  return w;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 4-D view {head_size, num_kv_heads, block_size, num_blocks} of a cache; box = one 128-byte chunk of
+// `block_size` rows of one kv head of one block, written to shared memory with the 128-byte swizzle.
+bool encode_cache_map(CUtensorMap* map, const void* cache, int elem_bytes, int head_size, int num_kv_heads,
+                      int block_size, int num_blocks) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return false;
+  const cuuint64_t e = static_cast<cuuint64_t>(elem_bytes);
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_size), static_cast<cuuint64_t>(num_kv_heads),
+                        static_cast<cuuint64_t>(block_size), static_cast<cuuint64_t>(num_blocks)};
+  cuuint64_t strides[3] = {head_size * e, num_kv_heads * head_size * e, block_size * num_kv_heads * head_size * e};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), 1, static_cast<cuuint32_t>(block_size), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = encode(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
+                      const_cast<void*>(cache), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool is_16bit(pa_dtype t) { return t == PA_F16 || t == PA_BF16; }
+bool is_dtype(pa_dtype t) { return t == PA_F16 || t == PA_BF16 || t == PA_FP8_E4M3; }
+int elem_bytes(pa_dtype t) { return t == PA_FP8_E4M3 ? 1 : 2; }
+bool supported_block_size(int bs) { return bs == 8 || bs == 16 || bs == 32 || bs == 64; }
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(pa_status status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARGUMENT: return "PA_ERR_INVALID_ARGUMENT: invalid argument (null/misaligned pointer, bad size or mapping)";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: valid but outside the supported head_size/block_size/dtype set";
+    case PA_ERR_WORKSPACE_TOO_SMALL: return "PA_ERR_WORKSPACE_TOO_SMALL: workspace smaller than pa_paged_attention_workspace_size()";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA: a CUDA call or kernel launch failed";
+  }
+  return "unknown pa_status";
+}
+
+int pa_paged_attention_partition_size(int num_seqs, int num_heads, int num_kv_heads, int max_context_len,
+                                      int partition_size) {
+  return plan_partition(num_seqs, num_heads, num_kv_heads, max_context_len, partition_size);
+}
+
+size_t pa_paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_size,
+                                         int max_context_len, int partition_size) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_size <= 0 || max_context_len < 0) return 0;
+  const int ps = plan_partition(num_seqs, num_heads, num_kv_heads, max_context_len, partition_size);
+  if (ps <= 0) return 0;
+  const int partitions = std::max(1, ceil_div(max_context_len, ps));
+  return workspace_layout(num_seqs, num_heads, head_size, partitions).total;
+}
+
+pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dtype, const void* key_cache,
+                             const void* value_cache, pa_dtype kv_dtype, const float* k_scale,
+                             const float* v_scale, const int32_t* block_tables, int max_blocks_per_seq,
+                             const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                             int head_size, int block_size, int num_blocks, int max_context_len, float scale,
+                             int partition_size, void* workspace, size_t workspace_bytes,
+                             pa_stream_t stream) {
+  // ---- validation: no CUDA call before every check has passed ----
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
+      head_size <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 ||
+      partition_size < 0 || !std::isfinite(scale))
+    return PA_ERR_INVALID_ARGUMENT;
+  if (!is_dtype(q_dtype) || !is_dtype(kv_dtype) || !is_16bit(q_dtype)) return PA_ERR_INVALID_ARGUMENT;
+  if (num_seqs == 0) return PA_OK;  // empty batch: nothing is read or written
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens || !workspace)
+    return PA_ERR_INVALID_ARGUMENT;
+  if (!aligned(out, 16) || !aligned(query, 16) || !aligned(key_cache, 16) || !aligned(value_cache, 16) ||
+      !aligned(workspace, 16) || !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return PA_ERR_INVALID_ARGUMENT;
+  const bool fp8 = kv_dtype == PA_FP8_E4M3;
+  if (fp8 && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4))) return PA_ERR_INVALID_ARGUMENT;
+  if (!fp8 && kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;
+  if (head_size != 64 && head_size != 128) return PA_ERR_UNSUPPORTED;
+  if (fp8 && head_size != 128) return PA_ERR_UNSUPPORTED;
+  if (!supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+  const int ps = plan_partition(num_seqs, num_heads, num_kv_heads, max_context_len, partition_size);
+  if (ps <= 0) return PA_ERR_INVALID_ARGUMENT;
+  const int partitions = std::max(1, ceil_div(max_context_len, ps));
+  int g_tile, subgroups;
+  group_tiling(num_heads / num_kv_heads, &g_tile, &subgroups);
+  if (num_seqs > 65535 || partitions > 65535 || static_cast<long>(num_kv_heads) * subgroups > 0x7fffffffL)
+    return PA_ERR_UNSUPPORTED;
+  const WorkspaceLayout ws = workspace_layout(num_seqs, num_heads, head_size, partitions);
+  if (workspace_bytes < ws.total) return PA_ERR_WORKSPACE_TOO_SMALL;
+
+  // ---- launch ----
+  CUtensorMap tk, tv;
+  const int eb = elem_bytes(kv_dtype);
+  if (!encode_cache_map(&tk, key_cache, eb, head_size, num_kv_heads, block_size, num_blocks) ||
+      !encode_cache_map(&tv, value_cache, eb, head_size, num_kv_heads, block_size, num_blocks))
+    return PA_ERR_CUDA;
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  pa::AttnArgs a{};
+  a.out = out;
+  a.query = query;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.part_m = partitions > 1 ? reinterpret_cast<float*>(wsb + ws.part_m) : nullptr;
+  a.part_l = partitions > 1 ? reinterpret_cast<float*>(wsb + ws.part_l) : nullptr;
+  a.part_o = partitions > 1 ? reinterpret_cast<float*>(wsb + ws.part_o) : nullptr;
+  a.error_word = reinterpret_cast<unsigned int*>(wsb);
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.group = num_heads / num_kv_heads;
+  a.subgroups = subgroups;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.partition_size = ps;
+  a.num_partitions = partitions;
+  a.scale_log2 = scale * pa::kLog2e;
+  const dim3 grid(static_cast<unsigned>(num_kv_heads * subgroups), static_cast<unsigned>(num_seqs),
+                  static_cast<unsigned>(partitions));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = q_dtype == PA_BF16 ? pa::launch_attention_bf16(tk, tv, a, fp8, head_size, g_tile, grid, st)
+                                     : pa::launch_attention_f16(tk, tv, a, fp8, head_size, g_tile, grid, st);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dtype in_dtype, void* key_cache,
+                               void* value_cache, pa_dtype kv_dtype, const float* k_scale, const float* v_scale,
+                               const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_size,
+                               int block_size, int num_blocks, pa_stream_t stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_size <= 0 || block_size <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID_ARGUMENT;
+  if (!is_dtype(in_dtype) || !is_dtype(kv_dtype) || !is_16bit(in_dtype)) return PA_ERR_INVALID_ARGUMENT;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_INVALID_ARGUMENT;
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(key_cache, 16) || !aligned(value_cache, 16) ||
+      !aligned(slot_mapping, 8))
+    return PA_ERR_INVALID_ARGUMENT;
+  const bool fp8 = kv_dtype == PA_FP8_E4M3;
+  if (fp8 && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4))) return PA_ERR_INVALID_ARGUMENT;
+  if (!fp8 && kv_dtype != in_dtype) return PA_ERR_UNSUPPORTED;
+  if (head_size % 8 != 0) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  const int row = num_kv_heads * head_size;
+  const int threads = static_cast<int>(std::min<size_t>(256, round_up(static_cast<size_t>(ceil_div(row, 8)), 32)));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid(static_cast<unsigned>(num_tokens));
+  if (in_dtype == PA_BF16) {
+    if (fp8)
+      pa::reshape_and_cache_kernel<__nv_bfloat16, __nv_fp8_e4m3><<<grid, threads, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(key), static_cast<const __nv_bfloat16*>(value),
+          static_cast<__nv_fp8_e4m3*>(key_cache), static_cast<__nv_fp8_e4m3*>(value_cache), k_scale, v_scale,
+          slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+    else
+      pa::reshape_and_cache_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, threads, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(key), static_cast<const __nv_bfloat16*>(value),
+          static_cast<__nv_bfloat16*>(key_cache), static_cast<__nv_bfloat16*>(value_cache), k_scale, v_scale,
+          slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+  } else {
+    if (fp8)
+      pa::reshape_and_cache_kernel<__half, __nv_fp8_e4m3><<<grid, threads, 0, st>>>(
+          static_cast<const __half*>(key), static_cast<const __half*>(value), static_cast<__nv_fp8_e4m3*>(key_cache),
+          static_cast<__nv_fp8_e4m3*>(value_cache), k_scale, v_scale, slot_mapping, num_kv_heads, head_size,
+          block_size, num_blocks);
+    else
+      pa::reshape_and_cache_kernel<__half, __half><<<grid, threads, 0, st>>>(
+          static_cast<const __half*>(key), static_cast<const __half*>(value), static_cast<__half*>(key_cache),
+          static_cast<__half*>(value_cache), k_scale, v_scale, slot_mapping, num_kv_heads, head_size, block_size,
+          num_blocks);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_copy_blocks(void* key_cache, void* value_cache, pa_dtype kv_dtype, const int64_t* block_mapping,
+                         int num_pairs, int num_kv_heads, int head_size, int block_size, int num_blocks,
+                         pa_stream_t stream) {
+  if (num_pairs < 0 || num_kv_heads <= 0 || head_size <= 0 || block_size <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID_ARGUMENT;
+  if (!is_dtype(kv_dtype)) return PA_ERR_INVALID_ARGUMENT;
+  if (!key_cache || !value_cache || (num_pairs > 0 && !block_mapping)) return PA_ERR_INVALID_ARGUMENT;
+  if (!aligned(key_cache, 16) || !aligned(value_cache, 16) || (block_mapping && !aligned(block_mapping, 8)))
+    return PA_ERR_INVALID_ARGUMENT;
+  const int64_t block_bytes = static_cast<int64_t>(block_size) * num_kv_heads * head_size * elem_bytes(kv_dtype);
+  if (block_bytes % 16 != 0) return PA_ERR_UNSUPPORTED;
+  if (num_pairs == 0) return PA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  pa::copy_blocks_kernel<<<dim3(static_cast<unsigned>(num_pairs), 2), 256, 0, st>>>(
+      static_cast<uint8_t*>(key_cache), static_cast<uint8_t*>(value_cache), block_mapping, block_bytes, num_blocks);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_copy_blocks_check(const int64_t* host_block_mapping, int num_pairs, int num_blocks) {
+  if (num_pairs < 0 || num_blocks <= 0 || (num_pairs > 0 && !host_block_mapping)) return PA_ERR_INVALID_ARGUMENT;
+  std::unordered_set<int64_t> srcs, dsts;
+  for (int p = 0; p < num_pairs; ++p) {
+    const int64_t s = host_block_mapping[2 * p], d = host_block_mapping[2 * p + 1];
+    if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) return PA_ERR_INVALID_ARGUMENT;
+    srcs.insert(s);
+    if (!dsts.insert(d).second) return PA_ERR_INVALID_ARGUMENT;
+  }
+  for (int64_t d : dsts)
+    if (srcs.count(d)) return PA_ERR_INVALID_ARGUMENT;
+  return PA_OK;
+}
+
+pa_status pa_get_device_error(const void* workspace, unsigned int* err_out, pa_stream_t stream) {
+  if (!workspace || !err_out || !aligned(workspace, 16)) return PA_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int value = 0;
+  if (cudaMemcpyAsync(&value, workspace, sizeof(value), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PA_ERR_CUDA;
+  *err_out = value;
+  return PA_OK;
+}
+
+pa_status pa_clear_device_error(void* workspace, pa_stream_t stream) {
+  if (!workspace || !aligned(workspace, 16)) return PA_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return cudaMemsetAsync(workspace, 0, sizeof(unsigned int), st) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // extern "C"

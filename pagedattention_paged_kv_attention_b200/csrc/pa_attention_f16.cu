@@ -1,0 +1,10 @@
+// Attention kernels instantiated for float16 queries (float16 or FP8-E4M3 caches).
+#include "pa_launch.cuh"
+
+namespace pa {
+cudaError_t launch_attention_f16(const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a, bool fp8_cache,
+                                 int D, int G, dim3 grid, cudaStream_t stream) {
+  if (fp8_cache) return launch_attention<__half, __nv_fp8_e4m3>(tk, tv, a, D, G, grid, stream);
+  return launch_attention<__half, __half>(tk, tv, a, D, G, grid, stream);
+}
+}  // namespace pa

@@ -1,0 +1,81 @@
+// pa_cache_ops.cuh -- writing new tokens into their slots and copy-on-write of whole blocks.
+//
+// reshape_and_cache: page "vLLM的诞生背景：大模型推理的痛点与PagedAttention的破局", section
+// "PagedAttention的破局思路" -- a sequence's KV grows into blocks allocated on demand; token i goes to
+// slot slot_mapping[i] = block * block_size + offset. FP8 caches (tutorial page "企业官网建设流程全解析",
+// sec. 3.2 "关键性能优化", FP8 storage of blocks) store E4M3(x / scale[kv head]).
+// copy_blocks: same page, section "PagedAttention的局限性" -- copy-on-write of shared blocks.
+// Both are pure data movement (plus the FP8 encode): 16-byte vector loads and stores, no staging.
+#pragma once
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+// One CTA per token; thread i handles 8 consecutive elements of the token's [Hkv][D] row.
+template <typename IT, typename KVT>
+__global__ void __launch_bounds__(256)
+reshape_and_cache_kernel(const IT* __restrict__ key, const IT* __restrict__ value, KVT* __restrict__ key_cache,
+                         KVT* __restrict__ value_cache, const float* __restrict__ k_scale,
+                         const float* __restrict__ v_scale, const int64_t* __restrict__ slot_mapping,
+                         int num_kv_heads, int head_size, int block_size, int num_blocks) {
+  const int64_t token = blockIdx.x;
+  const int64_t slot = slot_mapping[token];
+  if (slot < 0 || slot >= static_cast<int64_t>(num_blocks) * block_size) return;
+  const int64_t blk = slot / block_size;
+  const int64_t off = slot - blk * block_size;
+  const int row = num_kv_heads * head_size;  // elements per token
+  const IT* ksrc = key + token * row;
+  const IT* vsrc = value + token * row;
+  const int64_t dst_base = (blk * block_size + off) * row;
+  for (int e = threadIdx.x * 8; e < row; e += blockDim.x * 8) {
+    const uint4 kin = *reinterpret_cast<const uint4*>(ksrc + e);
+    const uint4 vin = *reinterpret_cast<const uint4*>(vsrc + e);
+    if constexpr (sizeof(KVT) == sizeof(IT)) {
+      *reinterpret_cast<uint4*>(key_cache + dst_base + e) = kin;
+      *reinterpret_cast<uint4*>(value_cache + dst_base + e) = vin;
+    } else {
+      // E4M3: code = cvt.rn.satfinite(x / scale), the division correctly rounded (IEEE).
+      const int h = e / head_size;
+      const float ks = k_scale[h], vs = v_scale[h];
+      const IT* kx = reinterpret_cast<const IT*>(&kin);
+      const IT* vx = reinterpret_cast<const IT*>(&vin);
+      uint32_t kout[2], vout[2];
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        uint32_t kw = 0, vw = 0;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int i = w * 4 + k * 2;
+          const float2 kf = make_float2(__fdiv_rn(to_f32(kx[i]), ks), __fdiv_rn(to_f32(kx[i + 1]), ks));
+          const float2 vf = make_float2(__fdiv_rn(to_f32(vx[i]), vs), __fdiv_rn(to_f32(vx[i + 1]), vs));
+          const uint32_t kc = __nv_cvt_float2_to_fp8x2(kf, __NV_SATFINITE, __NV_E4M3);
+          const uint32_t vc = __nv_cvt_float2_to_fp8x2(vf, __NV_SATFINITE, __NV_E4M3);
+          kw |= (kc & 0xffffu) << (16 * k);
+          vw |= (vc & 0xffffu) << (16 * k);
+        }
+        kout[w] = kw;
+        vout[w] = vw;
+      }
+      *reinterpret_cast<uint2*>(key_cache + dst_base + e) = make_uint2(kout[0], kout[1]);
+      *reinterpret_cast<uint2*>(value_cache + dst_base + e) = make_uint2(vout[0], vout[1]);
+    }
+  }
+}
+
+// One CTA per (pair, key|value): copy one contiguous block of `block_bytes` (a multiple of 16).
+__global__ void __launch_bounds__(256)
+copy_blocks_kernel(uint8_t* __restrict__ key_cache, uint8_t* __restrict__ value_cache,
+                   const int64_t* __restrict__ block_mapping, int64_t block_bytes, int num_blocks) {
+  const int pair = blockIdx.x;
+  const int64_t src = block_mapping[2 * pair];
+  const int64_t dst = block_mapping[2 * pair + 1];
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) return;
+  uint8_t* base = blockIdx.y == 0 ? key_cache : value_cache;
+  const uint4* s = reinterpret_cast<const uint4*>(base + src * block_bytes);
+  uint4* d = reinterpret_cast<uint4*>(base + dst * block_bytes);
+  const int64_t n = block_bytes / 16;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) d[i] = s[i];
+}
+
+}  // namespace pa

@@ -1,0 +1,169 @@
+// pa_device.cuh -- small sm_100a device helpers: mbarriers, TMA tile loads, bounded waits, packed
+// conversions. Hand-written inline PTX; no library kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "pa_errors.h"
+
+namespace pa {
+
+// ------------------------------------------------------------------------------------------------
+// Shared-memory addresses and mbarriers.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("{ .reg .b64 st; mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1; }"
+               ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Every wait in these kernels is bounded: after kWaitLimitNs without progress the waiter records
+// PA_DEVERR_TIMEOUT in the error word and returns false, so no kernel can spin forever.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s; a healthy wait lasts microseconds
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* error_word) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t start = global_timer_ns();
+  for (uint32_t spin = 0;; ++spin) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((spin & 63u) == 63u && global_timer_ns() - start > kWaitLimitNs) {
+      atomicOr(error_word, PA_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// TMA: 4-D tiled load global -> shared, completion counted on an mbarrier (no multicast).
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+        "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+// Named barrier over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// ------------------------------------------------------------------------------------------------
+// Packed conversions to float2 (8 elements = one 16-byte or 8-byte piece of a row).
+// ------------------------------------------------------------------------------------------------
+// bfloat16 is the upper half of a binary32: widening is a shift / mask, exact.
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+__device__ __forceinline__ float2 f16x2_to_float2(uint32_t w) {
+  __half2 h = *reinterpret_cast<__half2*>(&w);
+  return __half22float2(h);
+}
+
+// Two E4M3 codes (low byte = first element) -> two floats, exact (hardware conversion via f16).
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t w) {
+  __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w), __NV_E4M3);
+  __half2 h = *reinterpret_cast<__half2*>(&hr);
+  return __half22float2(h);
+}
+
+template <typename T>
+struct Elem;
+template <>
+struct Elem<__nv_bfloat16> {
+  static constexpr int kBytes = 2;
+  using Piece = uint4;  // 8 elements
+  __device__ static __forceinline__ void to_float(const Piece& p, float2 (&f)[4]) {
+    f[0] = bf16x2_to_float2(p.x);
+    f[1] = bf16x2_to_float2(p.y);
+    f[2] = bf16x2_to_float2(p.z);
+    f[3] = bf16x2_to_float2(p.w);
+  }
+};
+template <>
+struct Elem<__half> {
+  static constexpr int kBytes = 2;
+  using Piece = uint4;
+  __device__ static __forceinline__ void to_float(const Piece& p, float2 (&f)[4]) {
+    f[0] = f16x2_to_float2(p.x);
+    f[1] = f16x2_to_float2(p.y);
+    f[2] = f16x2_to_float2(p.z);
+    f[3] = f16x2_to_float2(p.w);
+  }
+};
+template <>
+struct Elem<__nv_fp8_e4m3> {
+  static constexpr int kBytes = 1;
+  using Piece = uint2;
+  __device__ static __forceinline__ void to_float(const Piece& p, float2 (&f)[4]) {
+    f[0] = e4m3x2_to_float2(static_cast<uint16_t>(p.x & 0xffffu));
+    f[1] = e4m3x2_to_float2(static_cast<uint16_t>(p.x >> 16));
+    f[2] = e4m3x2_to_float2(static_cast<uint16_t>(p.y & 0xffffu));
+    f[3] = e4m3x2_to_float2(static_cast<uint16_t>(p.y >> 16));
+  }
+};
+
+// Output conversion of 4 floats to the query dtype (round to nearest even), packed into 8 bytes.
+template <typename T>
+__device__ __forceinline__ uint2 pack4(float a, float b, float c, float d);
+template <>
+__device__ __forceinline__ uint2 pack4<__nv_bfloat16>(float a, float b, float c, float d) {
+  __nv_bfloat162 x = __floats2bfloat162_rn(a, b), y = __floats2bfloat162_rn(c, d);
+  return make_uint2(*reinterpret_cast<uint32_t*>(&x), *reinterpret_cast<uint32_t*>(&y));
+}
+template <>
+__device__ __forceinline__ uint2 pack4<__half>(float a, float b, float c, float d) {
+  __half2 x = __floats2half2_rn(a, b), y = __floats2half2_rn(c, d);
+  return make_uint2(*reinterpret_cast<uint32_t*>(&x), *reinterpret_cast<uint32_t*>(&y));
+}
+
+// Query element -> float.
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+}  // namespace pa

@@ -1,0 +1,149 @@
+"""Thin ctypes binding of libpagedattn.so (the C ABI in include/pagedattn.h).
+
+Argument marshalling only: tensors become device pointers and the current CUDA stream becomes a
+cudaStream_t; every step of the computation runs in the library's CUDA kernels. PyTorch is used for
+device memory and streams. Importing this module fails loudly if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_HERE, "libpagedattn.so")
+
+PA_OK, PA_ERR_INVALID_ARGUMENT, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL, PA_ERR_CUDA = range(5)
+PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
+PA_DEVERR_BLOCK_ID, PA_DEVERR_CONTEXT_LEN, PA_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
+WORKSPACE_HEADER_BYTES = 256
+
+# Every symbol the public header declares (checked by the CPU test suite).
+EXPORTS = (
+    "pa_paged_attention_partition_size", "pa_paged_attention_workspace_size", "pa_paged_attention",
+    "pa_reshape_and_cache", "pa_copy_blocks", "pa_copy_blocks_check", "pa_get_device_error",
+    "pa_clear_device_error", "pa_status_string",
+)
+
+if not os.path.exists(LIBRARY_PATH):
+    raise ImportError(f"{LIBRARY_PATH} is missing: build it with "
+                      "`python -m pagedattention_paged_kv_attention_b200.build` (no CPU fallback exists)")
+
+lib = ctypes.CDLL(LIBRARY_PATH)
+_p, _i, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+lib.pa_status_string.restype = ctypes.c_char_p
+lib.pa_status_string.argtypes = [_i]
+lib.pa_paged_attention_partition_size.restype = _i
+lib.pa_paged_attention_partition_size.argtypes = [_i, _i, _i, _i, _i]
+lib.pa_paged_attention_workspace_size.restype = _sz
+lib.pa_paged_attention_workspace_size.argtypes = [_i, _i, _i, _i, _i, _i]
+lib.pa_paged_attention.restype = _i
+lib.pa_paged_attention.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i, _f,
+                                   _i, _p, _sz, _p]
+lib.pa_reshape_and_cache.restype = _i
+lib.pa_reshape_and_cache.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _p]
+lib.pa_copy_blocks.restype = _i
+lib.pa_copy_blocks.argtypes = [_p, _p, _i, _p, _i, _i, _i, _i, _i, _p]
+lib.pa_copy_blocks_check.restype = _i
+lib.pa_copy_blocks_check.argtypes = [_p, _i, _i]
+lib.pa_get_device_error.restype = _i
+lib.pa_get_device_error.argtypes = [_p, ctypes.POINTER(ctypes.c_uint), _p]
+lib.pa_clear_device_error.restype = _i
+lib.pa_clear_device_error.argtypes = [_p, _p]
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib.pa_status_string(status).decode()}")
+
+
+def _check(status: int, where: str):
+    if status != PA_OK:
+        raise PagedAttnError(status, where)
+
+
+def dtype_code(t: torch.dtype) -> int:
+    if t == torch.float16:
+        return PA_F16
+    if t == torch.bfloat16:
+        return PA_BF16
+    if t in (torch.uint8, torch.float8_e4m3fn):
+        return PA_FP8_E4M3
+    raise ValueError(f"unsupported dtype {t}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def partition_size(num_seqs, num_heads, num_kv_heads, max_context_len, partition_size=0) -> int:
+    return lib.pa_paged_attention_partition_size(num_seqs, num_heads, num_kv_heads, max_context_len, partition_size)
+
+
+def workspace_size(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, partition_size=0) -> int:
+    return lib.pa_paged_attention_workspace_size(num_seqs, num_heads, num_kv_heads, head_size, max_context_len,
+                                                 partition_size)
+
+
+def make_workspace(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, partition_size=0,
+                   device="cuda") -> torch.Tensor:
+    """A zeroed workspace (error word cleared) sized for these arguments."""
+    n = workspace_size(num_seqs, num_heads, num_kv_heads, head_size, max_context_len, partition_size)
+    if n == 0:
+        raise ValueError("invalid sizes for a workspace")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def paged_attention(out, query, key_cache, value_cache, block_tables, context_lens, scale, max_context_len,
+                    workspace, k_scale=None, v_scale=None, partition_size=0, stream=None):
+    """out[S,H,d] = paged decode attention of query[S,H,d] over key/value_cache[NB,bs,Hkv,d]."""
+    S, H, d = query.shape
+    NB, bs, Hkv, d2 = key_cache.shape
+    st = lib.pa_paged_attention(
+        _ptr(out), _ptr(query), dtype_code(query.dtype), _ptr(key_cache), _ptr(value_cache),
+        dtype_code(key_cache.dtype), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), block_tables.shape[1],
+        _ptr(context_lens), S, H, Hkv, d, bs, NB, int(max_context_len), float(scale), int(partition_size),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "pa_paged_attention")
+    return out
+
+
+def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, k_scale=None, v_scale=None, stream=None):
+    """Write key/value[T,Hkv,d] into the caches at slot_mapping[T] (int64)."""
+    T, Hkv, d = key.shape
+    NB, bs = key_cache.shape[0], key_cache.shape[1]
+    st = lib.pa_reshape_and_cache(_ptr(key), _ptr(value), dtype_code(key.dtype), _ptr(key_cache),
+                                  _ptr(value_cache), dtype_code(key_cache.dtype), _ptr(k_scale), _ptr(v_scale),
+                                  _ptr(slot_mapping), T, Hkv, d, bs, NB, _stream(stream))
+    _check(st, "pa_reshape_and_cache")
+
+
+def copy_blocks(key_cache, value_cache, block_mapping, stream=None):
+    """Copy whole blocks block_mapping[N,2] (src, dst) (int64, device) in both caches."""
+    NB, bs, Hkv, d = key_cache.shape
+    st = lib.pa_copy_blocks(_ptr(key_cache), _ptr(value_cache), dtype_code(key_cache.dtype), _ptr(block_mapping),
+                            block_mapping.shape[0], Hkv, d, bs, NB, _stream(stream))
+    _check(st, "pa_copy_blocks")
+
+
+def copy_blocks_check(block_mapping_host: torch.Tensor, num_blocks: int) -> bool:
+    m = block_mapping_host.to(torch.int64).contiguous().cpu()
+    return lib.pa_copy_blocks_check(_ptr(m), m.shape[0], num_blocks) == PA_OK
+
+
+def get_device_error(workspace, stream=None) -> int:
+    v = ctypes.c_uint(0)
+    _check(lib.pa_get_device_error(_ptr(workspace), ctypes.byref(v), _stream(stream)), "pa_get_device_error")
+    return v.value
+
+
+def clear_device_error(workspace, stream=None):
+    _check(lib.pa_clear_device_error(_ptr(workspace), _stream(stream)), "pa_clear_device_error")

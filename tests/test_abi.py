@@ -1,0 +1,113 @@
+"""The C ABI without a GPU: the library builds, loads, exports every symbol the header declares, plans
+launches as documented, and rejects bad arguments with a status code before any CUDA call (every
+call below would fault or fail if it reached the device, and none needs one)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedattn.h")
+
+
+@pytest.fixture(scope="module")
+def P():
+    from pagedattention_paged_kv_attention_b200 import build
+    build.build()
+    from pagedattention_paged_kv_attention_b200 import pagedattn
+    return pagedattn
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports(P):
+    assert declared_functions() == sorted(P.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(P):
+    lib = ctypes.CDLL(P.LIBRARY_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(P):
+    for code in range(5):
+        assert P.lib.pa_status_string(code)
+    assert P.lib.pa_status_string(99) == b"unknown pa_status"
+
+
+def test_partition_planning(P):
+    assert P.partition_size(8, 32, 8, 32768, 512) == 512
+    assert P.partition_size(8, 32, 8, 32768, 100) == -1           # not a multiple of 64
+    assert P.partition_size(8, 32, 8, 32768, -64) == -1
+    assert P.partition_size(4, 8, 8, 100) >= 100                  # tiny: one partition
+    for args in [(64, 32, 32, 2048), (128, 64, 8, 4096), (256, 32, 8, 1536)]:
+        ps = P.partition_size(*args)
+        assert ps % 64 == 0 and 256 <= ps <= 1024
+
+
+def test_workspace_size(P):
+    S, H, Hkv, d = 8, 32, 8, 128
+    ws = P.workspace_size(S, H, Hkv, d, 32768, 512)
+    parts = 32768 // 512
+    assert ws >= 256 + S * H * parts * (d + 2) * 4
+    assert P.workspace_size(4, 8, 8, 64, 100, 0) == 256           # one partition: header only
+    assert P.workspace_size(4, 8, 3, 64, 100, 0) == 0             # H % Hkv != 0
+
+
+def call_attention(P, **over):
+    args = dict(out=16, query=16, q_dtype=P.PA_BF16, key_cache=16, value_cache=16, kv_dtype=P.PA_BF16, k_scale=None,
+                v_scale=None, block_tables=16, max_blocks_per_seq=4, context_lens=16, num_seqs=2, num_heads=8,
+                num_kv_heads=2, head_size=128, block_size=16, num_blocks=10, max_context_len=64, scale=0.1,
+                partition_size=0, workspace=16, workspace_bytes=1 << 20, stream=None)
+    args.update(over)
+    return P.lib.pa_paged_attention(*args.values())
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(out=None), 1), (dict(query=None), 1), (dict(workspace=None), 1), (dict(block_tables=None), 1),
+    (dict(out=8), 1), (dict(key_cache=24), 1), (dict(num_heads=6, num_kv_heads=4), 1),
+    (dict(num_kv_heads=0), 1), (dict(num_seqs=-1), 1), (dict(max_context_len=-1), 1),
+    (dict(scale=float("nan")), 1), (dict(partition_size=100), 1), (dict(q_dtype=2), 1), (dict(q_dtype=7), 1),
+    (dict(kv_dtype=2), 1),                                                   # FP8 without scales
+    (dict(head_size=96), 2), (dict(block_size=4), 2), (dict(block_size=128), 2),
+    (dict(kv_dtype=0), 2),                                                   # f16 cache with bf16 query
+    (dict(kv_dtype=2, k_scale=16, v_scale=16, head_size=64), 2),
+    (dict(workspace_bytes=255), 3), (dict(max_context_len=4096, partition_size=64, workspace_bytes=1024), 3),
+    (dict(num_seqs=0), 0),                                                   # empty batch: nothing to do
+])
+def test_attention_rejects_bad_arguments_without_cuda(P, over, status):
+    assert call_attention(P, **over) == status
+
+
+def test_reshape_and_copy_reject_bad_arguments(P):
+    L = P.lib
+    ok = dict(key=16, value=16, in_dtype=P.PA_BF16, key_cache=16, value_cache=16, kv_dtype=P.PA_BF16,
+              k_scale=None, v_scale=None, slot_mapping=16, num_tokens=3, num_kv_heads=2, head_size=64,
+              block_size=16, num_blocks=4, stream=None)
+
+    def rc(**over):
+        a = dict(ok)
+        a.update(over)
+        return L.pa_reshape_and_cache(*a.values())
+
+    assert rc(key=None) == 1 and rc(slot_mapping=4) == 1 and rc(num_tokens=-1) == 1
+    assert rc(kv_dtype=P.PA_FP8_E4M3) == 1                 # no scales
+    assert rc(kv_dtype=P.PA_F16) == 2 and rc(head_size=60) == 2
+    assert rc(num_tokens=0) == 0
+    assert L.pa_copy_blocks(16, 16, P.PA_BF16, None, 3, 2, 64, 16, 4, None) == 1
+    assert L.pa_copy_blocks(16, 16, P.PA_BF16, 16, -1, 2, 64, 16, 4, None) == 1
+    assert L.pa_copy_blocks(16, 16, P.PA_BF16, 16, 0, 2, 64, 16, 4, None) == 0
+
+
+def test_copy_blocks_check_on_host_mappings(P):
+    import torch
+    assert P.copy_blocks_check(torch.tensor([[0, 5], [1, 6]]), 8)
+    assert not P.copy_blocks_check(torch.tensor([[0, 5], [1, 5]]), 8)      # duplicate destination
+    assert not P.copy_blocks_check(torch.tensor([[0, 5], [5, 6]]), 8)      # destination is a source
+    assert not P.copy_blocks_check(torch.tensor([[0, 8]]), 8)              # outside the pool
+    assert P.copy_blocks_check(torch.zeros((0, 2), dtype=torch.int64), 8)
