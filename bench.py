@@ -211,12 +211,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="7b", choices=list(W.CONFIGS))
-    ap.add_argument("--partition-size", type=int, default=0)
+    ap.add_argument("--partition-size", type=int, default=None,
+                    help="tokens per split-K partition (default: the workload's, else the library's choice)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     cfg = W.CONFIGS[args.workload]
+    if args.partition_size is None:
+        args.partition_size = cfg.partition_size
     world, rank, local = dist_setup(args)
 
     if args.impl == "reference":
