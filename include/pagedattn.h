@@ -134,6 +134,34 @@ PA_API pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dty
                              void* workspace, size_t workspace_bytes, pa_stream_t stream);
 
 /*
+ * Paged attention without a caller-allocated workspace. The pages have no counterpart: this entry
+ * point exists for callers that cannot call cudaMalloc -- a plugin hosted by an engine that owns all
+ * device memory, or a serving loop that must not allocate (nor pay cudaMalloc's implicit device
+ * synchronisation) once it runs. It computes exactly what pa_paged_attention computes, with the same
+ * arguments and rules, except that its scratch memory is a fixed array inside the library:
+ *  - size: PA_STATIC_WORKSPACE_BYTES, reserved on every GPU that loads the library until the process
+ *    exits; a call whose pa_paged_attention_workspace_size(...) exceeds it returns
+ *    PA_ERR_WORKSPACE_TOO_SMALL without enqueuing anything;
+ *  - set-up: the first call on each device looks up the array's device address on that device (it
+ *    must be the current device); make that first call before any stream capture;
+ *  - sharing: every call on a device uses the same array, which keeps the last call's contents; calls
+ *    that overlap on the GPU (different streams without ordering) race and give undefined results;
+ *  - errors: the device error word lives in the array; when device_error_out (a DEVICE pointer to
+ *    one unsigned int, or NULL) is given, the call copies the word there on `stream` after its
+ *    kernels, then clears it for the next call.
+ * It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ */
+#define PA_STATIC_WORKSPACE_BYTES (32u << 20)
+PA_API pa_status pa_paged_attention_static(void* out, const void* query, pa_dtype q_dtype,
+                                    const void* key_cache, const void* value_cache, pa_dtype kv_dtype,
+                                    const float* k_scale, const float* v_scale,
+                                    const int32_t* block_tables, int max_blocks_per_seq,
+                                    const int32_t* context_lens, int num_seqs, int num_heads,
+                                    int num_kv_heads, int head_size, int block_size, int num_blocks,
+                                    int max_context_len, float scale, int partition_size,
+                                    unsigned int* device_error_out, pa_stream_t stream);
+
+/*
  * Write new tokens into their physical slots ([V] "PagedAttention的破局思路": blocks are filled as the
  * sequence grows). For token i with slot = slot_mapping[i] in [0, num_blocks*block_size):
  *     key_cache[slot / block_size][slot % block_size][h][:] = key[i][h][:]   (same for value)

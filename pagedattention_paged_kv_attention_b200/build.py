@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(HERE, "libpagedattn.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
-SOURCES = ["pa_api.cu", "pa_attention_bf16.cu", "pa_attention_f16.cu"]
+SOURCES = ["pa_api.cu", "pa_attention_bf16.cu", "pa_attention_f16.cu", "pa_static_workspace.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

@@ -23,7 +23,7 @@ WORKSPACE_HEADER_BYTES = 256
 EXPORTS = (
     "pa_paged_attention_partition_size", "pa_paged_attention_workspace_size", "pa_paged_attention",
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_copy_blocks_check", "pa_get_device_error",
-    "pa_clear_device_error", "pa_status_string",
+    "pa_clear_device_error", "pa_status_string", "pa_paged_attention_static",
 )
 
 if not os.path.exists(LIBRARY_PATH):
@@ -41,6 +41,9 @@ lib.pa_paged_attention_workspace_size.argtypes = [_i, _i, _i, _i, _i, _i]
 lib.pa_paged_attention.restype = _i
 lib.pa_paged_attention.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i, _f,
                                    _i, _p, _sz, _p]
+lib.pa_paged_attention_static.restype = _i
+lib.pa_paged_attention_static.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i,
+                                          _f, _i, _p, _p]
 lib.pa_reshape_and_cache.restype = _i
 lib.pa_reshape_and_cache.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 lib.pa_copy_blocks.restype = _i
@@ -113,6 +116,23 @@ def paged_attention(out, query, key_cache, value_cache, block_tables, context_le
         _ptr(context_lens), S, H, Hkv, d, bs, NB, int(max_context_len), float(scale), int(partition_size),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "pa_paged_attention")
+    return out
+
+
+def paged_attention_static(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                           max_context_len, k_scale=None, v_scale=None, partition_size=0, device_error_out=None,
+                           stream=None):
+    """paged_attention with the library's fixed scratch array instead of a caller workspace (for
+    callers that cannot allocate device memory). device_error_out: optional int32/uint32 device
+    tensor of one element that receives the device error word."""
+    S, H, d = query.shape
+    NB, bs, Hkv, d2 = key_cache.shape
+    st = lib.pa_paged_attention_static(
+        _ptr(out), _ptr(query), dtype_code(query.dtype), _ptr(key_cache), _ptr(value_cache),
+        dtype_code(key_cache.dtype), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), block_tables.shape[1],
+        _ptr(context_lens), S, H, Hkv, d, bs, NB, int(max_context_len), float(scale), int(partition_size),
+        _ptr(device_error_out), _stream(stream))
+    _check(st, "pa_paged_attention_static")
     return out
 
 
