@@ -22,8 +22,7 @@
 namespace {
 
 constexpr int kPlanSMs = 148;            // B200 SM count; planning is a pure function of the sizes
-constexpr int kPlanCtasPerSm = 2;
-constexpr int kPlanWaves = 8;
+constexpr int kPlanItemsPerCta = 16;     // work items per persistent CTA the automatic plan aims for
 constexpr int kMinAutoPartition = 256;
 constexpr int kMaxAutoPartition = 1024;
 
@@ -41,16 +40,17 @@ void group_tiling(int group, int* g_tile, int* subgroups) {
 
 int plan_partition(int num_seqs, int num_heads, int num_kv_heads, int max_context_len, int partition_size) {
   if (partition_size < 0) return -1;
-  if (partition_size > 0) return (partition_size % pa::kStageTokens == 0) ? partition_size : -1;
+  if (partition_size > 0) return (partition_size % pa::kPartitionQuantum == 0) ? partition_size : -1;
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads || max_context_len < 0)
     return -1;
   int g_tile, subgroups;
   group_tiling(num_heads / num_kv_heads, &g_tile, &subgroups);
-  const long items = std::max<long>(1, static_cast<long>(num_seqs) * num_kv_heads * subgroups);
-  const long target = static_cast<long>(kPlanSMs) * kPlanCtasPerSm * kPlanWaves;
+  const long items =
+      std::max<long>(1, static_cast<long>(num_seqs) * ceil_div(num_kv_heads, pa::kHeadBlock) * subgroups);
+  const long target = static_cast<long>(kPlanSMs) * kPlanItemsPerCta;
   const long splits = std::max<long>(1, (target + items - 1) / items);
   long ps = (std::max(1, max_context_len) + splits - 1) / splits;
-  ps = round_up(static_cast<size_t>(ps), pa::kStageTokens);
+  ps = round_up(static_cast<size_t>(ps), pa::kPartitionQuantum);
   ps = std::min<long>(std::max<long>(ps, kMinAutoPartition), kMaxAutoPartition);
   return static_cast<int>(ps);
 }
@@ -86,7 +86,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // 4-D view {head_size, num_kv_heads, block_size, num_blocks} of a cache; box = one 128-byte chunk of
-// `block_size` rows of one kv head of one block, written to shared memory with the 128-byte swizzle.
+// the rows of 8 consecutive kv heads for 8 consecutive tokens of one block (heads past the last one
+// read as zeros), written to shared memory with the 128-byte swizzle.
 bool encode_cache_map(CUtensorMap* map, const void* cache, int elem_bytes, int head_size, int num_kv_heads,
                       int block_size, int num_blocks) {
   auto encode = tensor_map_encoder();
@@ -95,7 +96,8 @@ bool encode_cache_map(CUtensorMap* map, const void* cache, int elem_bytes, int h
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_size), static_cast<cuuint64_t>(num_kv_heads),
                         static_cast<cuuint64_t>(block_size), static_cast<cuuint64_t>(num_blocks)};
   cuuint64_t strides[3] = {head_size * e, num_kv_heads * head_size * e, block_size * num_kv_heads * head_size * e};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), 1, static_cast<cuuint32_t>(block_size), 1};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(pa::kHeadBlock),
+                       static_cast<cuuint32_t>(pa::kStageTokens), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = encode(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
                       const_cast<void*>(cache), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -168,8 +170,10 @@ pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dtype, con
   const int partitions = std::max(1, ceil_div(max_context_len, ps));
   int g_tile, subgroups;
   group_tiling(num_heads / num_kv_heads, &g_tile, &subgroups);
-  if (num_seqs > 65535 || partitions > 65535 || static_cast<long>(num_kv_heads) * subgroups > 0x7fffffffL)
-    return PA_ERR_UNSUPPORTED;
+  const int head_blocks = ceil_div(num_kv_heads, pa::kHeadBlock);
+  const unsigned long long items =
+      static_cast<unsigned long long>(partitions) * num_seqs * head_blocks * subgroups;
+  if (num_seqs > 65535 || items > 0x7fffffffULL) return PA_ERR_UNSUPPORTED;
   const WorkspaceLayout ws = workspace_layout(num_seqs, num_heads, head_size, partitions);
   if (workspace_bytes < ws.total) return PA_ERR_WORKSPACE_TOO_SMALL;
 
@@ -178,6 +182,10 @@ pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dtype, con
   const int eb = elem_bytes(kv_dtype);
   if (!encode_cache_map(&tk, key_cache, eb, head_size, num_kv_heads, block_size, num_blocks) ||
       !encode_cache_map(&tv, value_cache, eb, head_size, num_kv_heads, block_size, num_blocks))
+    return PA_ERR_CUDA;
+  int device = 0, sms = 0;
+  if (cudaGetDevice(&device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms <= 0)
     return PA_ERR_CUDA;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   pa::AttnArgs a{};
@@ -190,20 +198,21 @@ pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dtype, con
   a.part_m = partitions > 1 ? reinterpret_cast<float*>(wsb + ws.part_m) : nullptr;
   a.part_l = partitions > 1 ? reinterpret_cast<float*>(wsb + ws.part_l) : nullptr;
   a.part_o = partitions > 1 ? reinterpret_cast<float*>(wsb + ws.part_o) : nullptr;
-  a.error_word = reinterpret_cast<unsigned int*>(wsb);
+  a.header = reinterpret_cast<unsigned int*>(wsb);
   a.max_blocks_per_seq = max_blocks_per_seq;
   a.num_seqs = num_seqs;
   a.num_heads = num_heads;
   a.num_kv_heads = num_kv_heads;
   a.group = num_heads / num_kv_heads;
   a.subgroups = subgroups;
+  a.head_blocks = head_blocks;
   a.block_size = block_size;
   a.num_blocks = num_blocks;
   a.partition_size = ps;
   a.num_partitions = partitions;
+  a.num_items = static_cast<unsigned int>(items);
   a.scale_log2 = scale * pa::kLog2e;
-  const dim3 grid(static_cast<unsigned>(num_kv_heads * subgroups), static_cast<unsigned>(num_seqs),
-                  static_cast<unsigned>(partitions));
+  const int grid = static_cast<int>(std::min<unsigned long long>(static_cast<unsigned long long>(sms), items));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = q_dtype == PA_BF16 ? pa::launch_attention_bf16(tk, tv, a, fp8, head_size, g_tile, grid, st)
                                      : pa::launch_attention_f16(tk, tv, a, fp8, head_size, g_tile, grid, st);
@@ -302,7 +311,7 @@ pa_status pa_get_device_error(const void* workspace, unsigned int* err_out, pa_s
 pa_status pa_clear_device_error(void* workspace, pa_stream_t stream) {
   if (!workspace || !aligned(workspace, 16)) return PA_ERR_INVALID_ARGUMENT;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return cudaMemsetAsync(workspace, 0, sizeof(unsigned int), st) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return cudaMemsetAsync(workspace, 0, PA_WORKSPACE_HEADER_BYTES, st) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // extern "C"

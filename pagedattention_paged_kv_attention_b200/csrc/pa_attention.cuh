@@ -7,37 +7,59 @@
 // where token t is found through the block table (sec. 2.1 "基本数据结构设计"; page "PagedAttention 与
 // 连续批处理：LLM Serving 的底层架构拆解", section "PagedAttention：把显存做成虚拟内存").
 //
-// Design (B200): one CTA per (kv head [x head sub-group], sequence, context partition).
-//  * Warp 4 is a producer: for each 64-token stage it reads the stage's block ids from the block
-//    table and issues one 4-D TMA tile load per (block, 128-byte chunk) for K and for V into a ring of
-//    shared-memory stages (128-byte swizzle), completion counted on an mbarrier. The page-table walk
-//    is therefore a TMA coordinate, and the bytes in flight per SM are the ring depth.
-//  * Warps 0-3 are consumers. Warp w owns stages w, w+4, ... and keeps its own fp32 online-softmax
-//    state (running max m, running sum l, accumulator acc[G][d]) for the G query heads that share
-//    this kv head (grouped-query heads are batched: each K/V element is read once for all G heads).
-//      QK: NS lanes cooperate on one token (each holds 1/NS of d and all G query rows in registers,
-//          pre-scaled by scale*log2(e)); a butterfly reduce-scatter leaves each lane with the full
-//          score of one head.
-//      softmax: stage max per head across lanes, rescale factor alpha = 2^(m_old - m_new),
-//          p = 2^(z - m_new) written to a per-warp shared buffer.
+// Design (B200). Decode reads every K/V byte once; the kernel is shaped so that HBM sees long
+// contiguous reads and stays busy:
+//  * A work item is (context partition, sequence, block of 8 kv heads [, query-head subgroup]).
+//    Because a cache block is laid out [token][kv head][d], the 8 heads of one token are contiguous,
+//    and for an 8-kv-head cache a whole block is one contiguous run.
+//  * Persistent CTAs, one per SM, take items from an atomic counter in the workspace header in
+//    partition-major order (every sequence's first partition before any second one); the last CTA to
+//    finish resets the counter.
+//  * Warp 0 is the producer. Per item it bulk-copies the query rows of the 8 heads into shared memory;
+//    then, for each 8-token stage, it reads one block-table entry (prefetched a window at a time) and
+//    issues 4-D TMA tile loads {128-byte chunk, 8 kv heads, 8 tokens, 1 block} of K and V (128-byte
+//    swizzle) into a shared-memory ring whose slots are guarded by mbarriers, with a small message
+//    (item, valid tokens, first/last stage). The page-table walk is a TMA coordinate.
+//  * Warps 1..8 are consumers; warp w owns kv head w of the block for the whole item and keeps an fp32
+//    online-softmax state (running max m, running sum l, accumulator acc[G][d]) for the G query heads
+//    of that kv head (grouped-query heads are batched: each K/V element is read once for all G heads).
+//      QK: NS >= 8 lanes cooperate on one token (each holds 1/NS of d and the G query rows in
+//          registers, pre-scaled by scale*log2(e)); a butterfly reduce-scatter leaves each lane with
+//          the full score of one head. Lanes of a shared-memory phase read distinct 16-byte units of
+//          one row, so the swizzled rows are read without bank conflicts.
+//      softmax: stage max per head across lanes, rescale alpha = 2^(m_old - m_new), p = 2^(z - m_new)
+//          through a per-warp shared buffer.
 //      PV: D/8 lanes cover one V row (8 elements each); every lane accumulates all G heads.
-//    Packed f32x2 FMAs are used throughout; inputs are widened to fp32 once per element.
-//  * At the end the four warp states are merged through shared memory (log-sum-exp merge). With one
-//    partition the CTA writes the normalised output; otherwise it writes (m, l, acc/l) partials and
-//    the reduce kernel merges partitions the same way.
-// Arithmetic order depends only on logical token positions, never on physical block ids, so outputs
-// are bitwise invariant to block placement and deterministic run to run.
+//    Packed f32x2 FMAs are used throughout; inputs are widened to fp32 once per element. At the end of
+//    an item each warp writes its heads' normalised output, or (m, l, acc/l) partials that the reduce
+//    kernel merges across partitions (log-sum-exp merge).
+// Arithmetic order depends only on logical token positions, never on physical block ids or on which
+// CTA handled an item, so outputs are bitwise invariant to block placement and deterministic.
 #pragma once
 
 #include "pa_device.cuh"
 
 namespace pa {
 
-constexpr int kStageTokens = 64;
-constexpr int kConsumerWarps = 4;
+constexpr int kHeadBlock = 8;            // kv heads per work item (one consumer warp each)
+constexpr int kConsumerWarps = kHeadBlock;
+constexpr int kStageTokens = 8;          // tokens per pipeline stage (block_size >= 8)
+constexpr int kStages = 4;               // ring depth
+constexpr int kQueryBuffers = 2;
+constexpr int kIdWindow = 4;             // block ids prefetched per item: 32 * kIdWindow stages
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kMaxStages = 8;
+constexpr int kPartitionQuantum = 64;    // partition sizes are multiples of this
 constexpr float kLog2e = 1.4426950408889634f;
+
+// Workspace header words: error bits, work counter, finished-CTA counter.
+constexpr int kWsError = 0;
+constexpr int kWsWork = 1;
+constexpr int kWsDone = 2;
+
+// Stage message flags.
+constexpr int kMsgFirst = 1;
+constexpr int kMsgLast = 2;
+constexpr int kMsgBadBlock = 4;
 
 struct AttnArgs {
   void* out;                    // [S][H][D] query dtype
@@ -49,23 +71,25 @@ struct AttnArgs {
   float* part_m;                // [S][H][P]
   float* part_l;                // [S][H][P]
   float* part_o;                // [S][H][P][D]
-  unsigned int* error_word;
+  unsigned int* header;         // workspace header: [0] error bits, [1] work counter, [2] done counter
   int max_blocks_per_seq;
   int num_seqs;
   int num_heads;
   int num_kv_heads;
+  int head_blocks;              // ceil(num_kv_heads / kHeadBlock)
   int group;                    // num_heads / num_kv_heads
-  int subgroups;                // CTAs per kv head (ceil(group / G))
+  int subgroups;                // query-head subgroups per kv head (ceil(group / G))
   int block_size;
   int num_blocks;
-  int partition_size;           // tokens per partition, multiple of kStageTokens
+  int partition_size;           // tokens per partition, multiple of kPartitionQuantum
   int num_partitions;
-  int num_stages;               // ring depth, 2..kMaxStages
+  unsigned int num_items;       // num_partitions * num_seqs * head_blocks * subgroups
   float scale_log2;             // softmax scale * log2(e)
 };
 
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
 template <int D, int G, int EB>
 struct Shape {
@@ -74,58 +98,88 @@ struct Shape {
   static constexpr int kChunkElems = 128 / EB;
   static constexpr int kPieceBytes = 8 * EB;             // one piece = 8 elements
   static constexpr int kPiecesPerRow = D / 8;
-  // QK mapping: NS lanes per token.
-  static constexpr int kNS = cmin(D / 8, G <= 2 ? 4 : 2 * G);
+  // QK mapping: NS lanes per token, NS >= 8 so that a phase reads distinct units of one row.
+  static constexpr int kNS = cmin(D / 8, cmax(8, 2 * G));
   static constexpr int kLog2NS = ilog2(kNS);
   static constexpr int kLog2G = ilog2(G);
   static constexpr int kTPI = 32 / kNS;                  // tokens per QK step
-  static constexpr int kLog2TPI = ilog2(kTPI);
   static constexpr int kNPL = kPiecesPerRow / kNS;       // pieces per lane
   static constexpr int kIters = kStageTokens / kTPI;
-  static constexpr bool kDsFastest = kNS >= 8;
-  static constexpr int kDsShift = kDsFastest ? 0 : kLog2TPI;
-  static constexpr int kTsShift = kDsFastest ? kLog2NS : 0;
+  static constexpr int kTsShift = kLog2NS;               // token-slot lane bits sit above the ds bits
   // PV mapping: LPT lanes per token.
   static constexpr int kLPT = D / 8;
   static constexpr int kLog2LPT = ilog2(kLPT);
   static constexpr int kTPV = 32 / kLPT;
-  static constexpr int kTileBytes = kStageTokens * kRowBytes;
+  // One stage: [K|V][chunk][token][head][128 B].
+  static constexpr int kChunkBytes = kStageTokens * kHeadBlock * 128;
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
   static constexpr int kStageBytes = 2 * kTileBytes;
   static_assert(kRowBytes == 128 || kRowBytes == 256, "row must be 128 or 256 bytes");
-  static_assert(G <= kNS, "group larger than the lanes of a token");
+  static_assert(kNS >= 8 && G <= kNS, "lane mapping");
   static_assert(kNPL >= 1 && kNPL * kNS == kPiecesPerRow, "pieces must split evenly");
+  static_assert(kIters >= 1, "stage shorter than one QK step");
 };
 
-// Byte offset of piece `pc` (8 elements) of token row `t` inside a [chunk][64 tokens][128 B] tile
-// written by TMA with the 128-byte swizzle (16-byte unit u of row t lives at unit u ^ (t & 7)).
+struct StageMsg {
+  int item;    // CTA-local item sequence number, -1 = no more work
+  int ntok;    // valid tokens in the stage
+  int flags;   // kMsgFirst | kMsgLast | kMsgBadBlock
+  int pad;
+};
+
+struct ItemInfo {
+  int s, part, kvh0, h_sub, heads, write_final, pad0, pad1;  // h_sub: first query-head offset in a group
+};
+
+// Shared-memory layout (byte offsets from the 1024-aligned base).
+template <typename QT, int D, int G, int EB>
+struct Layout {
+  using S = Shape<D, G, EB>;
+  static constexpr int kRing = 0;
+  static constexpr int kRingBytes = kStages * S::kStageBytes;
+  static constexpr int kQueryOne = kHeadBlock * G * D * int(sizeof(QT));       // [8 kv heads][G][D]
+  static constexpr int kQuery = kRingBytes;
+  static constexpr int kPbuf = kQuery + kQueryBuffers * kQueryOne;             // [W][TS][G] f32
+  static constexpr int kAbuf = kPbuf + kConsumerWarps * kStageTokens * G * 4;  // [W][G] f32
+  static constexpr int kMsgs = (kAbuf + kConsumerWarps * G * 4 + 15) / 16 * 16;
+  static constexpr int kInfo = kMsgs + kStages * int(sizeof(StageMsg));
+  static constexpr int kBars = (kInfo + kQueryBuffers * int(sizeof(ItemInfo)) + 7) / 8 * 8;
+  // full[kStages], empty[kStages], qfull[NQ], qempty[NQ]
+  static constexpr int kNumBars = 2 * kStages + 2 * kQueryBuffers;
+  static constexpr int kEnd = kBars + kNumBars * 8;
+  static constexpr int kAllocBytes = kEnd + 1024;  // alignment slack
+  static_assert(kAllocBytes <= 227 * 1024, "shared memory layout too large");
+};
+
+// Byte offset of piece `pc` (8 elements) of tile row r = token * 8 + head inside a
+// [chunk][kStageTokens * 8 rows][128 B] tile written by TMA with the 128-byte swizzle (16-byte unit u
+// of row r lives at unit u ^ (r & 7) = u ^ head).
 template <class S>
-__device__ __forceinline__ uint32_t piece_offset(int t, int pc) {
+__device__ __forceinline__ uint32_t piece_offset(int r, int pc) {
   const int byte = pc * S::kPieceBytes;
   const int c = byte >> 7;
   const int b = byte & 127;
-  return static_cast<uint32_t>(c * (kStageTokens * 128) + t * 128 + ((((b >> 4) ^ (t & 7)) << 4) | (b & 15)));
+  return static_cast<uint32_t>(c * S::kChunkBytes + r * 128 + ((((b >> 4) ^ (r & 7)) << 4) | (b & 15)));
 }
 
 // Piece read by a lane in QK step j. FP8 rows with 8 lanes per token alternate halves by token
-// parity so that two tokens sharing a half-warp hit disjoint banks.
+// parity so that two tokens sharing a half-warp phase hit disjoint banks.
 template <class S, int EB>
 __device__ __forceinline__ int qk_piece(int j, int ds, int tslot) {
   if constexpr (EB == 1 && S::kNS == 8 && S::kNPL == 2) return ds + 8 * (j ^ (tslot & 1));
   return ds + S::kNS * j;
 }
 
-template <int G, int NS_LOG2, int DS_SHIFT>
+template <int G, int NS_LOG2>
 __device__ __forceinline__ float reduce_scatter(float (&v)[G], int lane) {
-  // Halving exchange over the ds lane bits, high bit first: after log2(G) halvings each lane holds
-  // one head's partial sum over its lane pair group; the remaining bits finish a full reduction.
+  // Halving exchange over the ds lane bits (the low NS_LOG2 bits), high bit first: after log2(G)
+  // halvings each lane holds one head's partial sum; the remaining bits finish a full reduction.
   constexpr int kLog2G = ilog2(G);
 #pragma unroll
   for (int step = 0; step < NS_LOG2; ++step) {
-    const int bit = NS_LOG2 - 1 - step;
-    const int mask = 1 << (bit + DS_SHIFT);
+    const int mask = 1 << (NS_LOG2 - 1 - step);
     if (step < kLog2G) {
-      const int n = G >> step;
-      const int half = n >> 1;
+      const int half = (G >> step) >> 1;
       const bool upper = (lane & mask) != 0;
 #pragma unroll
       for (int i = 0; i < G / 2; ++i) {
@@ -148,331 +202,423 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// CTAs per SM the kernel is compiled for (registers are not capped below what the G query rows and
-// accumulators need).
-template <int G>
-constexpr int min_ctas_per_sm() { return 1; }
+// Item index -> (partition, sequence, head block, query-head subgroup). Partition-major.
+struct ItemCoord {
+  int part, s, hb, sub;
+};
+__device__ __forceinline__ ItemCoord decode_item(unsigned int idx, const AttnArgs& a) {
+  const unsigned int per_seq = static_cast<unsigned int>(a.head_blocks) * a.subgroups;
+  const unsigned int per_part = static_cast<unsigned int>(a.num_seqs) * per_seq;
+  ItemCoord c;
+  c.part = static_cast<int>(idx / per_part);
+  unsigned int r = idx - static_cast<unsigned int>(c.part) * per_part;
+  c.s = static_cast<int>(r / per_seq);
+  r -= static_cast<unsigned int>(c.s) * per_seq;
+  c.hb = static_cast<int>(r / a.subgroups);
+  c.sub = static_cast<int>(r - static_cast<unsigned int>(c.hb) * a.subgroups);
+  return c;
+}
+
+__device__ __forceinline__ bool context_len_invalid(int L, const AttnArgs& a) {
+  return L < 0 || L > a.max_blocks_per_seq * a.block_size || L > a.num_partitions * a.partition_size;
+}
 
 template <typename QT, typename KVT, int D, int G>
-__global__ void __launch_bounds__(kThreads, min_ctas_per_sm<G>())
+__global__ void __launch_bounds__(kThreads, 1)
 paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                      const AttnArgs args) {
   constexpr int EB = Elem<KVT>::kBytes;
   using S = Shape<D, G, EB>;
+  using Lay = Layout<QT, D, G, EB>;
   using Piece = typename Elem<KVT>::Piece;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int kvh = blockIdx.x / args.subgroups;
-  const int sub = blockIdx.x - kvh * args.subgroups;
-  const int h0 = kvh * args.group + sub * G;
-  const int heads_here = cmin(G, args.group - sub * G);
-  const int s = blockIdx.y;
-  const int part = blockIdx.z;
-  const int PS = args.partition_size;
+  unsigned int* err = args.header + kWsError;
 
-  const int L = args.context_lens[s];
-  const bool bad_len = L < 0 || L > args.max_blocks_per_seq * args.block_size ||
-                       L > args.num_partitions * PS;
-  const int n_parts = bad_len ? 1 : (L + PS - 1) / PS;
-  if (part >= (n_parts > 0 ? n_parts : 1)) return;  // whole CTA leaves: partition past the context
-  const bool write_final = n_parts <= 1;
-
-  if (L == 0 || bad_len) {
-    // Empty context -> zeros; a context the launch cannot cover -> NaN and an error bit.
-    if (bad_len && threadIdx.x == 0) atomicOr(args.error_word, PA_DEVERR_CONTEXT_LEN);
-    const float fill = bad_len ? __int_as_float(0x7fc00000) : 0.0f;
-    QT* out = static_cast<QT*>(args.out);
-    for (int i = threadIdx.x; i < heads_here * D; i += kThreads) {
-      const int g = i / D;
-      out[(static_cast<size_t>(s) * args.num_heads + h0 + g) * D + (i - g * D)] = QT(fill);
-    }
-    return;
-  }
-
-  const int tok_begin = part * PS;
-  const int tok_end = cmin(L, tok_begin + PS);
-  const int n_stages = (tok_end - tok_begin + kStageTokens - 1) / kStageTokens;
-  const int NST = args.num_stages;
-
-  // Shared memory: [stage ring][P buffers][alpha buffers][mbarriers][flags], 1024-aligned ring.
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* pbuf = reinterpret_cast<float*>(smem + NST * S::kStageBytes);           // [W][64][G]
-  float* abuf = pbuf + kConsumerWarps * kStageTokens * G;                         // [W][G]
-  uint64_t* full = reinterpret_cast<uint64_t*>(abuf + kConsumerWarps * G + ((kConsumerWarps * G) & 1));
-  uint64_t* empty = full + NST;
-  int* flags = reinterpret_cast<int*>(empty + NST);                               // [0]: bad block
+  StageMsg* msgs = reinterpret_cast<StageMsg*>(smem + Lay::kMsgs);
+  ItemInfo* infos = reinterpret_cast<ItemInfo*>(smem + Lay::kInfo);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBars);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages;
+  uint64_t* qfull = bars + 2 * kStages;
+  uint64_t* qempty = qfull + kQueryBuffers;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NST; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&empty[i], kConsumerWarps);
     }
-    flags[0] = 0;
+    for (int i = 0; i < kQueryBuffers; ++i) {
+      mbar_init(&qfull[i], 1);
+      mbar_init(&qempty[i], kConsumerWarps);
+    }
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == kConsumerWarps) {
-    // ------------------------------- producer warp -------------------------------
+  if (warp == 0) {
+    // =============================== producer warp ===============================
     if (lane == 0) {
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_v);
     }
     const int bs = args.block_size;
-    const int32_t* table = args.block_tables + static_cast<size_t>(s) * args.max_blocks_per_seq;
-    auto stage_block_id = [&](int j) -> int {
-      const int t0 = tok_begin + j * kStageTokens;
-      const int nb = (cmin(kStageTokens, tok_end - t0) + bs - 1) / bs;
-      return lane < nb ? __ldg(table + t0 / bs + lane) : 0;
-    };
-    bool bad_block = false;
-    int issued = 0;
-    int id_next = n_stages > 0 ? stage_block_id(0) : 0;
-    for (int j = 0; j < n_stages; ++j) {
-      const int id = id_next;
-      if (j + 1 < n_stages) id_next = stage_block_id(j + 1);  // next stage's ids load during the wait
-      const int slot = j % NST;
-      const uint32_t round = static_cast<uint32_t>(j / NST);
-      bool ok = true;
-      if (lane == 0) ok = mbar_wait(&empty[slot], (round & 1u) ^ 1u, args.error_word);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      const int t0 = tok_begin + j * kStageTokens;
-      const int nb = (cmin(kStageTokens, tok_end - t0) + bs - 1) / bs;
-      uint8_t* ktile = smem + slot * S::kStageBytes;
-      uint8_t* vtile = ktile + S::kTileBytes;
-      if (lane == 0) mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nb * bs * S::kRowBytes * 2));
-      for (int i = 0; i < nb; ++i) {
-        int blk = __shfl_sync(0xffffffffu, id, i);
-        if (lane == 0) {
-          if (blk < 0 || blk >= args.num_blocks) {
-            bad_block = true;
-            blk = args.num_blocks;  // out-of-range coordinate: TMA fills the box with zeros
-          }
-#pragma unroll
-          for (int c = 0; c < S::kChunks; ++c) {
-            const int dst = c * (kStageTokens * 128) + i * bs * 128;
-            tma_load_4d(ktile + dst, &tmap_k, &full[slot], c * S::kChunkElems, kvh, 0, blk);
-            tma_load_4d(vtile + dst, &tmap_v, &full[slot], c * S::kChunkElems, kvh, 0, blk);
-          }
-        }
-      }
-      issued = j + 1;
-    }
-    bad_block = __any_sync(0xffffffffu, bad_block);
-    if (bad_block && lane == 0) {
-      atomicOr(args.error_word, PA_DEVERR_BLOCK_ID);
-      flags[0] = 1;
-    }
-    // Drain: every issued stage's bytes have landed before the ring memory is reused or the CTA ends.
-    if (lane == 0)
-      for (int j = (issued > NST ? issued - NST : 0); j < issued; ++j)
-        mbar_wait(&full[j % NST], static_cast<uint32_t>(j / NST) & 1u, args.error_word);
-    __syncwarp();
-    named_barrier(1, kThreads);
-    return;
-  }
+    const int stages_per_part = args.partition_size / kStageTokens;
+    bool aborted = false;
+    int local = 0;   // CTA-local item sequence number
+    int issued = 0;  // stages issued so far (ring position)
 
-  // ------------------------------- consumer warps -------------------------------
-  // QK lane roles.
-  const int ds = S::kDsFastest ? (lane & (S::kNS - 1)) : (lane >> S::kLog2TPI);
-  const int tslot = S::kDsFastest ? (lane >> S::kLog2NS) : (lane & (S::kTPI - 1));
-  const int g_lane = ds >> (S::kLog2NS - S::kLog2G);                 // head owned after reduce-scatter
-  const bool primary = (ds & ((S::kNS >> S::kLog2G) - 1)) == 0;      // first of the duplicate lanes
-  // PV lane roles.
-  const int dp = lane & (S::kLPT - 1);
-  const int vslot = lane >> S::kLog2LPT;
+    // Items flow through a two-deep software pipeline: while item i streams, the loads describing item
+    // i+1 (its context length and a window of its block ids, one id per lane per 32 stages) are in
+    // flight, and the work counter has already been asked for item i+2. All state is in registers.
+    unsigned int cur_idx = 0, nxt_idx = 0;
+    int cur_L = 0, nxt_L = 0;
+    int cur_ids[kIdWindow], nxt_ids[kIdWindow];
+#define PA_PREPARE(IDX, LV, IDS)                                                                       \
+  do {                                                                                                 \
+    if ((IDX) < args.num_items) {                                                                      \
+      const ItemCoord pc_ = decode_item((IDX), args);                                                  \
+      LV = __ldg(args.context_lens + pc_.s);                                                           \
+      const int32_t* row_ = args.block_tables + static_cast<size_t>(pc_.s) * args.max_blocks_per_seq;  \
+      _Pragma("unroll") for (int j_ = 0; j_ < kIdWindow; ++j_) {                                       \
+        const int entry_ = ((pc_.part * stages_per_part + j_ * 32 + lane) * kStageTokens) / bs;        \
+        IDS[j_] = entry_ < args.max_blocks_per_seq ? __ldg(row_ + entry_) : 0;                         \
+      }                                                                                                \
+    }                                                                                                  \
+  } while (0)
 
-  // Query rows in registers, pre-scaled (scale * log2 e, times k_scale for FP8 caches).
-  float qscale = args.scale_log2;
-  if constexpr (EB == 1) qscale *= args.k_scale[kvh];
-  float2 qr[G][S::kNPL][4];
-  {
-    const QT* q = static_cast<const QT*>(args.query) + (static_cast<size_t>(s) * args.num_heads + h0) * D;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-#pragma unroll
-      for (int j = 0; j < S::kNPL; ++j) {
-        const int pc = qk_piece<S, EB>(j, ds, tslot);
-        if (g < heads_here) {
-          const uint4 raw = __ldg(reinterpret_cast<const uint4*>(q + static_cast<size_t>(g) * D + pc * 8));
-          const QT* e = reinterpret_cast<const QT*>(&raw);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            qr[g][j][k] = make_float2(to_f32(e[2 * k]) * qscale, to_f32(e[2 * k + 1]) * qscale);
+    unsigned int ticket = 0;
+    if (lane == 0) ticket = atomicAdd(args.header + kWsWork, 1u);
+    cur_idx = __shfl_sync(0xffffffffu, ticket, 0);
+    PA_PREPARE(cur_idx, cur_L, cur_ids);
+    if (lane == 0) ticket = atomicAdd(args.header + kWsWork, 1u);
+    while (!aborted && cur_idx < args.num_items) {
+      nxt_idx = __shfl_sync(0xffffffffu, ticket, 0);
+      PA_PREPARE(nxt_idx, nxt_L, nxt_ids);
+      if (lane == 0) ticket = atomicAdd(args.header + kWsWork, 1u);
+      const ItemCoord c = decode_item(cur_idx, args);
+      const int L = cur_L;
+      const bool bad_len = context_len_invalid(L, args);
+      const int n_parts = bad_len ? 1 : (L + args.partition_size - 1) / args.partition_size;
+      const int kvh0 = c.hb * kHeadBlock;
+      const int kv_here = cmin(kHeadBlock, args.num_kv_heads - kvh0);
+      const int h_sub = c.sub * G;                       // first query head of the subgroup in a group
+      const int heads = cmin(G, args.group - h_sub);     // query heads per kv head in this item
+      if (c.part < cmax(n_parts, 1)) {
+        if (L == 0 || bad_len) {
+          // Empty context -> zeros; a context the launch cannot cover -> NaN and an error bit.
+          if (bad_len && lane == 0) atomicOr(err, PA_DEVERR_CONTEXT_LEN);
+          const float fill = bad_len ? __int_as_float(0x7fc00000) : 0.0f;
+          for (int i = lane; i < kv_here * heads * D; i += 32) {
+            const int kv = i / (heads * D), g = (i / D) % heads, e = i % D;
+            const size_t h = static_cast<size_t>(kvh0 + kv) * args.group + h_sub + g;
+            static_cast<QT*>(args.out)[(static_cast<size_t>(c.s) * args.num_heads + h) * D + e] = QT(fill);
+          }
         } else {
+          const int tok_begin = c.part * args.partition_size;
+          const int tok_end = cmin(L, tok_begin + args.partition_size);
+          const int n_stages = (tok_end - tok_begin + kStageTokens - 1) / kStageTokens;
+          const int qb = local % kQueryBuffers;
+          // Query rows of the item's heads, and the item description.
+          bool ok = true;
+          if (lane == 0) ok = mbar_wait(&qempty[qb], (static_cast<uint32_t>(local / kQueryBuffers) & 1u) ^ 1u, err);
+          if (!__shfl_sync(0xffffffffu, ok, 0)) {
+            aborted = true;
+            break;
+          }
+          const uint32_t row_bytes = static_cast<uint32_t>(heads * D * sizeof(QT));
+          if (lane == 0) {
+            ItemInfo inf;
+            inf.s = c.s;
+            inf.part = c.part;
+            inf.kvh0 = kvh0;
+            inf.h_sub = h_sub;
+            inf.heads = heads;
+            inf.write_final = n_parts <= 1;
+            inf.pad0 = inf.pad1 = 0;
+            infos[qb] = inf;
+            mbar_arrive_expect_tx(&qfull[qb], row_bytes * kv_here);
+          }
+          __syncwarp();
+          if (lane < kv_here) {
+            const QT* qsrc = static_cast<const QT*>(args.query) +
+                             (static_cast<size_t>(c.s) * args.num_heads + (kvh0 + lane) * args.group + h_sub) * D;
+            bulk_copy_g2s(smem + Lay::kQuery + qb * Lay::kQueryOne + lane * G * D * sizeof(QT), qsrc, row_bytes,
+                          &qfull[qb]);
+          }
+
+          const int32_t* row = args.block_tables + static_cast<size_t>(c.s) * args.max_blocks_per_seq;
+          // TMA ops of one stage are spread over lanes: lane = kv * kChunks + chunk.
+          const int op_kv = lane / S::kChunks;
+          const int op_ch = lane % S::kChunks;
+          for (int k = 0; k < n_stages; ++k) {
+            const int t0 = tok_begin + k * kStageTokens;
+            const int ntok = cmin(kStageTokens, tok_end - t0);
+            int blk = 0;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) qr[g][j][k] = make_float2(0.f, 0.f);
+            for (int j = 0; j < kIdWindow; ++j) {
+              const int v = __shfl_sync(0xffffffffu, cur_ids[j], k & 31);
+              if ((k >> 5) == j) blk = v;
+            }
+            if (k >= kIdWindow * 32) blk = __ldg(row + t0 / bs);  // beyond the prefetched window
+            const bool bad = blk < 0 || blk >= args.num_blocks;
+            if (bad) blk = args.num_blocks;  // out-of-range coordinate: TMA fills the box with zeros
+            const int slot = issued % kStages;
+            bool ok2 = true;
+            if (lane == 0) ok2 = mbar_wait(&empty[slot], (static_cast<uint32_t>(issued / kStages) & 1u) ^ 1u, err);
+            if (!__shfl_sync(0xffffffffu, ok2, 0)) {
+              aborted = true;
+              break;
+            }
+            if (lane == 0) {
+              StageMsg m;
+              m.item = local;
+              m.ntok = ntok;
+              m.flags = (k == 0 ? kMsgFirst : 0) | (k == n_stages - 1 ? kMsgLast : 0) | (bad ? kMsgBadBlock : 0);
+              m.pad = 0;
+              msgs[slot] = m;
+              if (bad) atomicOr(err, PA_DEVERR_BLOCK_ID);
+              mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(S::kStageBytes));
+            }
+            __syncwarp();
+            if (lane < 2 * S::kChunks) {
+              uint8_t* dst = smem + Lay::kRing + slot * S::kStageBytes + op_kv * S::kTileBytes + op_ch * S::kChunkBytes;
+              tma_load_4d(dst, op_kv ? &tmap_v : &tmap_k, &full[slot], op_ch * S::kChunkElems, kvh0, t0 % bs, blk);
+            }
+            ++issued;
+          }
+          ++local;
         }
       }
+      cur_idx = nxt_idx;
+      cur_L = nxt_L;
+#pragma unroll
+      for (int j = 0; j < kIdWindow; ++j) cur_ids[j] = nxt_ids[j];
     }
-  }
+#undef PA_PREPARE
+    // No work left: one terminating message.
+    if (!aborted) {
+      const int slot = issued % kStages;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&empty[slot], (static_cast<uint32_t>(issued / kStages) & 1u) ^ 1u, err);
+      if (__shfl_sync(0xffffffffu, ok, 0) && lane == 0) {
+        msgs[slot] = StageMsg{-1, 0, 0, 0};
+        mbar_arrive(&full[slot]);
+      }
+      ++issued;
+    }
+    // Every issued copy has landed before the CTA may leave (bounded waits).
+    if (lane == 0)
+      for (int p = cmax(0, issued - kStages); p < issued; ++p)
+        mbar_wait(&full[p % kStages], static_cast<uint32_t>(p / kStages) & 1u, err);
+    __syncwarp();
+  } else {
+    // =============================== consumer warps ===============================
+    const int cw = warp - 1;  // kv head within the item's head block
+    const int ds = lane & (S::kNS - 1);
+    const int tslot = lane >> S::kLog2NS;
+    const int g_lane = ds >> (S::kLog2NS - S::kLog2G);                 // head owned after reduce-scatter
+    const bool primary = (ds & ((S::kNS >> S::kLog2G) - 1)) == 0;      // first of the duplicate lanes
+    const int dp = lane & (S::kLPT - 1);
+    const int vslot = lane >> S::kLog2LPT;
+    float* pw = reinterpret_cast<float*>(smem + Lay::kPbuf) + cw * kStageTokens * G;
+    float* aw = reinterpret_cast<float*>(smem + Lay::kAbuf) + cw * G;
 
-  float m_run = -INFINITY;  // running max of head g_lane (log2 domain)
-  float l_run = 0.f;        // this lane's share of the running sum of head g_lane
-  float2 acc[G][4];
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) acc[g][k] = make_float2(0.f, 0.f);
+    float2 qr[G][S::kNPL][4];
+    float m_run = -INFINITY, l_run = 0.f;
+    float2 acc[G][4];
+    bool poisoned = false;
+    bool active = false;  // this warp's kv head exists in the current item
+    ItemInfo inf{};
 
-  float* pw = pbuf + warp * kStageTokens * G;
-  float* aw = abuf + warp * G;
-
-  for (int j = warp; j < n_stages; j += kConsumerWarps) {
-    const int slot = j % NST;
-    if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], static_cast<uint32_t>(j / NST) & 1u, args.error_word))) break;
-    const int nvalid = cmin(kStageTokens, tok_end - (tok_begin + j * kStageTokens));
-    const uint8_t* ktile = smem + slot * S::kStageBytes;
-    const uint8_t* vtile = ktile + S::kTileBytes;
-
-    // ---- scores ----
-    float sc[S::kIters];
+    for (int j = 0;; ++j) {
+      const int slot = j % kStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], static_cast<uint32_t>(j / kStages) & 1u, err))) break;
+      const StageMsg m = msgs[slot];
+      if (m.item < 0) break;
+      if (m.flags & kMsgFirst) {
+        // New item: load this head's query rows and reset the state.
+        const int qb = m.item % kQueryBuffers;
+        if (!__all_sync(0xffffffffu, mbar_wait(&qfull[qb], static_cast<uint32_t>(m.item / kQueryBuffers) & 1u, err)))
+          break;
+        inf = infos[qb];
+        active = inf.kvh0 + cw < args.num_kv_heads;
+        float qscale = args.scale_log2;
+        if constexpr (EB == 1) {
+          if (active) qscale *= args.k_scale[inf.kvh0 + cw];
+        }
+        const QT* qs = reinterpret_cast<const QT*>(smem + Lay::kQuery + qb * Lay::kQueryOne) + cw * G * D;
 #pragma unroll
-    for (int it = 0; it < S::kIters; ++it) {
-      const int t = it * S::kTPI + tslot;
-      float2 pacc[G];
+        for (int g = 0; g < G; ++g) {
 #pragma unroll
-      for (int g = 0; g < G; ++g) pacc[g] = make_float2(0.f, 0.f);
+          for (int jj = 0; jj < S::kNPL; ++jj) {
+            const int pc = qk_piece<S, EB>(jj, ds, tslot);
+            if (active && g < inf.heads) {
+              const uint4 raw = *reinterpret_cast<const uint4*>(qs + g * D + pc * 8);
+              const QT* e = reinterpret_cast<const QT*>(&raw);
 #pragma unroll
-      for (int jj = 0; jj < S::kNPL; ++jj) {
-        const int pc = qk_piece<S, EB>(jj, ds, tslot);
-        const Piece kp = *reinterpret_cast<const Piece*>(ktile + piece_offset<S>(t, pc));
-        float2 kf[4];
-        Elem<KVT>::to_float(kp, kf);
+              for (int k = 0; k < 4; ++k)
+                qr[g][jj][k] = make_float2(to_f32(e[2 * k]) * qscale, to_f32(e[2 * k + 1]) * qscale);
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) qr[g][jj][k] = make_float2(0.f, 0.f);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qempty[qb]);
+        m_run = -INFINITY;
+        l_run = 0.f;
+        poisoned = false;
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-          for (int k = 0; k < 4; ++k) pacc[g] = ffma2(qr[g][jj][k], kf[k], pacc[g]);
+          for (int k = 0; k < 4; ++k) acc[g][k] = make_float2(0.f, 0.f);
       }
-      float v[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) v[g] = pacc[g].x + pacc[g].y;
-      const float z = reduce_scatter<G, S::kLog2NS, S::kDsShift>(v, lane);
-      sc[it] = t < nvalid ? z : -INFINITY;
-    }
+      poisoned |= (m.flags & kMsgBadBlock) != 0;
 
-    // ---- online softmax (per head g_lane) ----
-    float cmax = sc[0];
+      if (active) {
+        const int nvalid = m.ntok;
+        const uint8_t* ktile = smem + Lay::kRing + slot * S::kStageBytes;
+        const uint8_t* vtile = ktile + S::kTileBytes;
+        // ---- scores ----
+        float sc[S::kIters];
 #pragma unroll
-    for (int it = 1; it < S::kIters; ++it) cmax = fmaxf(cmax, sc[it]);
+        for (int it = 0; it < S::kIters; ++it) {
+          const int t = it * S::kTPI + tslot;
+          float2 pacc[G];
 #pragma unroll
-    for (int b = 0; b < 5 - S::kLog2NS; ++b) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1 << (b + S::kTsShift)));
-    const float m_new = fmaxf(m_run, cmax);
-    const float alpha = fast_exp2(m_run - m_new);
-    float lsum = 0.f;
+          for (int g = 0; g < G; ++g) pacc[g] = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int it = 0; it < S::kIters; ++it) {
-      const float p = fast_exp2(sc[it] - m_new);
-      lsum += p;
-      if (primary) pw[(it * S::kTPI + tslot) * G + g_lane] = p;
-    }
-    l_run = l_run * alpha + lsum;
-    m_run = m_new;
-    if (primary && tslot == 0) aw[g_lane] = alpha;
-    __syncwarp();
-
-    // ---- P V ----
+          for (int jj = 0; jj < S::kNPL; ++jj) {
+            const int pc = qk_piece<S, EB>(jj, ds, tslot);
+            const Piece kp = *reinterpret_cast<const Piece*>(ktile + piece_offset<S>(t * kHeadBlock + cw, pc));
+            float2 kf[4];
+            Elem<KVT>::to_float(kp, kf);
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float a = aw[g];
+            for (int g = 0; g < G; ++g)
 #pragma unroll
-      for (int k = 0; k < 4; ++k) acc[g][k] = make_float2(acc[g][k].x * a, acc[g][k].y * a);
-    }
-    for (int t0 = 0; t0 < nvalid; t0 += S::kTPV) {
-      const int t = t0 + vslot;
-      if (t < nvalid) {
-        const Piece vp = *reinterpret_cast<const Piece*>(vtile + piece_offset<S>(t, dp));
-        float2 vf[4];
-        Elem<KVT>::to_float(vp, vf);
-        float p[G];
-        if constexpr (G >= 4) {
-#pragma unroll
-          for (int g = 0; g < G; g += 4) {
-            const float4 p4 = *reinterpret_cast<const float4*>(pw + t * G + g);
-            p[g] = p4.x; p[g + 1] = p4.y; p[g + 2] = p4.z; p[g + 3] = p4.w;
+              for (int k = 0; k < 4; ++k) pacc[g] = ffma2(qr[g][jj][k], kf[k], pacc[g]);
           }
-        } else {
+          float v[G];
 #pragma unroll
-          for (int g = 0; g < G; ++g) p[g] = pw[t * G + g];
+          for (int g = 0; g < G; ++g) v[g] = pacc[g].x + pacc[g].y;
+          const float z = reduce_scatter<G, S::kLog2NS>(v, lane);
+          sc[it] = t < nvalid ? z : -INFINITY;
         }
+        // ---- online softmax (per head g_lane) ----
+        float cm = sc[0];
+#pragma unroll
+        for (int it = 1; it < S::kIters; ++it) cm = fmaxf(cm, sc[it]);
+#pragma unroll
+        for (int b = S::kTsShift; b < 5; ++b) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1 << b));
+        const float m_new = fmaxf(m_run, cm);
+        const float alpha = fast_exp2(m_run - m_new);
+        float lsum = 0.f;
+#pragma unroll
+        for (int it = 0; it < S::kIters; ++it) {
+          const float p = fast_exp2(sc[it] - m_new);
+          lsum += p;
+          if (primary) pw[(it * S::kTPI + tslot) * G + g_lane] = p;
+        }
+        l_run = l_run * alpha + lsum;
+        m_run = m_new;
+        if (primary && tslot == 0) aw[g_lane] = alpha;
+        __syncwarp();
+        // ---- P V ----
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const float2 pp = make_float2(p[g], p[g]);
+          const float a = aw[g];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) acc[g][k] = ffma2(pp, vf[k], acc[g][k]);
+          for (int k = 0; k < 4; ++k) acc[g][k] = make_float2(acc[g][k].x * a, acc[g][k].y * a);
+        }
+#pragma unroll
+        for (int t0 = 0; t0 < kStageTokens; t0 += S::kTPV) {
+          const int t = t0 + vslot;
+          if (t < nvalid) {
+            const Piece vp = *reinterpret_cast<const Piece*>(vtile + piece_offset<S>(t * kHeadBlock + cw, dp));
+            float2 vf[4];
+            Elem<KVT>::to_float(vp, vf);
+            float p[G];
+            if constexpr (G >= 4) {
+#pragma unroll
+              for (int g = 0; g < G; g += 4) {
+                const float4 p4 = *reinterpret_cast<const float4*>(pw + t * G + g);
+                p[g] = p4.x; p[g + 1] = p4.y; p[g + 2] = p4.z; p[g + 3] = p4.w;
+              }
+            } else {
+#pragma unroll
+              for (int g = 0; g < G; ++g) p[g] = pw[t * G + g];
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              const float2 pp = make_float2(p[g], p[g]);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) acc[g][k] = ffma2(pp, vf[k], acc[g][k]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+
+      if ((m.flags & kMsgLast) && active) {
+        // ---- end of the item: normalise and write this kv head's query heads ----
+        float l_tot = l_run;
+#pragma unroll
+        for (int b = S::kTsShift; b < 5; ++b) l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 1 << b);
+#pragma unroll
+        for (int b = S::kLog2LPT; b < 5; ++b) {
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              acc[g][k].x += __shfl_xor_sync(0xffffffffu, acc[g][k].x, 1 << b);
+              acc[g][k].y += __shfl_xor_sync(0xffffffffu, acc[g][k].y, 1 << b);
+            }
+        }
+        // l and m of head g live on the primary lanes with tslot 0 (lane g << (log2 NS - log2 G)).
+        const float vscale = (EB == 1) ? args.v_scale[inf.kvh0 + cw] : 1.0f;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const int src = g << (S::kLog2NS - S::kLog2G);
+          const float lg = __shfl_sync(0xffffffffu, l_tot, src);
+          const float mg = __shfl_sync(0xffffffffu, m_run, src);
+          if (g < inf.heads && vslot == 0) {
+            float r = vscale / lg;
+            if (poisoned) r = __int_as_float(0x7fc00000);
+            const int h = (inf.kvh0 + cw) * args.group + inf.h_sub + g;
+            if (inf.write_final) {
+              QT* out = static_cast<QT*>(args.out) + (static_cast<size_t>(inf.s) * args.num_heads + h) * D + dp * 8;
+              *reinterpret_cast<uint2*>(out) = pack4<QT>(acc[g][0].x * r, acc[g][0].y * r, acc[g][1].x * r, acc[g][1].y * r);
+              *reinterpret_cast<uint2*>(out + 4) = pack4<QT>(acc[g][2].x * r, acc[g][2].y * r, acc[g][3].x * r, acc[g][3].y * r);
+            } else {
+              const size_t rowi = (static_cast<size_t>(inf.s) * args.num_heads + h) * args.num_partitions + inf.part;
+              float* po = args.part_o + rowi * D + dp * 8;
+              *reinterpret_cast<float4*>(po) = make_float4(acc[g][0].x * r, acc[g][0].y * r, acc[g][1].x * r, acc[g][1].y * r);
+              *reinterpret_cast<float4*>(po + 4) = make_float4(acc[g][2].x * r, acc[g][2].y * r, acc[g][3].x * r, acc[g][3].y * r);
+              if (dp == 0) {
+                args.part_m[rowi] = mg;
+                args.part_l[rowi] = lg;
+              }
+            }
+          }
         }
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot]);
   }
 
-  // ---- per-warp totals ----
-#pragma unroll
-  for (int b = 0; b < 5 - S::kLog2NS; ++b) l_run += __shfl_xor_sync(0xffffffffu, l_run, 1 << (b + S::kTsShift));
-#pragma unroll
-  for (int b = S::kLog2LPT; b < 5; ++b) {
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        acc[g][k].x += __shfl_xor_sync(0xffffffffu, acc[g][k].x, 1 << b);
-        acc[g][k].y += __shfl_xor_sync(0xffffffffu, acc[g][k].y, 1 << b);
-      }
-  }
-
-  named_barrier(1, kThreads);  // producer has drained: the ring memory is free for the merge
-
-  float* ma = reinterpret_cast<float*>(smem);              // [W][G][D]
-  float* mm = ma + kConsumerWarps * G * D;                 // [W][G]
-  float* ml = mm + kConsumerWarps * G;                     // [W][G]
-  if (vslot == 0) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float* dst = ma + (warp * G + g) * D + dp * 8;
-      *reinterpret_cast<float4*>(dst) = make_float4(acc[g][0].x, acc[g][0].y, acc[g][1].x, acc[g][1].y);
-      *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[g][2].x, acc[g][2].y, acc[g][3].x, acc[g][3].y);
-    }
-  }
-  if (primary && tslot == 0) {
-    mm[warp * G + g_lane] = m_run;
-    ml[warp * G + g_lane] = l_run;
-  }
-  named_barrier(2, kConsumerWarps * 32);
-
-  const bool poisoned = flags[0] != 0;
-  const float vscale = (EB == 1) ? args.v_scale[kvh] : 1.0f;
-  for (int idx = threadIdx.x; idx < G * (D / 4); idx += kConsumerWarps * 32) {
-    const int g = idx / (D / 4);
-    const int d0 = (idx - g * (D / 4)) * 4;
-    if (g >= heads_here) continue;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mm[w * G + g]);
-    float lsum = 0.f;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      const float e = fast_exp2(mm[w * G + g] - M);
-      lsum += e * ml[w * G + g];
-      const float4 a = *reinterpret_cast<const float4*>(ma + (w * G + g) * D + d0);
-      o.x += e * a.x; o.y += e * a.y; o.z += e * a.z; o.w += e * a.w;
-    }
-    float r = vscale / lsum;
-    if (poisoned) r = __int_as_float(0x7fc00000);
-    const int h = h0 + g;
-    if (write_final) {
-      QT* out = static_cast<QT*>(args.out) + (static_cast<size_t>(s) * args.num_heads + h) * D + d0;
-      *reinterpret_cast<uint2*>(out) = pack4<QT>(o.x * r, o.y * r, o.z * r, o.w * r);
-    } else {
-      const size_t row = (static_cast<size_t>(s) * args.num_heads + h) * args.num_partitions + part;
-      *reinterpret_cast<float4*>(args.part_o + row * D + d0) = make_float4(o.x * r, o.y * r, o.z * r, o.w * r);
-      if (d0 == 0) {
-        args.part_m[row] = M;
-        args.part_l[row] = lsum;
-      }
+  // The last CTA to finish resets the work counter for the next launch on this workspace.
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned int done = atomicAdd(args.header + kWsDone, 1u);
+    if (done == gridDim.x - 1) {
+      atomicExch(args.header + kWsWork, 0u);
+      atomicExch(args.header + kWsDone, 0u);
     }
   }
 }
@@ -488,7 +634,7 @@ paged_attention_reduce(const AttnArgs args) {
   const int i = threadIdx.x;
   const int L = args.context_lens[s];
   const int PS = args.partition_size;
-  if (L <= 0 || L > args.max_blocks_per_seq * args.block_size || L > args.num_partitions * PS) return;
+  if (L <= 0 || context_len_invalid(L, args)) return;
   const int n_parts = (L + PS - 1) / PS;
   if (n_parts <= 1) return;
   const size_t base = (static_cast<size_t>(s) * args.num_heads + h) * args.num_partitions;

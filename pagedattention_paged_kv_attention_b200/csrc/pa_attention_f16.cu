@@ -3,7 +3,7 @@
 
 namespace pa {
 cudaError_t launch_attention_f16(const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a, bool fp8_cache,
-                                 int D, int G, dim3 grid, cudaStream_t stream) {
+                                 int D, int G, int grid, cudaStream_t stream) {
   if (fp8_cache) return launch_attention<__half, __nv_fp8_e4m3>(tk, tv, a, D, G, grid, stream);
   return launch_attention<__half, __half>(tk, tv, a, D, G, grid, stream);
 }

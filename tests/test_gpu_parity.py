@@ -7,8 +7,12 @@
   are compared byte for byte with the oracle's (reshape_and_cache and copy_blocks are bit-exact, and
   nothing else in the pool may change).
 * Split-K partition sizes from one stage to the whole context agree with the oracle.
-* Smaller ragged cases over every supported head size, block size, dtype and group size.
+* Smaller ragged cases over every supported head size, block size, dtype and group size. Their
+  contexts go down to one token, where outputs reach about 5 in magnitude; there each element is
+  bounded by the stated tolerance plus half an ulp of the output dtype at that magnitude.
 """
+import zlib
+
 import numpy as np
 import pytest
 import torch
@@ -16,7 +20,7 @@ import torch
 import oracle
 import workloads as W
 from helpers import bits16
-from steps import TOLERANCE, gpu_step, initial_pools, oracle_step, pool_bits, to_device_pool
+from steps import TOLERANCE, elementwise_bound, gpu_step, initial_pools, oracle_step, pool_bits, to_device_pool
 
 pytestmark = pytest.mark.gpu
 
@@ -86,7 +90,8 @@ LENS = [1, 2, 7, 8, 9, 63, 64, 65, 127, 200, 511, 513, 1000]
 
 @pytest.mark.parametrize("kv_dtype,dtype,d,bs,H,Hkv", CASES)
 def test_ragged_small_cases(P, kv_dtype, dtype, d, bs, H, Hkv):
-    cfg, w = small_case(kv_dtype, dtype, d, bs, H, Hkv, LENS, seed=hash((kv_dtype, dtype, d, bs, H, Hkv)) % 1000)
+    seed = zlib.crc32(repr((kv_dtype, dtype, d, bs, H, Hkv)).encode()) % 1000
+    cfg, w = small_case(kv_dtype, dtype, d, bs, H, Hkv, LENS, seed=seed)
     kc, vc = initial_pools(w)
     kc_dev, vc_dev = to_device_pool(kc, cfg), to_device_pool(vc, cfg)
     for ps in (0, 64, 192):
@@ -94,7 +99,10 @@ def test_ragged_small_cases(P, kv_dtype, dtype, d, bs, H, Hkv):
         out, ws = gpu_step(P, w, k2, v2, partition_size=ps)
         kcc, vcc = kc.copy(), vc.copy()
         ref = oracle_step(w, kcc, vcc)
-        assert max_abs_err(out, ref) <= TOLERANCE[kv_dtype], f"partition_size={ps}"
+        got = out.double().cpu().numpy()
+        assert np.all(np.isfinite(got))
+        excess = np.abs(got - ref) - elementwise_bound(ref, kv_dtype, dtype)
+        assert np.max(excess) <= 0, f"partition_size={ps}: worst excess {np.max(excess)}"
         assert P.get_device_error(ws) == 0
         assert torch.equal(pool_bits(k2), pool_bits(to_device_pool(kcc, cfg)))
         assert torch.equal(pool_bits(v2), pool_bits(to_device_pool(vcc, cfg)))
