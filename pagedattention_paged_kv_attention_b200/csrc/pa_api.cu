@@ -85,19 +85,21 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 4-D view {head_size, num_kv_heads, block_size, num_blocks} of a cache; box = one 128-byte chunk of
-// the rows of 8 consecutive kv heads for 8 consecutive tokens of one block (heads past the last one
-// read as zeros), written to shared memory with the 128-byte swizzle.
+// 4-D view of a cache; box = one 128-byte chunk of the rows of 8 consecutive tokens for 8 consecutive
+// kv heads of one block (heads past the last one read as zeros), written to shared memory with the
+// 128-byte swizzle.
 bool encode_cache_map(CUtensorMap* map, const void* cache, int elem_bytes, int head_size, int num_kv_heads,
                       int block_size, int num_blocks) {
   auto encode = tensor_map_encoder();
   if (!encode) return false;
   const cuuint64_t e = static_cast<cuuint64_t>(elem_bytes);
-  cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_size), static_cast<cuuint64_t>(num_kv_heads),
-                        static_cast<cuuint64_t>(block_size), static_cast<cuuint64_t>(num_blocks)};
-  cuuint64_t strides[3] = {head_size * e, num_kv_heads * head_size * e, block_size * num_kv_heads * head_size * e};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(pa::kHeadBlock),
-                       static_cast<cuuint32_t>(pa::kStageTokens), 1};
+  // Dimensions in the order {d, token, kv head, block}: the token dimension (stride Hkv*d) is listed
+  // before the head dimension (stride d), so a box lands in shared memory as [head][token][chunk].
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_size), static_cast<cuuint64_t>(block_size),
+                        static_cast<cuuint64_t>(num_kv_heads), static_cast<cuuint64_t>(num_blocks)};
+  cuuint64_t strides[3] = {num_kv_heads * head_size * e, head_size * e, block_size * num_kv_heads * head_size * e};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(pa::kStageTokens),
+                       static_cast<cuuint32_t>(pa::kHeadBlock), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = encode(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
                       const_cast<void*>(cache), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,

@@ -17,22 +17,27 @@
 //    finish resets the counter.
 //  * Warp 0 is the producer. Per item it bulk-copies the query rows of the 8 heads into shared memory;
 //    then, for each 8-token stage, it reads one block-table entry (prefetched a window at a time) and
-//    issues 4-D TMA tile loads {128-byte chunk, 8 kv heads, 8 tokens, 1 block} of K and V (128-byte
-//    swizzle) into a shared-memory ring whose slots are guarded by mbarriers, with a small message
-//    (item, valid tokens, first/last stage). The page-table walk is a TMA coordinate.
+//    issues 4-D TMA tile loads {128-byte chunk, 8 tokens, 8 kv heads, 1 block} of K and V (128-byte
+//    swizzle; the tensor map lists the token dimension before the head dimension, so each head's 8
+//    token rows form one swizzle atom) into a shared-memory ring whose slots are guarded by mbarriers,
+//    with a small message (item, valid tokens, first/last stage). The page-table walk is a TMA
+//    coordinate.
 //  * Warps 1..8 are consumers; warp w owns kv head w of the block for the whole item and keeps an fp32
 //    online-softmax state (running max m, running sum l, accumulator acc[G][d]) for the G query heads
 //    of that kv head (grouped-query heads are batched: each K/V element is read once for all G heads).
-//      QK: NS >= 8 lanes cooperate on one token (each holds 1/NS of d and the G query rows in
-//          registers, pre-scaled by scale*log2(e)); a butterfly reduce-scatter leaves each lane with
-//          the full score of one head. Lanes of a shared-memory phase read distinct 16-byte units of
-//          one row, so the swizzled rows are read without bank conflicts.
-//      softmax: stage max per head across lanes, rescale alpha = 2^(m_old - m_new), p = 2^(z - m_new)
-//          through a per-warp shared buffer.
-//      PV: D/8 lanes cover one V row (8 elements each); every lane accumulates all G heads.
-//    Packed f32x2 FMAs are used throughout; inputs are widened to fp32 once per element. At the end of
-//    an item each warp writes its heads' normalised output, or (m, l, acc/l) partials that the reduce
-//    kernel merges across partitions (log-sum-exp merge).
+//    Two ways to compute, chosen at compile time:
+//    - Tensor cores (16-bit caches, G >= 2): Q[G x d] K^T and P V are contractions over d and over the
+//      stage's tokens, done with warp-level mma.sync tiles (m16n8k16 for S = Q K^T with the query
+//      rows held as A fragments, m16n8k8 for O += P V); K^T and V come from the swizzled tiles through
+//      ldmatrix (V transposed). The score fragment becomes the P fragment in registers; the softmax
+//      statistics are per query head (one quad of lanes per head).
+//    - CUDA cores (G == 1, and FP8 caches): NS >= 8 lanes cooperate on one token (each holds 1/NS of
+//      d and the G query rows in registers, pre-scaled by scale*log2(e)); a butterfly reduce-scatter
+//      leaves each lane with the full score of one head; p goes through a per-warp shared buffer; for
+//      PV, D/8 lanes cover one V row and every lane accumulates all G heads; packed f32x2 FMAs.
+//    Either way: online softmax with alpha = 2^(m_old - m_new), p = 2^(z - m_new), fp32 statistics
+//    and accumulators. At the end of an item each warp writes its heads' normalised output, or
+//    (m, l, acc/l) partials that the reduce kernel merges across partitions (log-sum-exp merge).
 // Arithmetic order depends only on logical token positions, never on physical block ids or on which
 // CTA handled an item, so outputs are bitwise invariant to block placement and deterministic.
 #pragma once
@@ -110,10 +115,14 @@ struct Shape {
   static constexpr int kLPT = D / 8;
   static constexpr int kLog2LPT = ilog2(kLPT);
   static constexpr int kTPV = 32 / kLPT;
-  // One stage: [K|V][chunk][token][head][128 B].
+  // One stage: [K|V][chunk][head][token][128 B].
   static constexpr int kChunkBytes = kStageTokens * kHeadBlock * 128;
   static constexpr int kTileBytes = kChunks * kChunkBytes;
   static constexpr int kStageBytes = 2 * kTileBytes;
+  // Tensor-core path: 16-bit caches with at least two query heads per kv head.
+  static constexpr bool kMma = (EB == 2) && (G >= 2);
+  static constexpr int kKSteps = D / 16;                 // m16n8k16 steps over d
+  static constexpr int kNBlocks = D / 8;                 // n8 blocks of the output row
   static_assert(kRowBytes == 128 || kRowBytes == 256, "row must be 128 or 256 bytes");
   static_assert(kNS >= 8 && G <= kNS, "lane mapping");
   static_assert(kNPL >= 1 && kNPL * kNS == kPiecesPerRow, "pieces must split evenly");
@@ -151,9 +160,9 @@ struct Layout {
   static_assert(kAllocBytes <= 227 * 1024, "shared memory layout too large");
 };
 
-// Byte offset of piece `pc` (8 elements) of tile row r = token * 8 + head inside a
-// [chunk][kStageTokens * 8 rows][128 B] tile written by TMA with the 128-byte swizzle (16-byte unit u
-// of row r lives at unit u ^ (r & 7) = u ^ head).
+// Byte offset of piece `pc` (8 elements) of tile row r = head * 8 + token inside a
+// [chunk][8 heads * kStageTokens rows][128 B] tile written by TMA with the 128-byte swizzle (16-byte
+// unit u of row r lives at unit u ^ (r & 7) = u ^ token).
 template <class S>
 __device__ __forceinline__ uint32_t piece_offset(int r, int pc) {
   const int byte = pc * S::kPieceBytes;
@@ -386,7 +395,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             __syncwarp();
             if (lane < 2 * S::kChunks) {
               uint8_t* dst = smem + Lay::kRing + slot * S::kStageBytes + op_kv * S::kTileBytes + op_ch * S::kChunkBytes;
-              tma_load_4d(dst, op_kv ? &tmap_v : &tmap_k, &full[slot], op_ch * S::kChunkElems, kvh0, t0 % bs, blk);
+              tma_load_4d(dst, op_kv ? &tmap_v : &tmap_k, &full[slot], op_ch * S::kChunkElems, t0 % bs, kvh0, blk);
             }
             ++issued;
           }
@@ -430,6 +439,8 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     float2 qr[G][S::kNPL][4];
     float m_run = -INFINITY, l_run = 0.f;
     float2 acc[G][4];
+    uint32_t qa[S::kKSteps][2];   // tensor-core path: query A fragments (rows g = lane/4), a0 and a2
+    float o[S::kNBlocks][4];      // tensor-core path: output accumulator fragments
     bool poisoned = false;
     bool active = false;  // this warp's kv head exists in the current item
     ItemInfo inf{};
@@ -451,6 +462,17 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           if (active) qscale *= args.k_scale[inf.kvh0 + cw];
         }
         const QT* qs = reinterpret_cast<const QT*>(smem + Lay::kQuery + qb * Lay::kQueryOne) + cw * G * D;
+        if constexpr (S::kMma) {
+          const int g = lane >> 2, t4 = lane & 3;
+          const bool row_ok = active && g < inf.heads;
+#pragma unroll
+          for (int ks = 0; ks < S::kKSteps; ++ks) {
+            qa[ks][0] = row_ok ? *reinterpret_cast<const uint32_t*>(qs + g * D + ks * 16 + 2 * t4) : 0u;
+            qa[ks][1] = row_ok ? *reinterpret_cast<const uint32_t*>(qs + g * D + ks * 16 + 8 + 2 * t4) : 0u;
+          }
+#pragma unroll
+          for (int nb = 0; nb < S::kNBlocks; ++nb) o[nb][0] = o[nb][1] = o[nb][2] = o[nb][3] = 0.f;
+        } else
 #pragma unroll
         for (int g = 0; g < G; ++g) {
 #pragma unroll
@@ -480,7 +502,55 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
       }
       poisoned |= (m.flags & kMsgBadBlock) != 0;
 
-      if (active) {
+      if constexpr (S::kMma) {
+       if (active) {
+        // ---------------- tensor-core stage ----------------
+        const int nvalid = m.ntok;
+        const uint32_t kbase = smem_u32(smem + Lay::kRing + slot * S::kStageBytes);
+        const uint32_t vbase = kbase + S::kTileBytes;
+        const int t4 = lane & 3;
+        // ldmatrix row addresses: lane i points at token row i % 8 of this head, 16-byte unit i / 8.
+        const int lrow = cw * kStageTokens + (lane & 7);
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q4 = 0; q4 < S::kKSteps / 2; ++q4) {
+          uint32_t kb[4];
+          ldmatrix_x4(kbase + piece_offset<S>(lrow, q4 * 4 + (lane >> 3)), kb);
+          const uint32_t a0[4] = {qa[2 * q4][0], 0u, qa[2 * q4][1], 0u};
+          mma_16816<KVT>(sacc, a0, kb[0], kb[1]);
+          const uint32_t a1[4] = {qa[2 * q4 + 1][0], 0u, qa[2 * q4 + 1][1], 0u};
+          mma_16816<KVT>(sacc, a1, kb[2], kb[3]);
+        }
+        // Scores of query head lane/4 for tokens 2*t4 and 2*t4 + 1.
+        const float s0 = 2 * t4 < nvalid ? sacc[0] * args.scale_log2 : -INFINITY;
+        const float s1 = 2 * t4 + 1 < nvalid ? sacc[1] * args.scale_log2 : -INFINITY;
+        float cm = fmaxf(s0, s1);
+        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
+        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
+        const float m_new = fmaxf(m_run, cm);
+        const float alpha = fast_exp2(m_run - m_new);
+        const uint32_t pfrag = pack2<KVT>(fast_exp2(s0 - m_new), fast_exp2(s1 - m_new));
+        // The sum uses the rounded weights that enter P V, so the weights of the output sum to one.
+        const float2 pr = unpack2<KVT>(pfrag);
+        l_run = l_run * alpha + (pr.x + pr.y);
+        m_run = m_new;
+#pragma unroll
+        for (int nb = 0; nb < S::kNBlocks; ++nb) {
+          o[nb][0] *= alpha;
+          o[nb][1] *= alpha;
+        }
+        // V rows of tokens past the valid ones may hold anything (even NaN): zero their halves of the
+        // B fragments (low half = token 2*t4, high half = token 2*t4 + 1).
+        const uint32_t vmask = (2 * t4 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 1 < nvalid ? 0xffff0000u : 0u);
+#pragma unroll
+        for (int q4 = 0; q4 < S::kNBlocks / 4; ++q4) {
+          uint32_t vb[4];
+          ldmatrix_x4_trans(vbase + piece_offset<S>(lrow, q4 * 4 + (lane >> 3)), vb);
+#pragma unroll
+          for (int j4 = 0; j4 < 4; ++j4) mma_1688<KVT>(o[q4 * 4 + j4], pfrag, 0u, vb[j4] & vmask);
+        }
+       }
+      } else if (active) {
         const int nvalid = m.ntok;
         const uint8_t* ktile = smem + Lay::kRing + slot * S::kStageBytes;
         const uint8_t* vtile = ktile + S::kTileBytes;
@@ -495,7 +565,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
 #pragma unroll
           for (int jj = 0; jj < S::kNPL; ++jj) {
             const int pc = qk_piece<S, EB>(jj, ds, tslot);
-            const Piece kp = *reinterpret_cast<const Piece*>(ktile + piece_offset<S>(t * kHeadBlock + cw, pc));
+            const Piece kp = *reinterpret_cast<const Piece*>(ktile + piece_offset<S>(cw * kStageTokens + t, pc));
             float2 kf[4];
             Elem<KVT>::to_float(kp, kf);
 #pragma unroll
@@ -539,7 +609,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         for (int t0 = 0; t0 < kStageTokens; t0 += S::kTPV) {
           const int t = t0 + vslot;
           if (t < nvalid) {
-            const Piece vp = *reinterpret_cast<const Piece*>(vtile + piece_offset<S>(t * kHeadBlock + cw, dp));
+            const Piece vp = *reinterpret_cast<const Piece*>(vtile + piece_offset<S>(cw * kStageTokens + t, dp));
             float2 vf[4];
             Elem<KVT>::to_float(vp, vf);
             float p[G];
@@ -565,7 +635,35 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
 
-      if ((m.flags & kMsgLast) && active) {
+      if constexpr (S::kMma) {
+       if ((m.flags & kMsgLast) && active) {
+        // ---- end of the item (tensor-core path): row g = lane/4 is query head g ----
+        float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 1);
+        l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
+        const int g = lane >> 2, t4 = lane & 3;
+        if (g < inf.heads) {
+          float r = 1.0f / l_tot;
+          if (poisoned) r = __int_as_float(0x7fc00000);
+          const int h = (inf.kvh0 + cw) * args.group + inf.h_sub + g;
+          if (inf.write_final) {
+            QT* out = static_cast<QT*>(args.out) + (static_cast<size_t>(inf.s) * args.num_heads + h) * D + 2 * t4;
+#pragma unroll
+            for (int nb = 0; nb < S::kNBlocks; ++nb)
+              *reinterpret_cast<uint32_t*>(out + nb * 8) = pack2<QT>(o[nb][0] * r, o[nb][1] * r);
+          } else {
+            const size_t rowi = (static_cast<size_t>(inf.s) * args.num_heads + h) * args.num_partitions + inf.part;
+            float* po = args.part_o + rowi * D + 2 * t4;
+#pragma unroll
+            for (int nb = 0; nb < S::kNBlocks; ++nb)
+              *reinterpret_cast<float2*>(po + nb * 8) = make_float2(o[nb][0] * r, o[nb][1] * r);
+            if (t4 == 0) {
+              args.part_m[rowi] = m_run;
+              args.part_l[rowi] = l_tot;
+            }
+          }
+        }
+       }
+      } else if ((m.flags & kMsgLast) && active) {
         // ---- end of the item: normalise and write this kv head's query heads ----
         float l_tot = l_run;
 #pragma unroll
