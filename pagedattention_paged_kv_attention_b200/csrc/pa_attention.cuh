@@ -26,12 +26,13 @@
 //    online-softmax state (running max m, running sum l, accumulator acc[G][d]) for the G query heads
 //    of that kv head (grouped-query heads are batched: each K/V element is read once for all G heads).
 //    Two ways to compute, chosen at compile time:
-//    - Tensor cores (16-bit caches, G >= 2): Q[G x d] K^T and P V are contractions over d and over the
-//      stage's tokens, done with warp-level mma.sync tiles (m16n8k16 for S = Q K^T with the query
-//      rows held as A fragments, m16n8k8 for O += P V); K^T and V come from the swizzled tiles through
-//      ldmatrix (V transposed). The score fragment becomes the P fragment in registers; the softmax
-//      statistics are per query head (one quad of lanes per head).
-//    - CUDA cores (G == 1, and FP8 caches): NS >= 8 lanes cooperate on one token (each holds 1/NS of
+//    - Tensor cores (G >= 2): Q[G x d] K^T and P V are contractions over d and over the stage's
+//      tokens, done with warp-level mma.sync tiles (m16n8k16 for S = Q K^T with the query rows held as
+//      A fragments, m16n8k8 for O += P V). 16-bit K^T and V come from the swizzled tiles through
+//      ldmatrix (V transposed); FP8 pairs are read into the fragment layout and widened to f16 pairs
+//      by one hardware conversion (exact). The score fragment becomes the P fragment in registers;
+//      the softmax statistics are per query head (one quad of lanes per head).
+//    - CUDA cores (G == 1): NS >= 8 lanes cooperate on one token (each holds 1/NS of
 //      d and the G query rows in registers, pre-scaled by scale*log2(e)); a butterfly reduce-scatter
 //      leaves each lane with the full score of one head; p goes through a per-warp shared buffer; for
 //      PV, D/8 lanes cover one V row and every lane accumulates all G heads; packed f32x2 FMAs.
@@ -41,6 +42,8 @@
 // Arithmetic order depends only on logical token positions, never on physical block ids or on which
 // CTA handled an item, so outputs are bitwise invariant to block placement and deterministic.
 #pragma once
+
+#include <type_traits>
 
 #include "pa_device.cuh"
 
@@ -119,8 +122,9 @@ struct Shape {
   static constexpr int kChunkBytes = kStageTokens * kHeadBlock * 128;
   static constexpr int kTileBytes = kChunks * kChunkBytes;
   static constexpr int kStageBytes = 2 * kTileBytes;
-  // Tensor-core path: 16-bit caches with at least two query heads per kv head.
-  static constexpr bool kMma = (EB == 2) && (G >= 2);
+  // Tensor-core path: at least two query heads per kv head. FP8 caches enter the tensor cores as
+  // f16 (every E4M3 value is exact in f16), with f16 query fragments.
+  static constexpr bool kMma = G >= 2;
   static constexpr int kKSteps = D / 16;                 // m16n8k16 steps over d
   static constexpr int kNBlocks = D / 8;                 // n8 blocks of the output row
   static_assert(kRowBytes == 128 || kRowBytes == 256, "row must be 128 or 256 bytes");
@@ -240,6 +244,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
   using S = Shape<D, G, EB>;
   using Lay = Layout<QT, D, G, EB>;
   using Piece = typename Elem<KVT>::Piece;
+  using MmaT = typename std::conditional<EB == 2, KVT, __half>::type;  // tensor-core input type
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -467,8 +472,14 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           const bool row_ok = active && g < inf.heads;
 #pragma unroll
           for (int ks = 0; ks < S::kKSteps; ++ks) {
-            qa[ks][0] = row_ok ? *reinterpret_cast<const uint32_t*>(qs + g * D + ks * 16 + 2 * t4) : 0u;
-            qa[ks][1] = row_ok ? *reinterpret_cast<const uint32_t*>(qs + g * D + ks * 16 + 8 + 2 * t4) : 0u;
+            if constexpr (EB == 2) {
+              qa[ks][0] = row_ok ? *reinterpret_cast<const uint32_t*>(qs + g * D + ks * 16 + 2 * t4) : 0u;
+              qa[ks][1] = row_ok ? *reinterpret_cast<const uint32_t*>(qs + g * D + ks * 16 + 8 + 2 * t4) : 0u;
+            } else {
+              const QT* qrow = qs + g * D + ks * 16 + 2 * t4;
+              qa[ks][0] = row_ok ? pack2<__half>(to_f32(qrow[0]), to_f32(qrow[1])) : 0u;
+              qa[ks][1] = row_ok ? pack2<__half>(to_f32(qrow[8]), to_f32(qrow[9])) : 0u;
+            }
           }
 #pragma unroll
           for (int nb = 0; nb < S::kNBlocks; ++nb) o[nb][0] = o[nb][1] = o[nb][2] = o[nb][3] = 0.f;
@@ -512,26 +523,42 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         // ldmatrix row addresses: lane i points at token row i % 8 of this head, 16-byte unit i / 8.
         const int lrow = cw * kStageTokens + (lane & 7);
         float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (EB == 2) {
 #pragma unroll
-        for (int q4 = 0; q4 < S::kKSteps / 2; ++q4) {
-          uint32_t kb[4];
-          ldmatrix_x4(kbase + piece_offset<S>(lrow, q4 * 4 + (lane >> 3)), kb);
-          const uint32_t a0[4] = {qa[2 * q4][0], 0u, qa[2 * q4][1], 0u};
-          mma_16816<KVT>(sacc, a0, kb[0], kb[1]);
-          const uint32_t a1[4] = {qa[2 * q4 + 1][0], 0u, qa[2 * q4 + 1][1], 0u};
-          mma_16816<KVT>(sacc, a1, kb[2], kb[3]);
+          for (int q4 = 0; q4 < S::kKSteps / 2; ++q4) {
+            uint32_t kb[4];
+            ldmatrix_x4(kbase + piece_offset<S>(lrow, q4 * 4 + (lane >> 3)), kb);
+            const uint32_t a0[4] = {qa[2 * q4][0], 0u, qa[2 * q4][1], 0u};
+            mma_16816<MmaT>(sacc, a0, kb[0], kb[1]);
+            const uint32_t a1[4] = {qa[2 * q4 + 1][0], 0u, qa[2 * q4 + 1][1], 0u};
+            mma_16816<MmaT>(sacc, a1, kb[2], kb[3]);
+          }
+        } else {
+          // FP8 rows are 128 bytes (one swizzle chunk): B fragment b0 of step ks is the byte pair
+          // (ks*16 + 2*t4, +1) of token row lane/4, b1 the pair 8 bytes further.
+          const int tok = lane >> 2;
+          const uint8_t* krow = smem + Lay::kRing + slot * S::kStageBytes + (cw * kStageTokens + tok) * 128;
+#pragma unroll
+          for (int ks = 0; ks < S::kKSteps; ++ks) {
+            const uint8_t* unit = krow + ((ks ^ tok) << 4) + 2 * t4;
+            const uint32_t b0 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(unit));
+            const uint32_t b1 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(unit + 8));
+            const uint32_t a[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
+            mma_16816<MmaT>(sacc, a, b0, b1);
+          }
         }
         // Scores of query head lane/4 for tokens 2*t4 and 2*t4 + 1.
-        const float s0 = 2 * t4 < nvalid ? sacc[0] * args.scale_log2 : -INFINITY;
-        const float s1 = 2 * t4 + 1 < nvalid ? sacc[1] * args.scale_log2 : -INFINITY;
+        const float zscale = (EB == 1) ? args.scale_log2 * args.k_scale[inf.kvh0 + cw] : args.scale_log2;
+        const float s0 = 2 * t4 < nvalid ? sacc[0] * zscale : -INFINITY;
+        const float s1 = 2 * t4 + 1 < nvalid ? sacc[1] * zscale : -INFINITY;
         float cm = fmaxf(s0, s1);
         cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
         cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
         const float m_new = fmaxf(m_run, cm);
         const float alpha = fast_exp2(m_run - m_new);
-        const uint32_t pfrag = pack2<KVT>(fast_exp2(s0 - m_new), fast_exp2(s1 - m_new));
+        const uint32_t pfrag = pack2<MmaT>(fast_exp2(s0 - m_new), fast_exp2(s1 - m_new));
         // The sum uses the rounded weights that enter P V, so the weights of the output sum to one.
-        const float2 pr = unpack2<KVT>(pfrag);
+        const float2 pr = unpack2<MmaT>(pfrag);
         l_run = l_run * alpha + (pr.x + pr.y);
         m_run = m_new;
 #pragma unroll
@@ -542,12 +569,28 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         // V rows of tokens past the valid ones may hold anything (even NaN): zero their halves of the
         // B fragments (low half = token 2*t4, high half = token 2*t4 + 1).
         const uint32_t vmask = (2 * t4 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 1 < nvalid ? 0xffff0000u : 0u);
+        if constexpr (EB == 2) {
 #pragma unroll
-        for (int q4 = 0; q4 < S::kNBlocks / 4; ++q4) {
-          uint32_t vb[4];
-          ldmatrix_x4_trans(vbase + piece_offset<S>(lrow, q4 * 4 + (lane >> 3)), vb);
+          for (int q4 = 0; q4 < S::kNBlocks / 4; ++q4) {
+            uint32_t vb[4];
+            ldmatrix_x4_trans(vbase + piece_offset<S>(lrow, q4 * 4 + (lane >> 3)), vb);
 #pragma unroll
-          for (int j4 = 0; j4 < 4; ++j4) mma_1688<KVT>(o[q4 * 4 + j4], pfrag, 0u, vb[j4] & vmask);
+            for (int j4 = 0; j4 < 4; ++j4) mma_1688<MmaT>(o[q4 * 4 + j4], pfrag, 0u, vb[j4] & vmask);
+          }
+        } else {
+          // b0 of n-block nb = (V[token 2*t4][d], V[token 2*t4 + 1][d]) with d = nb*8 + lane/4.
+          const int g = lane >> 2;
+          const uint8_t* v0 = smem + Lay::kRing + slot * S::kStageBytes + S::kTileBytes + (cw * kStageTokens + 2 * t4) * 128;
+          const uint8_t* v1 = v0 + 128;
+          const int k0 = (2 * t4) & 7, k1 = (2 * t4 + 1) & 7;  // swizzle keys of the two rows
+#pragma unroll
+          for (int nb = 0; nb < S::kNBlocks; ++nb) {
+            const int byte = nb * 8 + g;
+            const uint32_t lo = v0[(((byte >> 4) ^ k0) << 4) | (byte & 15)];
+            const uint32_t hi = v1[(((byte >> 4) ^ k1) << 4) | (byte & 15)];
+            const uint32_t b0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo | (hi << 8)));
+            mma_1688<MmaT>(o[nb], pfrag, 0u, b0 & vmask);
+          }
         }
        }
       } else if (active) {
@@ -642,7 +685,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
         const int g = lane >> 2, t4 = lane & 3;
         if (g < inf.heads) {
-          float r = 1.0f / l_tot;
+          float r = ((EB == 1) ? args.v_scale[inf.kvh0 + cw] : 1.0f) / l_tot;
           if (poisoned) r = __int_as_float(0x7fc00000);
           const int h = (inf.kvh0 + cw) * args.group + inf.h_sub + g;
           if (inf.write_final) {

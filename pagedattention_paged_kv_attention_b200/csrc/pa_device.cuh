@@ -112,6 +112,12 @@ __device__ __forceinline__ float2 f16x2_to_float2(uint32_t w) {
   return __half22float2(h);
 }
 
+// Two E4M3 codes (low byte = first element) -> packed f16 pair, exact (one hardware conversion).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t w) {
+  __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w), __NV_E4M3);
+  return static_cast<uint32_t>(hr.x) | (static_cast<uint32_t>(hr.y) << 16);
+}
+
 // Two E4M3 codes (low byte = first element) -> two floats, exact (hardware conversion via f16).
 __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t w) {
   __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w), __NV_E4M3);
