@@ -281,6 +281,9 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     }
     const int bs = args.block_size;
     const int stages_per_part = args.partition_size / kStageTokens;
+    // K/V are read once per item: let L2 evict them first, keeping partial results, queries and
+    // block tables resident.
+    const uint64_t kv_policy = l2_policy_evict_first();
     bool aborted = false;
     int local = 0;   // CTA-local item sequence number
     int issued = 0;  // stages issued so far (ring position)
@@ -400,7 +403,8 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             __syncwarp();
             if (lane < 2 * S::kChunks) {
               uint8_t* dst = smem + Lay::kRing + slot * S::kStageBytes + op_kv * S::kTileBytes + op_ch * S::kChunkBytes;
-              tma_load_4d(dst, op_kv ? &tmap_v : &tmap_k, &full[slot], op_ch * S::kChunkElems, t0 % bs, kvh0, blk);
+              tma_load_4d_hint(dst, op_kv ? &tmap_v : &tmap_k, &full[slot], op_ch * S::kChunkElems, t0 % bs, kvh0, blk,
+                               kv_policy);
             }
             ++issued;
           }
@@ -476,9 +480,11 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
               qa[ks][0] = row_ok ? *reinterpret_cast<const uint32_t*>(qs + g * D + ks * 16 + 2 * t4) : 0u;
               qa[ks][1] = row_ok ? *reinterpret_cast<const uint32_t*>(qs + g * D + ks * 16 + 8 + 2 * t4) : 0u;
             } else {
-              const QT* qrow = qs + g * D + ks * 16 + 2 * t4;
+              // FP8 K fragments come from ldmatrix over byte rows (see the stage code): step ks holds
+              // d = 16*ks + 4*t4 + {0,1} in b0 and + {2,3} in b1, so the query uses the same order.
+              const QT* qrow = qs + g * D + ks * 16 + 4 * t4;
               qa[ks][0] = row_ok ? pack2<__half>(to_f32(qrow[0]), to_f32(qrow[1])) : 0u;
-              qa[ks][1] = row_ok ? pack2<__half>(to_f32(qrow[8]), to_f32(qrow[9])) : 0u;
+              qa[ks][1] = row_ok ? pack2<__half>(to_f32(qrow[2]), to_f32(qrow[3])) : 0u;
             }
           }
 #pragma unroll
@@ -534,17 +540,22 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             mma_16816<MmaT>(sacc, a1, kb[2], kb[3]);
           }
         } else {
-          // FP8 rows are 128 bytes (one swizzle chunk): B fragment b0 of step ks is the byte pair
-          // (ks*16 + 2*t4, +1) of token row lane/4, b1 the pair 8 bytes further.
-          const int tok = lane >> 2;
-          const uint8_t* krow = smem + Lay::kRing + slot * S::kStageBytes + (cw * kStageTokens + tok) * 128;
+          // FP8 rows are 128 bytes (one swizzle chunk, 16-byte unit u = 16 values of d). ldmatrix over
+          // the byte rows gives lane (g, t4) the 4 bytes d = 16u + 4*t4 + {0..3} of token g; the low
+          // pair becomes b0 and the high pair b1 after widening to f16.
+          static_assert(D == 128, "FP8 caches need head_size 128");
+          const uint32_t kaddr = kbase + lrow * 128;
 #pragma unroll
-          for (int ks = 0; ks < S::kKSteps; ++ks) {
-            const uint8_t* unit = krow + ((ks ^ tok) << 4) + 2 * t4;
-            const uint32_t b0 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(unit));
-            const uint32_t b1 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(unit + 8));
-            const uint32_t a[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
-            mma_16816<MmaT>(sacc, a, b0, b1);
+          for (int q4 = 0; q4 < S::kKSteps / 4; ++q4) {
+            uint32_t kb[4];
+            ldmatrix_x4(kaddr + (((q4 * 4 + (lane >> 3)) ^ (lane & 7)) << 4), kb);
+#pragma unroll
+            for (int j4 = 0; j4 < 4; ++j4) {
+              const uint32_t b0 = e4m3x2_to_f16x2(static_cast<uint16_t>(kb[j4] & 0xffffu));
+              const uint32_t b1 = e4m3x2_to_f16x2(static_cast<uint16_t>(kb[j4] >> 16));
+              const uint32_t a[4] = {qa[q4 * 4 + j4][0], 0u, qa[q4 * 4 + j4][1], 0u};
+              mma_16816<MmaT>(sacc, a, b0, b1);
+            }
           }
         }
         // Scores of query head lane/4 for tokens 2*t4 and 2*t4 + 1.
@@ -578,18 +589,23 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             for (int j4 = 0; j4 < 4; ++j4) mma_1688<MmaT>(o[q4 * 4 + j4], pfrag, 0u, vb[j4] & vmask);
           }
         } else {
-          // b0 of n-block nb = (V[token 2*t4][d], V[token 2*t4 + 1][d]) with d = nb*8 + lane/4.
-          const int g = lane >> 2;
-          const uint8_t* v0 = smem + Lay::kRing + slot * S::kStageBytes + S::kTileBytes + (cw * kStageTokens + 2 * t4) * 128;
-          const uint8_t* v1 = v0 + 128;
-          const int k0 = (2 * t4) & 7, k1 = (2 * t4 + 1) & 7;  // swizzle keys of the two rows
+          // ldmatrix.trans over the byte rows gives lane (g, t4) the bytes
+          // [V[2t4][16u+2g], V[2t4][16u+2g+1], V[2t4+1][16u+2g], V[2t4+1][16u+2g+1]]; one byte permute
+          // splits them into the even-d fragment (block 2u: d = 16u + 2g) and the odd-d fragment
+          // (block 2u + 1: d = 16u + 2g + 1).
+          const uint32_t vaddr = vbase + lrow * 128;
 #pragma unroll
-          for (int nb = 0; nb < S::kNBlocks; ++nb) {
-            const int byte = nb * 8 + g;
-            const uint32_t lo = v0[(((byte >> 4) ^ k0) << 4) | (byte & 15)];
-            const uint32_t hi = v1[(((byte >> 4) ^ k1) << 4) | (byte & 15)];
-            const uint32_t b0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo | (hi << 8)));
-            mma_1688<MmaT>(o[nb], pfrag, 0u, b0 & vmask);
+          for (int q4 = 0; q4 < S::kNBlocks / 8; ++q4) {
+            uint32_t vb[4];
+            ldmatrix_x4_trans(vaddr + (((q4 * 4 + (lane >> 3)) ^ (lane & 7)) << 4), vb);
+#pragma unroll
+            for (int j4 = 0; j4 < 4; ++j4) {
+              const int u = q4 * 4 + j4;
+              const uint32_t ev = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb[j4], 0u, 0x4420u)));
+              const uint32_t od = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb[j4], 0u, 0x4431u)));
+              mma_1688<MmaT>(o[2 * u], pfrag, 0u, ev & vmask);
+              mma_1688<MmaT>(o[2 * u + 1], pfrag, 0u, od & vmask);
+            }
           }
         }
        }
@@ -688,17 +704,32 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           float r = ((EB == 1) ? args.v_scale[inf.kvh0 + cw] : 1.0f) / l_tot;
           if (poisoned) r = __int_as_float(0x7fc00000);
           const int h = (inf.kvh0 + cw) * args.group + inf.h_sub + g;
+          const size_t rowi = (static_cast<size_t>(inf.s) * args.num_heads + h) * args.num_partitions + inf.part;
           if (inf.write_final) {
-            QT* out = static_cast<QT*>(args.out) + (static_cast<size_t>(inf.s) * args.num_heads + h) * D + 2 * t4;
+            QT* out = static_cast<QT*>(args.out) + (static_cast<size_t>(inf.s) * args.num_heads + h) * D;
+            if constexpr (EB == 2) {
 #pragma unroll
-            for (int nb = 0; nb < S::kNBlocks; ++nb)
-              *reinterpret_cast<uint32_t*>(out + nb * 8) = pack2<QT>(o[nb][0] * r, o[nb][1] * r);
+              for (int nb = 0; nb < S::kNBlocks; ++nb)
+                *reinterpret_cast<uint32_t*>(out + nb * 8 + 2 * t4) = pack2<QT>(o[nb][0] * r, o[nb][1] * r);
+            } else {
+              // Blocks 2u (even d) and 2u + 1 (odd d) together hold d = 16u + 4*t4 + {0, 1, 2, 3}.
+#pragma unroll
+              for (int u = 0; u < S::kNBlocks / 2; ++u)
+                *reinterpret_cast<uint2*>(out + u * 16 + 4 * t4) =
+                    pack4<QT>(o[2 * u][0] * r, o[2 * u + 1][0] * r, o[2 * u][1] * r, o[2 * u + 1][1] * r);
+            }
           } else {
-            const size_t rowi = (static_cast<size_t>(inf.s) * args.num_heads + h) * args.num_partitions + inf.part;
-            float* po = args.part_o + rowi * D + 2 * t4;
+            float* po = args.part_o + rowi * D;
+            if constexpr (EB == 2) {
 #pragma unroll
-            for (int nb = 0; nb < S::kNBlocks; ++nb)
-              *reinterpret_cast<float2*>(po + nb * 8) = make_float2(o[nb][0] * r, o[nb][1] * r);
+              for (int nb = 0; nb < S::kNBlocks; ++nb)
+                *reinterpret_cast<float2*>(po + nb * 8 + 2 * t4) = make_float2(o[nb][0] * r, o[nb][1] * r);
+            } else {
+#pragma unroll
+              for (int u = 0; u < S::kNBlocks / 2; ++u)
+                *reinterpret_cast<float4*>(po + u * 16 + 4 * t4) =
+                    make_float4(o[2 * u][0] * r, o[2 * u + 1][0] * r, o[2 * u][1] * r, o[2 * u + 1][1] * r);
+            }
             if (t4 == 0) {
               args.part_m[rowi] = m_run;
               args.part_l[rowi] = l_tot;
@@ -765,30 +796,52 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
 }
 
 // Split-K merge of partitions: out = sum_p w_p o_p / sum_p w_p with w_p = l_p 2^(m_p - max m).
-// One CTA of D threads per (query head, sequence); sequences with one partition (or an empty or
-// invalid context) were finished by the main kernel.
+// One warp per (sequence, query head): lanes hold 4 (or 2) consecutive elements of the row and walk
+// the partitions; the partition statistics are read once per lane group. Sequences with one
+// partition (or an empty or invalid context) were finished by the main kernel.
+constexpr int kReduceWarps = 4;
 template <typename QT, int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(kReduceWarps * 32)
 paged_attention_reduce(const AttnArgs args) {
-  const int h = blockIdx.x;
-  const int s = blockIdx.y;
-  const int i = threadIdx.x;
+  constexpr int kPer = D / 32;  // elements per lane: 4 for d = 128, 2 for d = 64
+  const int lane = threadIdx.x & 31;
+  const long row = static_cast<long>(blockIdx.x) * kReduceWarps + (threadIdx.x >> 5);
+  if (row >= static_cast<long>(args.num_seqs) * args.num_heads) return;
+  const int s = static_cast<int>(row / args.num_heads);
   const int L = args.context_lens[s];
   const int PS = args.partition_size;
   if (L <= 0 || context_len_invalid(L, args)) return;
   const int n_parts = (L + PS - 1) / PS;
   if (n_parts <= 1) return;
-  const size_t base = (static_cast<size_t>(s) * args.num_heads + h) * args.num_partitions;
+  const size_t base = static_cast<size_t>(row) * args.num_partitions;
   float M = -INFINITY;
-  for (int p = 0; p < n_parts; ++p) M = fmaxf(M, args.part_m[base + p]);
-  float wsum = 0.f, o = 0.f;
+  for (int p = lane; p < n_parts; p += 32) M = fmaxf(M, args.part_m[base + p]);
+#pragma unroll
+  for (int b = 16; b > 0; b >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, b));
+  float wsum = 0.f;
+  float acc[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
+  const float* po = args.part_o + base * D + lane * kPer;
+#pragma unroll 4
   for (int p = 0; p < n_parts; ++p) {
     const float w = args.part_l[base + p] * fast_exp2(args.part_m[base + p] - M);
     wsum += w;
-    o += w * args.part_o[(base + p) * D + i];
+    if constexpr (kPer == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(po + static_cast<size_t>(p) * D);
+      acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(po + static_cast<size_t>(p) * D);
+      acc[0] += w * v.x; acc[1] += w * v.y;
+    }
   }
-  QT* out = static_cast<QT*>(args.out) + (static_cast<size_t>(s) * args.num_heads + h) * D;
-  out[i] = QT(o / wsum);
+  const float r = 1.0f / wsum;
+  QT* out = static_cast<QT*>(args.out) + static_cast<size_t>(row) * D + lane * kPer;
+  if constexpr (kPer == 4) {
+    *reinterpret_cast<uint2*>(out) = pack4<QT>(acc[0] * r, acc[1] * r, acc[2] * r, acc[3] * r);
+  } else {
+    *reinterpret_cast<uint32_t*>(out) = pack2<QT>(acc[0] * r, acc[1] * r);
+  }
 }
 
 }  // namespace pa

@@ -23,7 +23,9 @@ cudaError_t launch_attention_one(const CUtensorMap& tk, const CUtensorMap& tv, c
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.num_partitions > 1) {
-    paged_attention_reduce<QT, D><<<dim3(a.num_heads, a.num_seqs), D, 0, stream>>>(a);
+    const long rows = static_cast<long>(a.num_heads) * a.num_seqs;
+    paged_attention_reduce<QT, D>
+        <<<static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps), kReduceWarps * 32, 0, stream>>>(a);
     e = cudaGetLastError();
   }
   return e;
