@@ -214,10 +214,17 @@ def main():
     ap.add_argument("--partition-size", type=int, default=None,
                     help="tokens per split-K partition (default: the workload's, else the library's choice)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--num-seqs", type=int, default=None,
+                    help="smaller batch of the same workload (profiling cases); default: the workload's")
+    ap.add_argument("--pool-blocks", type=int, default=None,
+                    help="override the pool size in blocks (profiling cases that must stay small)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     cfg = W.CONFIGS[args.workload]
+    if args.pool_blocks is not None:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, num_blocks=args.pool_blocks)
     if args.partition_size is None:
         args.partition_size = cfg.partition_size
     world, rank, local = dist_setup(args)
@@ -232,7 +239,7 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    w = W.make_workload(cfg, seed=cfg.seed + 1000 * rank, device=dev)
+    w = W.make_workload(cfg, seed=cfg.seed + 1000 * rank, device=dev, num_seqs=args.num_seqs)
     S, H, d = w.query.shape
     kv_bytes = 1 if cfg.kv_dtype == "fp8_e4m3" else 2
     ks = vs = None

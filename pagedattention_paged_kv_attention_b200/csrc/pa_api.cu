@@ -98,7 +98,7 @@ bool encode_cache_map(CUtensorMap* map, const void* cache, int elem_bytes, int h
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_size), static_cast<cuuint64_t>(block_size),
                         static_cast<cuuint64_t>(num_kv_heads), static_cast<cuuint64_t>(num_blocks)};
   cuuint64_t strides[3] = {num_kv_heads * head_size * e, head_size * e, block_size * num_kv_heads * head_size * e};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(pa::kStageTokens),
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(pa::kBoxTokens),
                        static_cast<cuuint32_t>(pa::kHeadBlock), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = encode(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,

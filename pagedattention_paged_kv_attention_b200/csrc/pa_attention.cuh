@@ -51,8 +51,9 @@ namespace pa {
 
 constexpr int kHeadBlock = 8;            // kv heads per work item (one consumer warp each)
 constexpr int kConsumerWarps = kHeadBlock;
-constexpr int kStageTokens = 8;          // tokens per pipeline stage (block_size >= 8)
-constexpr int kStages = 4;               // ring depth
+constexpr int kBoxTokens = 8;            // tokens per TMA box (block_size >= 8); one swizzle atom
+constexpr int kMaxStages = 8;            // ring depth cap (the depth itself is per variant, see Layout)
+constexpr int kSmemBudget = 200 * 1024;  // shared memory the layout may use (of 227 KB per CTA)
 constexpr int kQueryBuffers = 2;
 constexpr int kIdWindow = 4;             // block ids prefetched per item: 32 * kIdWindow stages
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
@@ -112,14 +113,18 @@ struct Shape {
   static constexpr int kLog2G = ilog2(G);
   static constexpr int kTPI = 32 / kNS;                  // tokens per QK step
   static constexpr int kNPL = kPiecesPerRow / kNS;       // pieces per lane
-  static constexpr int kIters = kStageTokens / kTPI;
+  // A stage is kGroups boxes of 8 tokens: 8 for 16-bit caches, 16 for FP8 (same bytes per stage).
+  static constexpr int kGroups = (EB == 1) ? 2 : 1;
+  static constexpr int kTS = kBoxTokens * kGroups;      // tokens per stage
+  static constexpr int kIters = kTS / kTPI;
   static constexpr int kTsShift = kLog2NS;               // token-slot lane bits sit above the ds bits
   // PV mapping: LPT lanes per token.
   static constexpr int kLPT = D / 8;
   static constexpr int kLog2LPT = ilog2(kLPT);
   static constexpr int kTPV = 32 / kLPT;
-  // One stage: [K|V][chunk][head][token][128 B].
-  static constexpr int kChunkBytes = kStageTokens * kHeadBlock * 128;
+  // One stage: [K|V][chunk][group][head][8 tokens][128 B]; tile row r = group*64 + head*8 + token%8.
+  static constexpr int kBoxBytes = kBoxTokens * kHeadBlock * 128;
+  static constexpr int kChunkBytes = kGroups * kBoxBytes;
   static constexpr int kTileBytes = kChunks * kChunkBytes;
   static constexpr int kStageBytes = 2 * kTileBytes;
   // Tensor-core path: at least two query heads per kv head. FP8 caches enter the tensor cores as
@@ -148,12 +153,16 @@ struct ItemInfo {
 template <typename QT, int D, int G, int EB>
 struct Layout {
   using S = Shape<D, G, EB>;
+  static constexpr int kQueryOne = kHeadBlock * G * D * int(sizeof(QT));       // [8 kv heads][G][D]
+  static constexpr int kSmall = kConsumerWarps * S::kTS * G * 4 + kConsumerWarps * G * 4 + 1024;
+  // Ring depth: as many stages as the budget leaves after the query buffers and small tables.
+  static constexpr int kStages = cmin(kMaxStages, (kSmemBudget - kQueryBuffers * kQueryOne - kSmall) / S::kStageBytes);
+  static_assert(kStages >= 2, "ring too shallow");
   static constexpr int kRing = 0;
   static constexpr int kRingBytes = kStages * S::kStageBytes;
-  static constexpr int kQueryOne = kHeadBlock * G * D * int(sizeof(QT));       // [8 kv heads][G][D]
   static constexpr int kQuery = kRingBytes;
   static constexpr int kPbuf = kQuery + kQueryBuffers * kQueryOne;             // [W][TS][G] f32
-  static constexpr int kAbuf = kPbuf + kConsumerWarps * kStageTokens * G * 4;  // [W][G] f32
+  static constexpr int kAbuf = kPbuf + kConsumerWarps * S::kTS * G * 4;      // [W][G] f32
   static constexpr int kMsgs = (kAbuf + kConsumerWarps * G * 4 + 15) / 16 * 16;
   static constexpr int kInfo = kMsgs + kStages * int(sizeof(StageMsg));
   static constexpr int kBars = (kInfo + kQueryBuffers * int(sizeof(ItemInfo)) + 7) / 8 * 8;
@@ -164,9 +173,11 @@ struct Layout {
   static_assert(kAllocBytes <= 227 * 1024, "shared memory layout too large");
 };
 
-// Byte offset of piece `pc` (8 elements) of tile row r = head * 8 + token inside a
-// [chunk][8 heads * kStageTokens rows][128 B] tile written by TMA with the 128-byte swizzle (16-byte
-// unit u of row r lives at unit u ^ (r & 7) = u ^ token).
+// Tile row of token t (within the stage) of kv head `head`: boxes of 8 tokens, each [head][token].
+__device__ __forceinline__ int tile_row(int head, int t) { return (t >> 3) * (kHeadBlock * kBoxTokens) + head * kBoxTokens + (t & 7); }
+
+// Byte offset of piece `pc` (8 elements) of tile row r inside a [chunk][rows][128 B] tile written by
+// TMA with the 128-byte swizzle (16-byte unit u of row r lives at unit u ^ (r & 7) = u ^ (token % 8)).
 template <class S>
 __device__ __forceinline__ uint32_t piece_offset(int r, int pc) {
   const int byte = pc * S::kPieceBytes;
@@ -245,6 +256,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
   using Lay = Layout<QT, D, G, EB>;
   using Piece = typename Elem<KVT>::Piece;
   using MmaT = typename std::conditional<EB == 2, KVT, __half>::type;  // tensor-core input type
+  constexpr int kStages = Lay::kStages;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -280,7 +292,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
       tma_prefetch_desc(&tmap_v);
     }
     const int bs = args.block_size;
-    const int stages_per_part = args.partition_size / kStageTokens;
+    const int boxes_per_part = args.partition_size / kBoxTokens;
     // K/V are read once per item: let L2 evict them first, keeping partial results, queries and
     // block tables resident.
     const uint64_t kv_policy = l2_policy_evict_first();
@@ -289,7 +301,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     int issued = 0;  // stages issued so far (ring position)
 
     // Items flow through a two-deep software pipeline: while item i streams, the loads describing item
-    // i+1 (its context length and a window of its block ids, one id per lane per 32 stages) are in
+    // i+1 (its context length and a window of its block ids, one id per lane per 32 boxes) are in
     // flight, and the work counter has already been asked for item i+2. All state is in registers.
     unsigned int cur_idx = 0, nxt_idx = 0;
     int cur_L = 0, nxt_L = 0;
@@ -301,7 +313,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
       LV = __ldg(args.context_lens + pc_.s);                                                           \
       const int32_t* row_ = args.block_tables + static_cast<size_t>(pc_.s) * args.max_blocks_per_seq;  \
       _Pragma("unroll") for (int j_ = 0; j_ < kIdWindow; ++j_) {                                       \
-        const int entry_ = ((pc_.part * stages_per_part + j_ * 32 + lane) * kStageTokens) / bs;        \
+        const int entry_ = ((pc_.part * boxes_per_part + j_ * 32 + lane) * kBoxTokens) / bs;           \
         IDS[j_] = entry_ < args.max_blocks_per_seq ? __ldg(row_ + entry_) : 0;                         \
       }                                                                                                \
     }                                                                                                  \
@@ -337,7 +349,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         } else {
           const int tok_begin = c.part * args.partition_size;
           const int tok_end = cmin(L, tok_begin + args.partition_size);
-          const int n_stages = (tok_end - tok_begin + kStageTokens - 1) / kStageTokens;
+          const int n_stages = (tok_end - tok_begin + S::kTS - 1) / S::kTS;
           const int qb = local % kQueryBuffers;
           // Query rows of the item's heads, and the item description.
           bool ok = true;
@@ -368,21 +380,28 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           }
 
           const int32_t* row = args.block_tables + static_cast<size_t>(c.s) * args.max_blocks_per_seq;
-          // TMA ops of one stage are spread over lanes: lane = kv * kChunks + chunk.
-          const int op_kv = lane / S::kChunks;
+          // TMA ops of one stage are spread over lanes: lane = (box * 2 + kv) * kChunks + chunk.
+          const int op_box = lane / (2 * S::kChunks);
+          const int op_kv = (lane / S::kChunks) & 1;
           const int op_ch = lane % S::kChunks;
           for (int k = 0; k < n_stages; ++k) {
-            const int t0 = tok_begin + k * kStageTokens;
-            const int ntok = cmin(kStageTokens, tok_end - t0);
+            const int t0 = tok_begin + k * S::kTS;
+            const int ntok = cmin(S::kTS, tok_end - t0);
+            const int nbox = (ntok + kBoxTokens - 1) / kBoxTokens;
+            // Block id of this lane's box: item-relative box rel sits in window register rel >> 5 of
+            // lane rel & 31.
+            const int rel = k * S::kGroups + (op_box < S::kGroups ? op_box : 0);
             int blk = 0;
 #pragma unroll
             for (int j = 0; j < kIdWindow; ++j) {
-              const int v = __shfl_sync(0xffffffffu, cur_ids[j], k & 31);
-              if ((k >> 5) == j) blk = v;
+              const int v = __shfl_sync(0xffffffffu, cur_ids[j], rel & 31);
+              if ((rel >> 5) == j) blk = v;
             }
-            if (k >= kIdWindow * 32) blk = __ldg(row + t0 / bs);  // beyond the prefetched window
-            const bool bad = blk < 0 || blk >= args.num_blocks;
+            const bool mine = op_box < nbox;  // this lane issues a TMA op for this stage
+            if (rel >= kIdWindow * 32 && mine) blk = __ldg(row + (t0 + op_box * kBoxTokens) / bs);  // beyond the window
+            bool bad = mine && (blk < 0 || blk >= args.num_blocks);
             if (bad) blk = args.num_blocks;  // out-of-range coordinate: TMA fills the box with zeros
+            bad = __any_sync(0xffffffffu, bad);
             const int slot = issued % kStages;
             bool ok2 = true;
             if (lane == 0) ok2 = mbar_wait(&empty[slot], (static_cast<uint32_t>(issued / kStages) & 1u) ^ 1u, err);
@@ -398,13 +417,14 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
               m.pad = 0;
               msgs[slot] = m;
               if (bad) atomicOr(err, PA_DEVERR_BLOCK_ID);
-              mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(S::kStageBytes));
+              mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nbox * 2 * S::kChunks * S::kBoxBytes));
             }
             __syncwarp();
-            if (lane < 2 * S::kChunks) {
-              uint8_t* dst = smem + Lay::kRing + slot * S::kStageBytes + op_kv * S::kTileBytes + op_ch * S::kChunkBytes;
-              tma_load_4d_hint(dst, op_kv ? &tmap_v : &tmap_k, &full[slot], op_ch * S::kChunkElems, t0 % bs, kvh0, blk,
-                               kv_policy);
+            if (mine && lane < 2 * S::kChunks * S::kGroups) {
+              uint8_t* dst = smem + Lay::kRing + slot * S::kStageBytes + op_kv * S::kTileBytes + op_ch * S::kChunkBytes +
+                             op_box * S::kBoxBytes;
+              tma_load_4d_hint(dst, op_kv ? &tmap_v : &tmap_k, &full[slot], op_ch * S::kChunkElems,
+                               (t0 + op_box * kBoxTokens) % bs, kvh0, blk, kv_policy);
             }
             ++issued;
           }
@@ -442,7 +462,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     const bool primary = (ds & ((S::kNS >> S::kLog2G) - 1)) == 0;      // first of the duplicate lanes
     const int dp = lane & (S::kLPT - 1);
     const int vslot = lane >> S::kLog2LPT;
-    float* pw = reinterpret_cast<float*>(smem + Lay::kPbuf) + cw * kStageTokens * G;
+    float* pw = reinterpret_cast<float*>(smem + Lay::kPbuf) + cw * S::kTS * G;
     float* aw = reinterpret_cast<float*>(smem + Lay::kAbuf) + cw * G;
 
     float2 qr[G][S::kNPL][4];
@@ -522,55 +542,71 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
       if constexpr (S::kMma) {
        if (active) {
         // ---------------- tensor-core stage ----------------
+        constexpr int NG = S::kGroups;
         const int nvalid = m.ntok;
         const uint32_t kbase = smem_u32(smem + Lay::kRing + slot * S::kStageBytes);
         const uint32_t vbase = kbase + S::kTileBytes;
         const int t4 = lane & 3;
-        // ldmatrix row addresses: lane i points at token row i % 8 of this head, 16-byte unit i / 8.
-        const int lrow = cw * kStageTokens + (lane & 7);
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (EB == 2) {
+        // ldmatrix row addresses: lane i points at token row i % 8 of this head (in box gr), unit i / 8.
+        float sacc[NG][4];
 #pragma unroll
-          for (int q4 = 0; q4 < S::kKSteps / 2; ++q4) {
-            uint32_t kb[4];
-            ldmatrix_x4(kbase + piece_offset<S>(lrow, q4 * 4 + (lane >> 3)), kb);
-            const uint32_t a0[4] = {qa[2 * q4][0], 0u, qa[2 * q4][1], 0u};
-            mma_16816<MmaT>(sacc, a0, kb[0], kb[1]);
-            const uint32_t a1[4] = {qa[2 * q4 + 1][0], 0u, qa[2 * q4 + 1][1], 0u};
-            mma_16816<MmaT>(sacc, a1, kb[2], kb[3]);
-          }
-        } else {
-          // FP8 rows are 128 bytes (one swizzle chunk, 16-byte unit u = 16 values of d). ldmatrix over
-          // the byte rows gives lane (g, t4) the 4 bytes d = 16u + 4*t4 + {0..3} of token g; the low
-          // pair becomes b0 and the high pair b1 after widening to f16.
-          static_assert(D == 128, "FP8 caches need head_size 128");
-          const uint32_t kaddr = kbase + lrow * 128;
+        for (int gr = 0; gr < NG; ++gr) {
+          sacc[gr][0] = sacc[gr][1] = sacc[gr][2] = sacc[gr][3] = 0.f;
+          const int lrow = tile_row(cw, gr * kBoxTokens + (lane & 7));
+          if constexpr (EB == 2) {
 #pragma unroll
-          for (int q4 = 0; q4 < S::kKSteps / 4; ++q4) {
-            uint32_t kb[4];
-            ldmatrix_x4(kaddr + (((q4 * 4 + (lane >> 3)) ^ (lane & 7)) << 4), kb);
+            for (int q4 = 0; q4 < S::kKSteps / 2; ++q4) {
+              uint32_t kb[4];
+              ldmatrix_x4(kbase + piece_offset<S>(lrow, q4 * 4 + (lane >> 3)), kb);
+              const uint32_t a0[4] = {qa[2 * q4][0], 0u, qa[2 * q4][1], 0u};
+              mma_16816<MmaT>(sacc[gr], a0, kb[0], kb[1]);
+              const uint32_t a1[4] = {qa[2 * q4 + 1][0], 0u, qa[2 * q4 + 1][1], 0u};
+              mma_16816<MmaT>(sacc[gr], a1, kb[2], kb[3]);
+            }
+          } else {
+            // FP8 rows are 128 bytes (one swizzle chunk, 16-byte unit u = 16 values of d). ldmatrix
+            // over the byte rows gives lane (g, t4) the 4 bytes d = 16u + 4*t4 + {0..3} of token g; the
+            // low pair becomes b0 and the high pair b1 after widening to f16.
+            static_assert(D == 128, "FP8 caches need head_size 128");
+            const uint32_t kaddr = kbase + lrow * 128;
 #pragma unroll
-            for (int j4 = 0; j4 < 4; ++j4) {
-              const uint32_t b0 = e4m3x2_to_f16x2(static_cast<uint16_t>(kb[j4] & 0xffffu));
-              const uint32_t b1 = e4m3x2_to_f16x2(static_cast<uint16_t>(kb[j4] >> 16));
-              const uint32_t a[4] = {qa[q4 * 4 + j4][0], 0u, qa[q4 * 4 + j4][1], 0u};
-              mma_16816<MmaT>(sacc, a, b0, b1);
+            for (int q4 = 0; q4 < S::kKSteps / 4; ++q4) {
+              uint32_t kb[4];
+              ldmatrix_x4(kaddr + (((q4 * 4 + (lane >> 3)) ^ (lane & 7)) << 4), kb);
+#pragma unroll
+              for (int j4 = 0; j4 < 4; ++j4) {
+                const uint32_t b0 = e4m3x2_to_f16x2(static_cast<uint16_t>(kb[j4] & 0xffffu));
+                const uint32_t b1 = e4m3x2_to_f16x2(static_cast<uint16_t>(kb[j4] >> 16));
+                const uint32_t a[4] = {qa[q4 * 4 + j4][0], 0u, qa[q4 * 4 + j4][1], 0u};
+                mma_16816<MmaT>(sacc[gr], a, b0, b1);
+              }
             }
           }
         }
-        // Scores of query head lane/4 for tokens 2*t4 and 2*t4 + 1.
+        // Scores of query head lane/4 for tokens 8*gr + 2*t4 and 8*gr + 2*t4 + 1.
         const float zscale = (EB == 1) ? args.scale_log2 * args.k_scale[inf.kvh0 + cw] : args.scale_log2;
-        const float s0 = 2 * t4 < nvalid ? sacc[0] * zscale : -INFINITY;
-        const float s1 = 2 * t4 + 1 < nvalid ? sacc[1] * zscale : -INFINITY;
-        float cm = fmaxf(s0, s1);
+        float sv[NG][2];
+        float cm = -INFINITY;
+#pragma unroll
+        for (int gr = 0; gr < NG; ++gr) {
+          sv[gr][0] = gr * kBoxTokens + 2 * t4 < nvalid ? sacc[gr][0] * zscale : -INFINITY;
+          sv[gr][1] = gr * kBoxTokens + 2 * t4 + 1 < nvalid ? sacc[gr][1] * zscale : -INFINITY;
+          cm = fmaxf(cm, fmaxf(sv[gr][0], sv[gr][1]));
+        }
         cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
         cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
         const float m_new = fmaxf(m_run, cm);
         const float alpha = fast_exp2(m_run - m_new);
-        const uint32_t pfrag = pack2<MmaT>(fast_exp2(s0 - m_new), fast_exp2(s1 - m_new));
-        // The sum uses the rounded weights that enter P V, so the weights of the output sum to one.
-        const float2 pr = unpack2<MmaT>(pfrag);
-        l_run = l_run * alpha + (pr.x + pr.y);
+        uint32_t pfrag[NG];
+        float psum = 0.f;
+#pragma unroll
+        for (int gr = 0; gr < NG; ++gr) {
+          pfrag[gr] = pack2<MmaT>(fast_exp2(sv[gr][0] - m_new), fast_exp2(sv[gr][1] - m_new));
+          // The sum uses the rounded weights that enter P V, so the weights of the output sum to one.
+          const float2 pr = unpack2<MmaT>(pfrag[gr]);
+          psum += pr.x + pr.y;
+        }
+        l_run = l_run * alpha + psum;
         m_run = m_new;
 #pragma unroll
         for (int nb = 0; nb < S::kNBlocks; ++nb) {
@@ -578,33 +614,46 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           o[nb][1] *= alpha;
         }
         // V rows of tokens past the valid ones may hold anything (even NaN): zero their halves of the
-        // B fragments (low half = token 2*t4, high half = token 2*t4 + 1).
-        const uint32_t vmask = (2 * t4 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 1 < nvalid ? 0xffff0000u : 0u);
+        // B fragments (low half = token 2*t4, high half = token 2*t4 + 1 of each box).
+        uint32_t vmask[NG];
+#pragma unroll
+        for (int gr = 0; gr < NG; ++gr)
+          vmask[gr] = (gr * kBoxTokens + 2 * t4 < nvalid ? 0x0000ffffu : 0u) |
+                      (gr * kBoxTokens + 2 * t4 + 1 < nvalid ? 0xffff0000u : 0u);
         if constexpr (EB == 2) {
+          static_assert(NG == 1, "16-bit caches use one box per stage");
+          const int lrow = tile_row(cw, lane & 7);
 #pragma unroll
           for (int q4 = 0; q4 < S::kNBlocks / 4; ++q4) {
             uint32_t vb[4];
             ldmatrix_x4_trans(vbase + piece_offset<S>(lrow, q4 * 4 + (lane >> 3)), vb);
 #pragma unroll
-            for (int j4 = 0; j4 < 4; ++j4) mma_1688<MmaT>(o[q4 * 4 + j4], pfrag, 0u, vb[j4] & vmask);
+            for (int j4 = 0; j4 < 4; ++j4) mma_1688<MmaT>(o[q4 * 4 + j4], pfrag[0], 0u, vb[j4] & vmask[0]);
           }
         } else {
-          // ldmatrix.trans over the byte rows gives lane (g, t4) the bytes
+          // ldmatrix.trans over the byte rows of box gr gives lane (g, t4) the bytes
           // [V[2t4][16u+2g], V[2t4][16u+2g+1], V[2t4+1][16u+2g], V[2t4+1][16u+2g+1]]; one byte permute
           // splits them into the even-d fragment (block 2u: d = 16u + 2g) and the odd-d fragment
-          // (block 2u + 1: d = 16u + 2g + 1).
-          const uint32_t vaddr = vbase + lrow * 128;
+          // (block 2u + 1: d = 16u + 2g + 1). The two boxes are the two k-halves of an m16n8k16 step.
+          static_assert(NG == 2, "FP8 caches use two boxes per stage");
+          const uint32_t a[4] = {pfrag[0], 0u, pfrag[1], 0u};
+          const uint32_t vaddr0 = vbase + tile_row(cw, lane & 7) * 128;
+          const uint32_t vaddr1 = vbase + tile_row(cw, kBoxTokens + (lane & 7)) * 128;
 #pragma unroll
           for (int q4 = 0; q4 < S::kNBlocks / 8; ++q4) {
-            uint32_t vb[4];
-            ldmatrix_x4_trans(vaddr + (((q4 * 4 + (lane >> 3)) ^ (lane & 7)) << 4), vb);
+            const uint32_t off = ((q4 * 4 + (lane >> 3)) ^ (lane & 7)) << 4;
+            uint32_t vb0[4], vb1[4];
+            ldmatrix_x4_trans(vaddr0 + off, vb0);
+            ldmatrix_x4_trans(vaddr1 + off, vb1);
 #pragma unroll
             for (int j4 = 0; j4 < 4; ++j4) {
               const int u = q4 * 4 + j4;
-              const uint32_t ev = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb[j4], 0u, 0x4420u)));
-              const uint32_t od = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb[j4], 0u, 0x4431u)));
-              mma_1688<MmaT>(o[2 * u], pfrag, 0u, ev & vmask);
-              mma_1688<MmaT>(o[2 * u + 1], pfrag, 0u, od & vmask);
+              const uint32_t ev0 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb0[j4], 0u, 0x4420u))) & vmask[0];
+              const uint32_t ev1 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb1[j4], 0u, 0x4420u))) & vmask[1];
+              const uint32_t od0 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb0[j4], 0u, 0x4431u))) & vmask[0];
+              const uint32_t od1 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb1[j4], 0u, 0x4431u))) & vmask[1];
+              mma_16816<MmaT>(o[2 * u], a, ev0, ev1);
+              mma_16816<MmaT>(o[2 * u + 1], a, od0, od1);
             }
           }
         }
@@ -624,7 +673,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
 #pragma unroll
           for (int jj = 0; jj < S::kNPL; ++jj) {
             const int pc = qk_piece<S, EB>(jj, ds, tslot);
-            const Piece kp = *reinterpret_cast<const Piece*>(ktile + piece_offset<S>(cw * kStageTokens + t, pc));
+            const Piece kp = *reinterpret_cast<const Piece*>(ktile + piece_offset<S>(tile_row(cw, t), pc));
             float2 kf[4];
             Elem<KVT>::to_float(kp, kf);
 #pragma unroll
@@ -665,10 +714,10 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           for (int k = 0; k < 4; ++k) acc[g][k] = make_float2(acc[g][k].x * a, acc[g][k].y * a);
         }
 #pragma unroll
-        for (int t0 = 0; t0 < kStageTokens; t0 += S::kTPV) {
+        for (int t0 = 0; t0 < S::kTS; t0 += S::kTPV) {
           const int t = t0 + vslot;
           if (t < nvalid) {
-            const Piece vp = *reinterpret_cast<const Piece*>(vtile + piece_offset<S>(cw * kStageTokens + t, dp));
+            const Piece vp = *reinterpret_cast<const Piece*>(vtile + piece_offset<S>(tile_row(cw, t), dp));
             float2 vf[4];
             Elem<KVT>::to_float(vp, vf);
             float p[G];
