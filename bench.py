@@ -166,6 +166,8 @@ def run_reference(args, cfg, world, rank):
     if rank != 0:
         return
     import oracle
+    import dataclasses
+    cfg = dataclasses.replace(cfg, num_blocks=None)  # the sample's pool: 1.2x its blocks (placement only)
     # pick a sample of sequences so that one step takes about 1 s
     n, dt = 1, 0.0
     while True:
@@ -369,7 +371,9 @@ def main():
 
 def cpu_baseline(cfg, seconds):
     """The oracle (as it stands) on a bounded sample of the same workload, on the host cores."""
+    import dataclasses
     import oracle
+    cfg = dataclasses.replace(cfg, num_blocks=None)  # the sample's pool: 1.2x its blocks (placement only)
     n = 1
     while True:
         w = W.make_workload(cfg, seed=cfg.seed, num_seqs=n, prefilled=True)
