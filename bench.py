@@ -138,6 +138,8 @@ def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl != "reference":
+        torch.cuda.set_device(local)  # before NCCL comes up, so each rank's collectives use its own GPU
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl" if args.impl != "reference" else "gloo",
