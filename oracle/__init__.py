@@ -58,6 +58,8 @@ def _bind(path):
     L.or_reshape_and_cache.argtypes = [p, p, i, p, p, i, p, p, p, i64, i, i, i, i64]
     L.or_copy_blocks.restype = i
     L.or_copy_blocks.argtypes = [p, p, i, p, i64, i, i, i, i64]
+    L.or_swap_blocks.restype = i
+    L.or_swap_blocks.argtypes = [p, p, p, p, i, p, i64, i, i, i, i64, i64]
     return L
 
 
@@ -207,6 +209,21 @@ def copy_blocks(key_cache, value_cache, kv_dtype, block_mapping):
                               bm.shape[0], Hkv, d, bs, NB)
     if st != 0:
         raise OracleError(f"or_copy_blocks failed with status {st}")
+
+
+def swap_blocks(dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, kv_dtype, block_mapping):
+    """Copy whole blocks src_pool[src] -> dst_pool[dst] for each (src, dst) pair, in place on dst."""
+    for a in (dst_key_cache, dst_value_cache, src_key_cache, src_value_cache):
+        assert a.flags.c_contiguous
+    bm = _c(block_mapping, np.int64).reshape(-1, 2)
+    NBs, bs, Hkv, d = src_key_cache.shape
+    NBd = dst_key_cache.shape[0]
+    assert dst_key_cache.shape[1:] == src_key_cache.shape[1:]
+    st = lib().or_swap_blocks(_ptr(dst_key_cache), _ptr(dst_value_cache), _ptr(src_key_cache),
+                              _ptr(src_value_cache), dtype_code(kv_dtype), _ptr(bm), bm.shape[0], Hkv, d, bs,
+                              NBs, NBd)
+    if st != 0:
+        raise OracleError(f"or_swap_blocks failed with status {st}")
 
 
 def quantize_e4m3(values_bits, in_dtype, scale_per_head):

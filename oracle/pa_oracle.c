@@ -355,3 +355,26 @@ int or_copy_blocks(void* key_cache, void* value_cache, int kv_dtype, const int64
   }
   return OR_OK;
 }
+
+/* ------------------------------------------------------------------------------------------------
+ * Swapping blocks between two pools ([C] "PagedAttention：把显存做成虚拟内存": pages of inactive
+ * sequences are moved to CPU memory and brought back when needed): for each pair (src, dst) the whole
+ * key block and the whole value block of the source pool are copied into block dst of the other pool.
+ * --------------------------------------------------------------------------------------------- */
+int or_swap_blocks(void* dst_key_cache, void* dst_value_cache, const void* src_key_cache,
+                   const void* src_value_cache, int kv_dtype, const int64_t* block_mapping,
+                   int64_t num_pairs, int num_kv_heads, int head_size, int block_size,
+                   int64_t src_num_blocks, int64_t dst_num_blocks) {
+  if (!dst_key_cache || !dst_value_cache || !src_key_cache || !src_value_cache || (!block_mapping && num_pairs > 0))
+    return OR_BAD_ARG;
+  size_t elem = (kv_dtype == OR_E4M3) ? 1 : 2;
+  size_t block_bytes = (size_t)block_size * num_kv_heads * head_size * elem;
+  for (int64_t p = 0; p < num_pairs; ++p) {
+    int64_t src = block_mapping[2 * p], dst = block_mapping[2 * p + 1];
+    if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) return OR_BAD_BLOCK;
+    memcpy((char*)dst_key_cache + dst * block_bytes, (const char*)src_key_cache + src * block_bytes, block_bytes);
+    memcpy((char*)dst_value_cache + dst * block_bytes, (const char*)src_value_cache + src * block_bytes, block_bytes);
+  }
+  return OR_OK;
+}
+

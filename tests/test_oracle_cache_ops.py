@@ -1,4 +1,4 @@
-"""Pins for the oracle's reshape_and_cache and copy_blocks (CPU only).
+"""Pins for the oracle's reshape_and_cache, copy_blocks and swap_blocks (CPU only).
 
 16-bit caches: written slots hold exactly the input bits, every other byte is untouched (checked
 against a byte copy of the pool and this test's own slot arithmetic). FP8 caches: the stored code is
@@ -97,3 +97,24 @@ def test_copy_blocks_rejects_out_of_range_ids():
     vc = np.zeros_like(kc)
     with pytest.raises(oracle.OracleError):
         oracle.copy_blocks(kc, vc, "bf16", np.array([[0, 4]], np.int64))
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8_e4m3"])
+def test_swap_blocks_moves_whole_blocks_between_pools(kv_dtype):
+    rng = np.random.default_rng(5)
+    dt = np.uint8 if kv_dtype == "fp8_e4m3" else np.uint16
+    dev_k = rng.integers(0, np.iinfo(dt).max, (12, 8, 2, 16)).astype(dt)
+    dev_v = rng.integers(0, np.iinfo(dt).max, (12, 8, 2, 16)).astype(dt)
+    host_k = np.zeros((5, 8, 2, 16), dt)
+    host_v = np.zeros_like(host_k)
+    out_pairs = np.array([[3, 0], [7, 4], [11, 2]], np.int64)          # swap-out: device -> host
+    oracle.swap_blocks(host_k, host_v, dev_k, dev_v, kv_dtype, out_pairs)
+    for s, d in out_pairs:
+        assert np.array_equal(host_k[d], dev_k[s]) and np.array_equal(host_v[d], dev_v[s])
+    assert np.all(host_k[[1, 3]] == 0) and np.all(host_v[[1, 3]] == 0)  # untouched host blocks
+    back_k, back_v = np.zeros_like(dev_k), np.zeros_like(dev_v)
+    oracle.swap_blocks(back_k, back_v, host_k, host_v, kv_dtype, out_pairs[:, ::-1].copy())  # swap-in
+    for s, d in out_pairs:
+        assert np.array_equal(back_k[s], dev_k[s]) and np.array_equal(back_v[s], dev_v[s])
+    with pytest.raises(oracle.OracleError):
+        oracle.swap_blocks(host_k, host_v, dev_k, dev_v, kv_dtype, np.array([[12, 0]], np.int64))
