@@ -214,6 +214,8 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--op", default="decode", choices=["decode", "swap"],
+                    help="decode: the decode step (default); swap: swap_blocks host<->device throughput")
     ap.add_argument("--workload", default="7b", choices=list(W.CONFIGS))
     ap.add_argument("--partition-size", type=int, default=None,
                     help="tokens per split-K partition (default: the workload's, else the library's choice)")
@@ -233,6 +235,12 @@ def main():
         args.partition_size = cfg.partition_size
     world, rank, local = dist_setup(args)
 
+    if args.op == "swap":
+        if rank == 0:
+            run_swap(args, cfg)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     if args.impl == "reference":
         run_reference(args, cfg, world, rank)
         if world > 1:
@@ -369,6 +377,55 @@ def main():
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+
+
+def run_swap(args, cfg, num_blocks=1024):
+    """swap_blocks throughput: num_blocks random blocks of the workload's pool out to a pinned host pool
+    and back in, each direction one launch, CUDA-event timed; beside it a plain copy of the same bytes
+    between pinned host memory and the device (the link's ceiling for contiguous transfers)."""
+    from pagedattention_paged_kv_attention_b200 import pagedattn as P
+    dev = torch.device("cuda", torch.cuda.current_device())
+    kv = torch.bfloat16 if cfg.kv_dtype == "bf16" else (torch.float16 if cfg.kv_dtype == "f16" else torch.uint8)
+    shape = (cfg.num_blocks or 4096, cfg.block_size, cfg.num_kv_heads, cfg.head_size)
+    dk = torch.randn(shape, device=dev).to(kv) if kv != torch.uint8 else torch.randint(0, 120, shape, device=dev, dtype=kv)
+    dv = dk.clone()
+    hk = torch.empty((num_blocks,) + shape[1:], dtype=kv).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    g = torch.Generator().manual_seed(cfg.seed)
+    src = torch.randperm(shape[0], generator=g)[:num_blocks]
+    out_map = torch.stack([src, torch.arange(num_blocks)], 1).to(dev)
+    in_map = torch.stack([torch.arange(num_blocks), torch.randperm(shape[0], generator=g)[:num_blocks]], 1).to(dev)
+    nbytes = 2 * hk.numel() * hk.element_size()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    t_out = timed(lambda: P.swap_blocks(hk, hv, dk, dv, out_map))
+    t_in = timed(lambda: P.swap_blocks(dk, dv, hk, hv, in_map))
+    flat_d = torch.empty(hk.numel() * 2, dtype=kv, device=dev)
+    flat_h = torch.empty(hk.numel() * 2, dtype=kv).pin_memory()
+    t_d2h = timed(lambda: flat_h.copy_(flat_d, non_blocking=True))
+    t_h2d = timed(lambda: flat_d.copy_(flat_h, non_blocking=True))
+    gbs = lambda ms: round(nbytes / (ms * 1e-3) / 1e9, 2)
+    line = {"metric": "swap_blocks host<->device GB/s", "value": gbs((t_out + t_in) / 2), "unit": "GB/s",
+            "impl": "ours", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "dtype": cfg.kv_dtype, "data": "synthetic",
+            "config": {"workload": f"{num_blocks} random blocks of the {cfg.name} pool shape {list(shape[1:])}",
+                       "bytes_per_direction": nbytes},
+            "swap_out_gbs": gbs(t_out), "swap_in_gbs": gbs(t_in),
+            "roofline": {"bound": "host link", "copy_d2h_gbs": gbs(t_d2h), "copy_h2d_gbs": gbs(t_h2d),
+                         "frac_out": round(t_d2h / t_out, 3), "frac_in": round(t_h2d / t_in, 3)},
+            "gpu_launches": 2 * args.steps}
+    print(json.dumps(line), flush=True)
 
 
 def cpu_baseline(cfg, seconds):

@@ -197,6 +197,24 @@ PA_API pa_status pa_copy_blocks(void* key_cache, void* value_cache, pa_dtype kv_
                          int head_size, int block_size, int num_blocks, pa_stream_t stream);
 
 /*
+ * Swap whole blocks between two pools ([C] "PagedAttention：把显存做成虚拟内存": pages of inactive
+ * sequences are moved to CPU memory and brought back when needed). For each pair p, the key block and
+ * the value block block_mapping[p][0] of the source pool are copied to block block_mapping[p][1] of the
+ * destination pool; both pools have the cache layout above with the same block shape.
+ *  dst_*, src_*   pool base pointers; each may be device memory or PINNED host memory (cudaHostAlloc /
+ *                 cudaHostRegister / torch pin_memory), reached by the kernel through its unified
+ *                 address. Pageable host memory is refused with PA_ERR_INVALID_ARGUMENT.
+ *  block_mapping  [num_pairs][2] int64 (src, dst), device or pinned host memory. Pairs with an id outside
+ *                 its pool are skipped. Destinations must be distinct (otherwise the copies race).
+ *  src_num_blocks, dst_num_blocks  pool sizes in blocks.
+ * One launch moves every pair (no per-block copy calls). Asynchronous on `stream`.
+ */
+PA_API pa_status pa_swap_blocks(void* dst_key_cache, void* dst_value_cache, const void* src_key_cache,
+                                const void* src_value_cache, pa_dtype kv_dtype, const int64_t* block_mapping,
+                                int num_pairs, int num_kv_heads, int head_size, int block_size,
+                                int src_num_blocks, int dst_num_blocks, pa_stream_t stream);
+
+/*
  * Host-side check of a copy_blocks mapping (host pointer, [num_pairs][2] int64): every id in
  * [0, num_blocks), destinations distinct, no destination also a source. PA_OK or
  * PA_ERR_INVALID_ARGUMENT. Makes no CUDA call.
@@ -211,6 +229,16 @@ PA_API pa_status pa_get_device_error(const void* workspace, unsigned int* err_ou
 
 /* Zero the device error word of a workspace (enqueued on `stream`, asynchronous). */
 PA_API pa_status pa_clear_device_error(void* workspace, pa_stream_t stream);
+
+/*
+ * Self-test of failure detection (no counterpart on the pages): every wait inside these kernels is
+ * bounded, and on expiry sets PA_DEVERR_TIMEOUT and lets the kernel finish instead of hanging. This call
+ * launches a one-warp kernel that waits, with the bounded-wait routine the kernels use, on an mbarrier
+ * that nothing ever arrives on; after limit_ns nanoseconds (1 ns .. 10 s) it ORs PA_DEVERR_TIMEOUT into
+ * *device_error_word (a DEVICE pointer) and returns. Asynchronous on `stream`; the context stays usable.
+ */
+PA_API pa_status pa_selftest_wait_timeout(unsigned int* device_error_word, unsigned long long limit_ns,
+                                          pa_stream_t stream);
 
 /* Static description of a status code. Never NULL. */
 PA_API const char* pa_status_string(pa_status status);

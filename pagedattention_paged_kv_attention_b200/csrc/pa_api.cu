@@ -285,6 +285,50 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, pa_dtype kv_dtype, 
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+namespace {
+// Device-reachable address of a pointer (device memory, managed memory, or pinned/registered host
+// memory); nullptr for pageable host memory or an unknown pointer.
+void* device_reachable(const void* p) {
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error of an unknown pointer
+    return nullptr;
+  }
+  if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) return const_cast<void*>(p);
+  if (attr.type == cudaMemoryTypeHost) return attr.devicePointer;
+  return nullptr;
+}
+}  // namespace
+
+pa_status pa_swap_blocks(void* dst_key_cache, void* dst_value_cache, const void* src_key_cache,
+                         const void* src_value_cache, pa_dtype kv_dtype, const int64_t* block_mapping, int num_pairs,
+                         int num_kv_heads, int head_size, int block_size, int src_num_blocks, int dst_num_blocks,
+                         pa_stream_t stream) {
+  if (num_pairs < 0 || num_kv_heads <= 0 || head_size <= 0 || block_size <= 0 || src_num_blocks <= 0 ||
+      dst_num_blocks <= 0 || !is_dtype(kv_dtype))
+    return PA_ERR_INVALID_ARGUMENT;
+  if (!dst_key_cache || !dst_value_cache || !src_key_cache || !src_value_cache || (num_pairs > 0 && !block_mapping))
+    return PA_ERR_INVALID_ARGUMENT;
+  if (!aligned(dst_key_cache, 16) || !aligned(dst_value_cache, 16) || !aligned(src_key_cache, 16) ||
+      !aligned(src_value_cache, 16) || (block_mapping && !aligned(block_mapping, 8)))
+    return PA_ERR_INVALID_ARGUMENT;
+  const int64_t block_bytes = static_cast<int64_t>(block_size) * num_kv_heads * head_size * elem_bytes(kv_dtype);
+  if (block_bytes % 16 != 0) return PA_ERR_UNSUPPORTED;
+  if (num_pairs == 0) return PA_OK;
+  // Every pool and the mapping must be reachable from the GPU; pageable host memory is refused here
+  // (a kernel touching it would fault).
+  void* dk = device_reachable(dst_key_cache);
+  void* dv = device_reachable(dst_value_cache);
+  void* sk = device_reachable(src_key_cache);
+  void* sv = device_reachable(src_value_cache);
+  void* bm = device_reachable(block_mapping);
+  if (!dk || !dv || !sk || !sv || !bm) return PA_ERR_INVALID_ARGUMENT;
+  pa::swap_blocks_kernel<<<dim3(static_cast<unsigned>(num_pairs), 2), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint8_t*>(dk), static_cast<uint8_t*>(dv), static_cast<const uint8_t*>(sk),
+      static_cast<const uint8_t*>(sv), static_cast<const int64_t*>(bm), block_bytes, src_num_blocks, dst_num_blocks);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 pa_status pa_copy_blocks_check(const int64_t* host_block_mapping, int num_pairs, int num_blocks) {
   if (num_pairs < 0 || num_blocks <= 0 || (num_pairs > 0 && !host_block_mapping)) return PA_ERR_INVALID_ARGUMENT;
   std::unordered_set<int64_t> srcs, dsts;
@@ -297,6 +341,13 @@ pa_status pa_copy_blocks_check(const int64_t* host_block_mapping, int num_pairs,
   for (int64_t d : dsts)
     if (srcs.count(d)) return PA_ERR_INVALID_ARGUMENT;
   return PA_OK;
+}
+
+pa_status pa_selftest_wait_timeout(unsigned int* device_error_word, unsigned long long limit_ns, pa_stream_t stream) {
+  if (!device_error_word || !aligned(device_error_word, 4) || limit_ns == 0 || limit_ns > 10000000000ull)
+    return PA_ERR_INVALID_ARGUMENT;
+  pa::selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(device_error_word, limit_ns);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_get_device_error(const void* workspace, unsigned int* err_out, pa_stream_t stream) {

@@ -78,4 +78,34 @@ copy_blocks_kernel(uint8_t* __restrict__ key_cache, uint8_t* __restrict__ value_
   for (int64_t i = threadIdx.x; i < n; i += blockDim.x) d[i] = s[i];
 }
 
+// Swapping blocks between two pools that may live in different memories (device, or pinned host
+// memory reached through its unified address): one CTA per (pair, key|value), 16-byte vectors. Page
+// "PagedAttention 与连续批处理：LLM Serving 的底层架构拆解", section "PagedAttention：把显存做成虚拟内存":
+// pages of inactive sequences go to CPU memory and come back when needed.
+__global__ void __launch_bounds__(256)
+swap_blocks_kernel(uint8_t* __restrict__ dst_key, uint8_t* __restrict__ dst_value, const uint8_t* __restrict__ src_key,
+                   const uint8_t* __restrict__ src_value, const int64_t* __restrict__ block_mapping,
+                   int64_t block_bytes, int src_num_blocks, int dst_num_blocks) {
+  const int pair = blockIdx.x;
+  const int64_t src = block_mapping[2 * pair];
+  const int64_t dst = block_mapping[2 * pair + 1];
+  if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) return;
+  const uint4* s = reinterpret_cast<const uint4*>((blockIdx.y == 0 ? src_key : src_value) + src * block_bytes);
+  uint4* d = reinterpret_cast<uint4*>((blockIdx.y == 0 ? dst_key : dst_value) + dst * block_bytes);
+  const int64_t n = block_bytes / 16;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) d[i] = s[i];
+}
+
+// Self-test of the bounded wait used by every pipeline wait: an mbarrier that nothing ever arrives on
+// is waited for with a short limit; the wait must give up, set PA_DEVERR_TIMEOUT and return.
+__global__ void selftest_wait_kernel(unsigned int* error_word, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0u, error_word, limit_ns);
+}
+
 }  // namespace pa

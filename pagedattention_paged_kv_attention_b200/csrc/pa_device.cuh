@@ -56,12 +56,13 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // PA_DEVERR_TIMEOUT in the error word and returns false, so no kernel can spin forever.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s; a healthy wait lasts microseconds
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* error_word) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* error_word,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t start = global_timer_ns();
   for (uint32_t spin = 0;; ++spin) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((spin & 63u) == 63u && global_timer_ns() - start > kWaitLimitNs) {
+    if ((spin & 63u) == 63u && global_timer_ns() - start > limit_ns) {
       atomicOr(error_word, PA_DEVERR_TIMEOUT);
       return false;
     }

@@ -23,7 +23,8 @@ WORKSPACE_HEADER_BYTES = 256
 EXPORTS = (
     "pa_paged_attention_partition_size", "pa_paged_attention_workspace_size", "pa_paged_attention",
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_copy_blocks_check", "pa_get_device_error",
-    "pa_clear_device_error", "pa_status_string", "pa_paged_attention_static",
+    "pa_clear_device_error", "pa_status_string", "pa_paged_attention_static", "pa_selftest_wait_timeout",
+    "pa_swap_blocks",
 )
 
 if not os.path.exists(LIBRARY_PATH):
@@ -48,12 +49,16 @@ lib.pa_reshape_and_cache.restype = _i
 lib.pa_reshape_and_cache.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 lib.pa_copy_blocks.restype = _i
 lib.pa_copy_blocks.argtypes = [_p, _p, _i, _p, _i, _i, _i, _i, _i, _p]
+lib.pa_swap_blocks.restype = _i
+lib.pa_swap_blocks.argtypes = [_p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _p]
 lib.pa_copy_blocks_check.restype = _i
 lib.pa_copy_blocks_check.argtypes = [_p, _i, _i]
 lib.pa_get_device_error.restype = _i
 lib.pa_get_device_error.argtypes = [_p, ctypes.POINTER(ctypes.c_uint), _p]
 lib.pa_clear_device_error.restype = _i
 lib.pa_clear_device_error.argtypes = [_p, _p]
+lib.pa_selftest_wait_timeout.restype = _i
+lib.pa_selftest_wait_timeout.argtypes = [_p, ctypes.c_ulonglong, _p]
 
 
 class PagedAttnError(RuntimeError):
@@ -154,6 +159,16 @@ def copy_blocks(key_cache, value_cache, block_mapping, stream=None):
     _check(st, "pa_copy_blocks")
 
 
+def swap_blocks(dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, block_mapping, stream=None):
+    """Copy whole blocks src_pool[m[i,0]] -> dst_pool[m[i,1]]; pools on the device or in pinned host memory."""
+    NBs, bs, Hkv, d = src_key_cache.shape
+    NBd = dst_key_cache.shape[0]
+    st = lib.pa_swap_blocks(_ptr(dst_key_cache), _ptr(dst_value_cache), _ptr(src_key_cache), _ptr(src_value_cache),
+                            dtype_code(src_key_cache.dtype), _ptr(block_mapping), block_mapping.shape[0], Hkv, d, bs,
+                            NBs, NBd, _stream(stream))
+    _check(st, "pa_swap_blocks")
+
+
 def copy_blocks_check(block_mapping_host: torch.Tensor, num_blocks: int) -> bool:
     m = block_mapping_host.to(torch.int64).contiguous().cpu()
     return lib.pa_copy_blocks_check(_ptr(m), m.shape[0], num_blocks) == PA_OK
@@ -163,6 +178,13 @@ def get_device_error(workspace, stream=None) -> int:
     v = ctypes.c_uint(0)
     _check(lib.pa_get_device_error(_ptr(workspace), ctypes.byref(v), _stream(stream)), "pa_get_device_error")
     return v.value
+
+
+def selftest_wait_timeout(device_error_word, limit_ns, stream=None):
+    """Run the bounded-wait self-test: a wait that nothing satisfies gives up after limit_ns and ORs
+    PA_DEVERR_TIMEOUT into device_error_word (a one-element int32 device tensor)."""
+    _check(lib.pa_selftest_wait_timeout(_ptr(device_error_word), int(limit_ns), _stream(stream)),
+           "pa_selftest_wait_timeout")
 
 
 def clear_device_error(workspace, stream=None):
