@@ -1,4 +1,4 @@
-"""One decode step (reshape_and_cache -> copy_blocks -> paged_attention) run two ways on the same
+"""One decode step (copy_blocks -> reshape_and_cache -> paged_attention) run two ways on the same
 seeded inputs: through the oracle on the CPU, and through the C-ABI library on the GPU.
 
 Test infrastructure: the GPU side gets its inputs from the generator (and, for FP8 caches, the
@@ -39,11 +39,11 @@ def oracle_step(w, kc, vc, write_new=True, copy=True):
     cfg = w.cfg
     ks = None if w.k_scale is None else w.k_scale.numpy()
     vs = None if w.v_scale is None else w.v_scale.numpy()
+    if copy and w.cow_mapping.shape[0]:
+        oracle.copy_blocks(kc, vc, cfg.kv_dtype, w.cow_mapping.numpy())
     if write_new:
         oracle.reshape_and_cache(bits16(w.new_key), bits16(w.new_value), cfg.dtype, kc, vc, cfg.kv_dtype,
                                  w.slot_mapping.numpy(), ks, vs)
-    if copy and w.cow_mapping.shape[0]:
-        oracle.copy_blocks(kc, vc, cfg.kv_dtype, w.cow_mapping.numpy())
     return oracle.paged_attention(bits16(w.query), cfg.dtype, kc, vc, cfg.kv_dtype, w.block_tables.numpy(),
                                   w.context_lens.numpy(), cfg.softmax_scale, ks, vs)
 
@@ -67,10 +67,10 @@ def gpu_step(P, w, kc_dev, vc_dev, write_new=True, copy=True, partition_size=0, 
     dev = kc_dev.device
     ks = None if w.k_scale is None else w.k_scale.to(dev)
     vs = None if w.v_scale is None else w.v_scale.to(dev)
-    if write_new:
-        P.reshape_and_cache(w.new_key.to(dev), w.new_value.to(dev), kc_dev, vc_dev, w.slot_mapping.to(dev), ks, vs)
     if copy and w.cow_mapping.shape[0]:
         P.copy_blocks(kc_dev, vc_dev, w.cow_mapping.to(dev))
+    if write_new:
+        P.reshape_and_cache(w.new_key.to(dev), w.new_value.to(dev), kc_dev, vc_dev, w.slot_mapping.to(dev), ks, vs)
     bt = (w.block_tables if block_tables is None else block_tables).to(dev)
     cl = (w.context_lens if context_lens is None else context_lens).to(dev)
     mcl = int(cl.max().item()) if max_context_len is None and cl.numel() else (max_context_len or 0)

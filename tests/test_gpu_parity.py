@@ -1,8 +1,8 @@
 """GPU parity: the C-ABI library against the oracle on the same seeded inputs.
 
 * Every config of the workload table at its full size, in the launch configuration the benchmark
-  uses (automatic partition size): one decode step (reshape_and_cache of the new tokens, copy_blocks
-  of the copy-on-write pairs, paged attention). Every attention output is compared element by element
+  uses (automatic partition size): one decode step (copy_blocks of the copy-on-write pairs,
+  reshape_and_cache of the new tokens, paged attention). Every attention output is compared element by element
   with the oracle (max-abs within the stated tolerance); the whole key and value pools after the step
   are compared byte for byte with the oracle's (reshape_and_cache and copy_blocks are bit-exact, and
   nothing else in the pool may change).
