@@ -214,7 +214,7 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--op", default="decode", choices=["decode", "swap"],
+    ap.add_argument("--op", default="decode", choices=["decode", "swap", "layers"],
                     help="decode: the decode step (default); swap: swap_blocks host<->device throughput")
     ap.add_argument("--workload", default="7b", choices=list(W.CONFIGS))
     ap.add_argument("--partition-size", type=int, default=None,
@@ -235,9 +235,9 @@ def main():
         args.partition_size = cfg.partition_size
     world, rank, local = dist_setup(args)
 
-    if args.op == "swap":
+    if args.op in ("swap", "layers"):
         if rank == 0:
-            run_swap(args, cfg)
+            (run_swap if args.op == "swap" else run_layers)(args, cfg)
         if world > 1:
             torch.distributed.destroy_process_group()
         return
@@ -276,9 +276,9 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     def step(q, nk, nv, slots, tables, clens, o, ev=None):
-        P.reshape_and_cache(nk, nv, key_cache, value_cache, slots, ks, vs)
-        if w.cow_mapping.shape[0]:
+        if w.cow_mapping.shape[0]:      # copy-on-write first, so a copied block then takes its new token
             P.copy_blocks(key_cache, value_cache, w.cow_mapping)
+        P.reshape_and_cache(nk, nv, key_cache, value_cache, slots, ks, vs)
         if ev is not None:
             ev[0].record(stream)
         P.paged_attention(o, q, key_cache, value_cache, tables, clens, cfg.softmax_scale, mcl, ws, ks, vs,
@@ -425,6 +425,90 @@ def run_swap(args, cfg, num_blocks=1024):
             "roofline": {"bound": "host link", "copy_d2h_gbs": gbs(t_d2h), "copy_h2d_gbs": gbs(t_h2d),
                          "frac_out": round(t_d2h / t_out, 3), "frac_in": round(t_h2d / t_in, 3)},
             "gpu_launches": 2 * args.steps}
+    print(json.dumps(line), flush=True)
+
+
+def run_layers(args, cfg, num_layers=32, pool_blocks=2048, cow_pairs=64):
+    """The cache ops of one decode step over every layer of the model: reshape_and_cache of the batch's
+    new tokens (distinct random slots) and copy_blocks of cow_pairs copy-on-write pairs, each as ONE
+    launch covering all num_layers layers, CUDA-event timed; beside it the same work as one launch
+    per layer. Bytes: each token's K and V row read and written, each pair's K and V block read and
+    written, per layer. The step's data (over 0.5 GB) exceeds L2, so no flush is needed."""
+    from pagedattention_paged_kv_attention_b200 import pagedattn as P
+    dev = torch.device("cuda", torch.cuda.current_device())
+    kv = torch.bfloat16 if cfg.kv_dtype == "bf16" else (torch.float16 if cfg.kv_dtype == "f16" else torch.uint8)
+    it = torch.bfloat16 if cfg.dtype == "bf16" else torch.float16
+    T, Hkv, d, bs = cfg.num_seqs, cfg.num_kv_heads, cfg.head_size, cfg.block_size
+    shape = (pool_blocks, bs, Hkv, d)
+    g = torch.Generator(device=dev).manual_seed(cfg.seed)
+    kc = [torch.empty(shape, dtype=kv, device=dev) for _ in range(num_layers)]
+    vc = [torch.empty(shape, dtype=kv, device=dev) for _ in range(num_layers)]
+    for t in kc + vc:
+        t.view(torch.uint8).random_(0, 120, generator=g)
+    keys = [torch.randn((T, Hkv, d), generator=g, device=dev).to(it) for _ in range(num_layers)]
+    values = [torch.randn((T, Hkv, d), generator=g, device=dev).to(it) for _ in range(num_layers)]
+    fp8 = kv == torch.uint8
+    ks = [torch.full((Hkv,), 0.01, device=dev) for _ in range(num_layers)] if fp8 else None
+    vs = [torch.full((Hkv,), 0.01, device=dev) for _ in range(num_layers)] if fp8 else None
+    perm = torch.randperm(pool_blocks * bs, generator=g, device=dev)
+    slots = perm[:T].to(torch.int64)
+    bperm = torch.randperm(pool_blocks, generator=g, device=dev)
+    pairs = torch.stack([bperm[:cow_pairs], bperm[cow_pairs:2 * cow_pairs]], 1).to(torch.int64).contiguous()
+    ptr = P.pointer_array
+    arrays = [ptr(keys), ptr(values), ptr(kc), ptr(vc)]
+    sarr = (ptr(ks), ptr(vs)) if fp8 else (None, None)
+    ke, ve = kc[0].element_size(), it.itemsize
+    reshape_bytes = num_layers * 2 * T * Hkv * d * (ve + ke)
+    copy_bytes = num_layers * 2 * 2 * cow_pairs * bs * Hkv * d * ke
+    lib, stream = P.lib, P._stream(None)
+    code_in, code_kv = P.dtype_code(it), P.dtype_code(kv)
+
+    def fused():
+        # pointer arrays built once, as a caller holding its layers' caches would keep them
+        P._check(lib.pa_reshape_and_cache_layers(
+            arrays[0].data_ptr(), arrays[1].data_ptr(), code_in, arrays[2].data_ptr(), arrays[3].data_ptr(),
+            code_kv, sarr[0].data_ptr() if fp8 else None, sarr[1].data_ptr() if fp8 else None, slots.data_ptr(),
+            T, num_layers, Hkv, d, bs, pool_blocks, stream), "pa_reshape_and_cache_layers")
+        P._check(lib.pa_copy_blocks_layers(arrays[2].data_ptr(), arrays[3].data_ptr(), num_layers, code_kv,
+                                           pairs.data_ptr(), cow_pairs, Hkv, d, bs, pool_blocks, stream),
+                 "pa_copy_blocks_layers")
+
+    def per_layer():
+        for l in range(num_layers):
+            P.reshape_and_cache(keys[l], values[l], kc[l], vc[l], slots, ks[l] if fp8 else None,
+                                vs[l] if fp8 else None)
+            P.copy_blocks(kc[l], vc[l], pairs)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    peaks = measured_peaks()
+    peak = peaks.get("hbm_gbs") if peaks else None
+    with ClockSampler(gpu_selector(dev)) as clocks:
+        t_fused = timed(fused)
+        t_loop = timed(per_layer)
+    total = reshape_bytes + copy_bytes
+    gbs = lambda nb, ms: round(nb / (ms * 1e-3) / 1e9, 2)
+    line = {"metric": "multi-layer cache ops GB/s", "value": gbs(total, t_fused), "unit": "GB/s", "impl": "ours",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_fused, 4),
+            "higher_is_better": True, "dtype": cfg.kv_dtype, "data": "synthetic",
+            "config": {"workload": f"{cfg.name} cache shape, {num_layers} layers, {T} new tokens, "
+                                   f"{cow_pairs} copy-on-write pairs, pool {pool_blocks} blocks per layer",
+                       "l2": "step data larger than L2", "bytes_per_step": total},
+            "per_layer_launches": {"ms_per_step": round(t_loop, 4), "value": gbs(total, t_loop)},
+            "roofline": {"bound": "hbm", "achieved": gbs(total, t_fused), "peak": peak, "unit": "GB/s",
+                         "frac": round(gbs(total, t_fused) / peak, 3) if peak else None, "traffic": None,
+                         "peak_source": "measured" if peak else None},
+            "clocks": clocks.summary(), "gpu_launches": 2 * args.steps}
     print(json.dumps(line), flush=True)
 
 

@@ -62,7 +62,8 @@ typedef enum pa_status {
   PA_ERR_INVALID_ARGUMENT = 1,          /* null/misaligned pointer, negative size, bad mapping, ... */
   PA_ERR_UNSUPPORTED = 2,               /* valid but outside the supported set above */
   PA_ERR_WORKSPACE_TOO_SMALL = 3,       /* workspace_bytes < pa_paged_attention_workspace_size(...) */
-  PA_ERR_CUDA = 4                       /* a CUDA runtime/driver call or a launch failed */
+  PA_ERR_CUDA = 4,                      /* a CUDA runtime/driver call or a launch failed */
+  PA_ERR_OUT_OF_BLOCKS = 5              /* block manager: the pool has too few free blocks (no change) */
 } pa_status;
 
 typedef enum pa_dtype {
@@ -175,7 +176,8 @@ PA_API pa_status pa_paged_attention_static(void* out, const void* query, pa_dtyp
  *  k_scale,
  *  v_scale        [num_kv_heads] fp32, required for PA_FP8_E4M3.
  *  slot_mapping   [num_tokens] int64.
- * Two tokens mapped to the same slot race (the result is one of them).
+ * Two tokens mapped to the same slot race (the result is one of them). num_tokens == 0 is a no-op
+ * (pointers may then be null).
  */
 PA_API pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dtype in_dtype,
                                void* key_cache, void* value_cache, pa_dtype kv_dtype,
@@ -195,6 +197,30 @@ PA_API pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dty
 PA_API pa_status pa_copy_blocks(void* key_cache, void* value_cache, pa_dtype kv_dtype,
                          const int64_t* block_mapping, int num_pairs, int num_kv_heads,
                          int head_size, int block_size, int num_blocks, pa_stream_t stream);
+
+/*
+ * reshape_and_cache for every layer of a model in one launch. The same slot_mapping applies to all
+ * layers; layer l reads keys[l]/values[l] ([num_tokens][num_kv_heads][head_size], in_dtype) and writes
+ * key_caches[l]/value_caches[l] (scales k_scales[l]/v_scales[l] for FP8). The pointer arrays are
+ * DEVICE arrays of num_layers device pointers, each 16-byte aligned; the library cannot inspect them
+ * (an invalid entry is the caller's error). Same semantics per layer as pa_reshape_and_cache.
+ */
+PA_API pa_status pa_reshape_and_cache_layers(const void* const* keys, const void* const* values, pa_dtype in_dtype,
+                                             void* const* key_caches, void* const* value_caches, pa_dtype kv_dtype,
+                                             const float* const* k_scales, const float* const* v_scales,
+                                             const int64_t* slot_mapping, int num_tokens, int num_layers,
+                                             int num_kv_heads, int head_size, int block_size, int num_blocks,
+                                             pa_stream_t stream);
+
+/*
+ * copy_blocks for every layer in one launch: the same (src, dst) mapping applied to key_caches[l] and
+ * value_caches[l] for l < num_layers (DEVICE arrays of device pointers, as above). Same semantics per
+ * layer as pa_copy_blocks.
+ */
+PA_API pa_status pa_copy_blocks_layers(void* const* key_caches, void* const* value_caches, int num_layers,
+                                       pa_dtype kv_dtype, const int64_t* block_mapping, int num_pairs,
+                                       int num_kv_heads, int head_size, int block_size, int num_blocks,
+                                       pa_stream_t stream);
 
 /*
  * Swap whole blocks between two pools ([C] "PagedAttention：把显存做成虚拟内存": pages of inactive

@@ -124,6 +124,7 @@ const char* pa_status_string(pa_status status) {
     case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: valid but outside the supported head_size/block_size/dtype set";
     case PA_ERR_WORKSPACE_TOO_SMALL: return "PA_ERR_WORKSPACE_TOO_SMALL: workspace smaller than pa_paged_attention_workspace_size()";
     case PA_ERR_CUDA: return "PA_ERR_CUDA: a CUDA call or kernel launch failed";
+    case PA_ERR_OUT_OF_BLOCKS: return "PA_ERR_OUT_OF_BLOCKS: too few free blocks in the pool (state unchanged)";
   }
   return "unknown pa_status";
 }
@@ -228,6 +229,7 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dtype in_d
   if (num_tokens < 0 || num_kv_heads <= 0 || head_size <= 0 || block_size <= 0 || num_blocks <= 0)
     return PA_ERR_INVALID_ARGUMENT;
   if (!is_dtype(in_dtype) || !is_dtype(kv_dtype) || !is_16bit(in_dtype)) return PA_ERR_INVALID_ARGUMENT;
+  if (num_tokens == 0) return PA_OK;  // empty batch: nothing is read, pointers may be null
   if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_INVALID_ARGUMENT;
   if (!aligned(key, 16) || !aligned(value, 16) || !aligned(key_cache, 16) || !aligned(value_cache, 16) ||
       !aligned(slot_mapping, 8))
@@ -282,6 +284,66 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, pa_dtype kv_dtype, 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   pa::copy_blocks_kernel<<<dim3(static_cast<unsigned>(num_pairs), 2), 256, 0, st>>>(
       static_cast<uint8_t*>(key_cache), static_cast<uint8_t*>(value_cache), block_mapping, block_bytes, num_blocks);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_reshape_and_cache_layers(const void* const* keys, const void* const* values, pa_dtype in_dtype,
+                                      void* const* key_caches, void* const* value_caches, pa_dtype kv_dtype,
+                                      const float* const* k_scales, const float* const* v_scales,
+                                      const int64_t* slot_mapping, int num_tokens, int num_layers, int num_kv_heads,
+                                      int head_size, int block_size, int num_blocks, pa_stream_t stream) {
+  if (num_tokens < 0 || num_layers < 0 || num_kv_heads <= 0 || head_size <= 0 || block_size <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID_ARGUMENT;
+  if (!is_dtype(in_dtype) || !is_dtype(kv_dtype) || !is_16bit(in_dtype)) return PA_ERR_INVALID_ARGUMENT;
+  if (num_tokens == 0 || num_layers == 0) return PA_OK;  // nothing is read, pointers may be null
+  if (!keys || !values || !key_caches || !value_caches || !slot_mapping) return PA_ERR_INVALID_ARGUMENT;
+  if (!aligned(keys, 8) || !aligned(values, 8) || !aligned(key_caches, 8) || !aligned(value_caches, 8) ||
+      !aligned(slot_mapping, 8))
+    return PA_ERR_INVALID_ARGUMENT;
+  const bool fp8 = kv_dtype == PA_FP8_E4M3;
+  if (fp8 && (!k_scales || !v_scales || !aligned(k_scales, 8) || !aligned(v_scales, 8))) return PA_ERR_INVALID_ARGUMENT;
+  if (!fp8 && kv_dtype != in_dtype) return PA_ERR_UNSUPPORTED;
+  if (head_size % 8 != 0 || num_layers > 65535) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0 || num_layers == 0) return PA_OK;
+  const int row = num_kv_heads * head_size;
+  const int threads = static_cast<int>(std::min<size_t>(256, round_up(static_cast<size_t>(ceil_div(row, 8)), 32)));
+  const dim3 grid(static_cast<unsigned>(num_tokens), static_cast<unsigned>(num_layers));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float* const* ks = fp8 ? k_scales : nullptr;
+  const float* const* vs = fp8 ? v_scales : nullptr;
+  if (in_dtype == PA_BF16) {
+    if (fp8)
+      pa::reshape_and_cache_layers_kernel<__nv_bfloat16, __nv_fp8_e4m3><<<grid, threads, 0, st>>>(
+          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+    else
+      pa::reshape_and_cache_layers_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, threads, 0, st>>>(
+          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+  } else {
+    if (fp8)
+      pa::reshape_and_cache_layers_kernel<__half, __nv_fp8_e4m3><<<grid, threads, 0, st>>>(
+          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+    else
+      pa::reshape_and_cache_layers_kernel<__half, __half><<<grid, threads, 0, st>>>(
+          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_copy_blocks_layers(void* const* key_caches, void* const* value_caches, int num_layers, pa_dtype kv_dtype,
+                                const int64_t* block_mapping, int num_pairs, int num_kv_heads, int head_size,
+                                int block_size, int num_blocks, pa_stream_t stream) {
+  if (num_pairs < 0 || num_layers < 0 || num_kv_heads <= 0 || head_size <= 0 || block_size <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID_ARGUMENT;
+  if (!is_dtype(kv_dtype)) return PA_ERR_INVALID_ARGUMENT;
+  if (!key_caches || !value_caches || (num_pairs > 0 && !block_mapping)) return PA_ERR_INVALID_ARGUMENT;
+  if (!aligned(key_caches, 8) || !aligned(value_caches, 8) || (block_mapping && !aligned(block_mapping, 8)))
+    return PA_ERR_INVALID_ARGUMENT;
+  const int64_t block_bytes = static_cast<int64_t>(block_size) * num_kv_heads * head_size * elem_bytes(kv_dtype);
+  if (block_bytes % 16 != 0 || num_layers > 65535) return PA_ERR_UNSUPPORTED;
+  if (num_pairs == 0 || num_layers == 0) return PA_OK;
+  pa::copy_blocks_layers_kernel<<<dim3(static_cast<unsigned>(num_pairs), 2, static_cast<unsigned>(num_layers)), 256, 0,
+                                  reinterpret_cast<cudaStream_t>(stream)>>>(key_caches, value_caches, block_mapping,
+                                                                            block_bytes, num_blocks);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -14,11 +14,12 @@ namespace pa {
 
 // One CTA per token; thread i handles 8 consecutive elements of the token's [Hkv][D] row.
 template <typename IT, typename KVT>
-__global__ void __launch_bounds__(256)
-reshape_and_cache_kernel(const IT* __restrict__ key, const IT* __restrict__ value, KVT* __restrict__ key_cache,
-                         KVT* __restrict__ value_cache, const float* __restrict__ k_scale,
-                         const float* __restrict__ v_scale, const int64_t* __restrict__ slot_mapping,
-                         int num_kv_heads, int head_size, int block_size, int num_blocks) {
+__device__ __forceinline__ void reshape_and_cache_token(const IT* __restrict__ key, const IT* __restrict__ value,
+                                                        KVT* __restrict__ key_cache, KVT* __restrict__ value_cache,
+                                                        const float* __restrict__ k_scale,
+                                                        const float* __restrict__ v_scale,
+                                                        const int64_t* __restrict__ slot_mapping, int num_kv_heads,
+                                                        int head_size, int block_size, int num_blocks) {
   const int64_t token = blockIdx.x;
   const int64_t slot = slot_mapping[token];
   if (slot < 0 || slot >= static_cast<int64_t>(num_blocks) * block_size) return;
@@ -63,6 +64,31 @@ reshape_and_cache_kernel(const IT* __restrict__ key, const IT* __restrict__ valu
   }
 }
 
+template <typename IT, typename KVT>
+__global__ void __launch_bounds__(256)
+reshape_and_cache_kernel(const IT* __restrict__ key, const IT* __restrict__ value, KVT* __restrict__ key_cache,
+                         KVT* __restrict__ value_cache, const float* __restrict__ k_scale,
+                         const float* __restrict__ v_scale, const int64_t* __restrict__ slot_mapping,
+                         int num_kv_heads, int head_size, int block_size, int num_blocks) {
+  reshape_and_cache_token<IT, KVT>(key, value, key_cache, value_cache, k_scale, v_scale, slot_mapping, num_kv_heads,
+                                   head_size, block_size, num_blocks);
+}
+
+// All layers in one launch: grid (tokens, layers); per-layer pointers come from device arrays.
+template <typename IT, typename KVT>
+__global__ void __launch_bounds__(256)
+reshape_and_cache_layers_kernel(const void* const* __restrict__ keys, const void* const* __restrict__ values,
+                                void* const* __restrict__ key_caches, void* const* __restrict__ value_caches,
+                                const float* const* __restrict__ k_scales, const float* const* __restrict__ v_scales,
+                                const int64_t* __restrict__ slot_mapping, int num_kv_heads, int head_size,
+                                int block_size, int num_blocks) {
+  const int layer = blockIdx.y;
+  reshape_and_cache_token<IT, KVT>(static_cast<const IT*>(keys[layer]), static_cast<const IT*>(values[layer]),
+                                   static_cast<KVT*>(key_caches[layer]), static_cast<KVT*>(value_caches[layer]),
+                                   k_scales ? k_scales[layer] : nullptr, v_scales ? v_scales[layer] : nullptr,
+                                   slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+}
+
 // One CTA per (pair, key|value): copy one contiguous block of `block_bytes` (a multiple of 16).
 __global__ void __launch_bounds__(256)
 copy_blocks_kernel(uint8_t* __restrict__ key_cache, uint8_t* __restrict__ value_cache,
@@ -72,6 +98,21 @@ copy_blocks_kernel(uint8_t* __restrict__ key_cache, uint8_t* __restrict__ value_
   const int64_t dst = block_mapping[2 * pair + 1];
   if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) return;
   uint8_t* base = blockIdx.y == 0 ? key_cache : value_cache;
+  const uint4* s = reinterpret_cast<const uint4*>(base + src * block_bytes);
+  uint4* d = reinterpret_cast<uint4*>(base + dst * block_bytes);
+  const int64_t n = block_bytes / 16;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) d[i] = s[i];
+}
+
+// Copy-on-write over all layers in one launch: grid (pairs, key|value, layers).
+__global__ void __launch_bounds__(256)
+copy_blocks_layers_kernel(void* const* __restrict__ key_caches, void* const* __restrict__ value_caches,
+                          const int64_t* __restrict__ block_mapping, int64_t block_bytes, int num_blocks) {
+  const int pair = blockIdx.x;
+  const int64_t src = block_mapping[2 * pair];
+  const int64_t dst = block_mapping[2 * pair + 1];
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) return;
+  uint8_t* base = static_cast<uint8_t*>(blockIdx.y == 0 ? key_caches[blockIdx.z] : value_caches[blockIdx.z]);
   const uint4* s = reinterpret_cast<const uint4*>(base + src * block_bytes);
   uint4* d = reinterpret_cast<uint4*>(base + dst * block_bytes);
   const int64_t n = block_bytes / 16;

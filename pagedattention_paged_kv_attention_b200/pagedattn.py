@@ -14,7 +14,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIBRARY_PATH = os.path.join(_HERE, "libpagedattn.so")
 
-PA_OK, PA_ERR_INVALID_ARGUMENT, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL, PA_ERR_CUDA = range(5)
+PA_OK, PA_ERR_INVALID_ARGUMENT, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL, PA_ERR_CUDA, PA_ERR_OUT_OF_BLOCKS = range(6)
 PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
 PA_DEVERR_BLOCK_ID, PA_DEVERR_CONTEXT_LEN, PA_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 WORKSPACE_HEADER_BYTES = 256
@@ -24,7 +24,11 @@ EXPORTS = (
     "pa_paged_attention_partition_size", "pa_paged_attention_workspace_size", "pa_paged_attention",
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_copy_blocks_check", "pa_get_device_error",
     "pa_clear_device_error", "pa_status_string", "pa_paged_attention_static", "pa_selftest_wait_timeout",
-    "pa_swap_blocks",
+    "pa_swap_blocks", "pa_reshape_and_cache_layers", "pa_copy_blocks_layers",
+    # include/pa_block_manager.h
+    "pa_bm_create", "pa_bm_destroy", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_append_slots",
+    "pa_bm_block_tables", "pa_bm_plan_decode", "pa_bm_free_sequence", "pa_bm_swap_out", "pa_bm_swap_in",
+    "pa_bm_num_free_blocks", "pa_bm_sequence_info", "pa_bm_ref_count",
 )
 
 if not os.path.exists(LIBRARY_PATH):
@@ -49,6 +53,39 @@ lib.pa_reshape_and_cache.restype = _i
 lib.pa_reshape_and_cache.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 lib.pa_copy_blocks.restype = _i
 lib.pa_copy_blocks.argtypes = [_p, _p, _i, _p, _i, _i, _i, _i, _i, _p]
+lib.pa_reshape_and_cache_layers.restype = _i
+lib.pa_reshape_and_cache_layers.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]
+lib.pa_copy_blocks_layers.restype = _i
+lib.pa_copy_blocks_layers.argtypes = [_p, _p, _i, _i, _p, _i, _i, _i, _i, _i, _p]
+_i64 = ctypes.c_int64
+_ip = ctypes.POINTER(ctypes.c_int)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+lib.pa_bm_create.restype = _i
+lib.pa_bm_create.argtypes = [_i, _i, _i, ctypes.POINTER(_p)]
+lib.pa_bm_destroy.restype = None
+lib.pa_bm_destroy.argtypes = [_p]
+lib.pa_bm_add_sequence.restype = _i
+lib.pa_bm_add_sequence.argtypes = [_p, _i64, _i64, _i64, _i64, _p, _i64, _i64p]
+lib.pa_bm_fork.restype = _i
+lib.pa_bm_fork.argtypes = [_p, _i64, _i64]
+lib.pa_bm_append_slots.restype = _i
+lib.pa_bm_append_slots.argtypes = [_p, _p, _i, _p, _p, _ip]
+lib.pa_bm_block_tables.restype = _i
+lib.pa_bm_block_tables.argtypes = [_p, _p, _i, _p, _i, ctypes.c_int32, _p]
+lib.pa_bm_plan_decode.restype = _i
+lib.pa_bm_plan_decode.argtypes = [_p, _p, _i, _p, _p, _ip, _p, _i, ctypes.c_int32, _p]
+lib.pa_bm_free_sequence.restype = _i
+lib.pa_bm_free_sequence.argtypes = [_p, _i64]
+lib.pa_bm_swap_out.restype = _i
+lib.pa_bm_swap_out.argtypes = [_p, _i64, _p, _i, _ip]
+lib.pa_bm_swap_in.restype = _i
+lib.pa_bm_swap_in.argtypes = [_p, _i64, _p, _i, _ip]
+lib.pa_bm_num_free_blocks.restype = _i
+lib.pa_bm_num_free_blocks.argtypes = [_p, _ip, _ip]
+lib.pa_bm_sequence_info.restype = _i
+lib.pa_bm_sequence_info.argtypes = [_p, _i64, _i64p, _ip, _ip]
+lib.pa_bm_ref_count.restype = _i
+lib.pa_bm_ref_count.argtypes = [_p, _i, _ip]
 lib.pa_swap_blocks.restype = _i
 lib.pa_swap_blocks.argtypes = [_p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _p]
 lib.pa_copy_blocks_check.restype = _i
@@ -157,6 +194,37 @@ def copy_blocks(key_cache, value_cache, block_mapping, stream=None):
     st = lib.pa_copy_blocks(_ptr(key_cache), _ptr(value_cache), dtype_code(key_cache.dtype), _ptr(block_mapping),
                             block_mapping.shape[0], Hkv, d, bs, NB, _stream(stream))
     _check(st, "pa_copy_blocks")
+
+
+def pointer_array(tensors, device="cuda"):
+    """A device int64 array holding the data pointers of `tensors` (for the *_layers calls)."""
+    return torch.tensor([t.data_ptr() for t in tensors], dtype=torch.int64, device=device)
+
+
+def reshape_and_cache_layers(keys, values, key_caches, value_caches, slot_mapping, k_scales=None, v_scales=None,
+                             stream=None):
+    """reshape_and_cache over all layers in one launch; arguments are per-layer lists of tensors."""
+    L = len(key_caches)
+    T, Hkv, d = keys[0].shape
+    NB, bs = key_caches[0].shape[0], key_caches[0].shape[1]
+    arrays = [pointer_array(x) for x in (keys, values, key_caches, value_caches)]
+    ks = pointer_array(k_scales) if k_scales is not None else None
+    vs = pointer_array(v_scales) if v_scales is not None else None
+    st = lib.pa_reshape_and_cache_layers(*[_ptr(a) for a in arrays[:2]], dtype_code(keys[0].dtype),
+                                         *[_ptr(a) for a in arrays[2:]], dtype_code(key_caches[0].dtype), _ptr(ks),
+                                         _ptr(vs), _ptr(slot_mapping), T, L, Hkv, d, bs, NB, _stream(stream))
+    _check(st, "pa_reshape_and_cache_layers")
+    return arrays  # keep the pointer arrays alive until the stream has used them
+
+
+def copy_blocks_layers(key_caches, value_caches, block_mapping, stream=None):
+    """copy_blocks over all layers in one launch (per-layer lists of cache tensors)."""
+    NB, bs, Hkv, d = key_caches[0].shape
+    kp, vp = pointer_array(key_caches), pointer_array(value_caches)
+    st = lib.pa_copy_blocks_layers(_ptr(kp), _ptr(vp), len(key_caches), dtype_code(key_caches[0].dtype),
+                                   _ptr(block_mapping), block_mapping.shape[0], Hkv, d, bs, NB, _stream(stream))
+    _check(st, "pa_copy_blocks_layers")
+    return kp, vp
 
 
 def swap_blocks(dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, block_mapping, stream=None):

@@ -8,7 +8,8 @@ import re
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "pagedattn.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if h.endswith(".h")]
 
 
 @pytest.fixture(scope="module")
@@ -20,7 +21,7 @@ def P():
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    text = "".join(open(h).read() for h in HEADERS)
     return sorted(set(re.findall(r"PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", text)))
 
 
@@ -111,3 +112,25 @@ def test_copy_blocks_check_on_host_mappings(P):
     assert not P.copy_blocks_check(torch.tensor([[0, 5], [5, 6]]), 8)      # destination is a source
     assert not P.copy_blocks_check(torch.tensor([[0, 8]]), 8)              # outside the pool
     assert P.copy_blocks_check(torch.zeros((0, 2), dtype=torch.int64), 8)
+
+
+def test_layer_ops_reject_bad_arguments(P):
+    L = P.lib
+    ok = dict(keys=16, values=16, in_dtype=P.PA_BF16, key_caches=16, value_caches=16, kv_dtype=P.PA_BF16,
+              k_scales=None, v_scales=None, slot_mapping=16, num_tokens=3, num_layers=4, num_kv_heads=2,
+              head_size=64, block_size=16, num_blocks=4, stream=None)
+
+    def rc(**over):
+        a = dict(ok)
+        a.update(over)
+        return L.pa_reshape_and_cache_layers(*a.values())
+
+    assert rc(keys=None) == 1 and rc(key_caches=12) == 1 and rc(num_layers=-1) == 1
+    assert rc(kv_dtype=P.PA_FP8_E4M3) == 1                 # no scale arrays
+    assert rc(kv_dtype=P.PA_F16) == 2 and rc(head_size=60) == 2 and rc(num_layers=70000) == 2
+    assert rc(num_tokens=0) == 0 and rc(num_layers=0) == 0
+    cb = L.pa_copy_blocks_layers
+    assert cb(None, 16, 4, P.PA_BF16, 16, 3, 2, 64, 16, 4, None) == 1
+    assert cb(16, 16, 4, P.PA_BF16, None, 3, 2, 64, 16, 4, None) == 1
+    assert cb(16, 16, 4, P.PA_BF16, 16, 3, 1, 4, 1, 4, None) == 2          # an 8-byte block: not 16-byte vectors
+    assert cb(16, 16, 4, P.PA_BF16, 16, 0, 2, 64, 16, 4, None) == 0        # no pairs
