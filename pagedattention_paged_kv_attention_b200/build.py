@@ -2,8 +2,8 @@
 
     python -m pagedattention_paged_kv_attention_b200.build [--force] [-D NAME=VALUE ...]
 
-Each .cu translation unit is compiled in parallel, then linked into one shared library next to this
-file. The library exports only the C ABI declared in include/pagedattn.h.
+Each translation unit (.cu, and the host-only .cpp) is compiled in parallel, then linked into one shared library next to this
+file. The library exports only the C ABI declared in include/*.h.
 """
 import concurrent.futures
 import os
@@ -17,7 +17,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(HERE, "libpagedattn.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
-SOURCES = ["pa_api.cu", "pa_attention_bf16.cu", "pa_attention_f16.cu", "pa_static_workspace.cu"]
+SOURCES = ["pa_api.cu", "pa_attention_bf16.cu", "pa_attention_f16.cu", "pa_static_workspace.cu",
+           "pa_block_manager.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
@@ -43,7 +44,7 @@ def build(force=False, defines=(), output=None, verbose=False):
     dflags = [f"-D{d}" for d in defines]
 
     def compile_one(src):
-        obj = os.path.join(build_dir, src.replace(".cu", ".o"))
+        obj = os.path.join(build_dir, os.path.splitext(src)[0] + ".o")
         cmd = [NVCC, *ARCH, *FLAGS, *dflags, "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             cmd += ["-Xptxas", "-v"]
@@ -58,8 +59,7 @@ def build(force=False, defines=(), output=None, verbose=False):
         for _, log in results:
             sys.stderr.write(log)
     tmp = output + f".tmp{os.getpid()}"
-    link = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *[o for o, _ in results], "-lcuda"
-            if False else "-ldl"]
+    link = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *[o for o, _ in results], "-ldl"]
     r = subprocess.run(link, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")
