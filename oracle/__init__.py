@@ -54,6 +54,8 @@ def _bind(path):
     L.or_paged_attention.restype = i
     L.or_paged_attention.argtypes = [p, p, i, p, p, i, p, p, p, i, p, i, i, i, i, i, i,
                                      ctypes.c_double, i]
+    L.or_paged_prefill.restype = i
+    L.or_paged_prefill.argtypes = [p, p, i, p, p, i, p, p, p, i, p, p, i, i, i, i, i, i, ctypes.c_double, i]
     L.or_reshape_and_cache.restype = i
     L.or_reshape_and_cache.argtypes = [p, p, i, p, p, i, p, p, p, i64, i, i, i, i64]
     L.or_copy_blocks.restype = i
@@ -178,6 +180,35 @@ def paged_attention(query_bits, q_dtype, key_cache, value_cache, kv_dtype, block
                                   num_threads or default_threads())
     if st != 0:
         raise OracleError(f"or_paged_attention failed with status {st}")
+    return out
+
+
+def paged_prefill(query_bits, q_dtype, key_cache, value_cache, kv_dtype, block_tables, context_lens,
+                  q_start, scale, k_scale=None, v_scale=None, num_threads=None):
+    """fp64 output [T, H, d] of causal paged prefill attention (definition in pa_oracle.c).
+
+    query_bits: uint16 [T, H, d], the query chunks of all sequences back to back; q_start: int32
+    [S + 1] row offsets (q_start[0] = 0, q_start[S] = T); context_lens: int32 [S], each including
+    its chunk; other arguments as in paged_attention.
+    """
+    q = _c(query_bits, np.uint16)
+    kc = key_cache if key_cache.flags.c_contiguous else np.ascontiguousarray(key_cache)
+    vc = value_cache if value_cache.flags.c_contiguous else np.ascontiguousarray(value_cache)
+    bt = _c(block_tables, np.int32)
+    cl = _c(context_lens, np.int32)
+    qs = _c(q_start, np.int32)
+    T, H, d = q.shape
+    NB, bs, Hkv, d2 = kc.shape
+    S = cl.shape[0]
+    assert d2 == d and vc.shape == kc.shape and bt.shape[0] == S and qs.shape == (S + 1,) and qs[-1] == T
+    ks = None if k_scale is None else _c(k_scale, np.float32)
+    vs = None if v_scale is None else _c(v_scale, np.float32)
+    out = np.zeros((T, H, d), np.float64)
+    st = lib().or_paged_prefill(_ptr(out), _ptr(q), dtype_code(q_dtype), _ptr(kc), _ptr(vc), dtype_code(kv_dtype),
+                                _ptr(ks), _ptr(vs), _ptr(bt), bt.shape[1], _ptr(cl), _ptr(qs), S, H, Hkv, d, bs,
+                                NB, float(scale), num_threads or default_threads())
+    if st != 0:
+        raise OracleError(f"or_paged_prefill failed with status {st}")
     return out
 
 

@@ -378,3 +378,142 @@ int or_swap_blocks(void* dst_key_cache, void* dst_value_cache, const void* src_k
   return OR_OK;
 }
 
+
+/* ------------------------------------------------------------------------------------------------
+ * Paged prefill attention: a chunk of new query tokens per sequence over the paged cache, causal.
+ * Prefill (the prompt) is the compute-bound phase ([C] "对 agent 开发者的启示"); each token attends
+ * only to the keys and values of its prefix ([C] "PagedAttention：把显存做成虚拟内存": a token needs
+ * the KV of the tokens before it), with the [T] sec. 2.2 formula over that prefix.
+ *
+ * Sequence s has n_s = q_start[s+1] - q_start[s] query rows (rows q_start[s] .. q_start[s+1]-1 of
+ * query/out), and L_s = context_lens[s] cached tokens that already include the chunk's own keys and
+ * values. The chunk is the last n_s of those tokens (reading: a chunk continues the sequence), so
+ * query j of the chunk sits at position p = L_s - n_s + j and attends to t = 0 .. p:
+ *   z_t = scale * sum_i q[row][h][i] * k_t[i],  out[row][h][:] = sum_t exp(z_t - m) v_t / sum_t exp(z_t - m)
+ * with m = max_t z_t, k_t and v_t found through block_tables[s] as in decode.
+ * --------------------------------------------------------------------------------------------- */
+typedef struct {
+  double* out;                 /* [T][H][d] */
+  const void* query;           /* [T][H][d] in q_dtype */
+  int q_dtype;
+  const void* key_cache;
+  const void* value_cache;
+  int kv_dtype;
+  const float* k_scale;
+  const float* v_scale;
+  const int32_t* block_tables; /* [S][max_blocks_per_seq] */
+  int max_blocks_per_seq;
+  const int32_t* context_lens; /* [S] */
+  const int32_t* q_start;      /* [S + 1] */
+  int num_seqs, num_heads, num_kv_heads, head_size, block_size, num_blocks;
+  double scale;
+  int num_threads, thread_index, status;
+} or_prefill_job;
+
+static int prefill_one(const or_prefill_job* a, int s, int row, int h, double* z) {
+  const int d = a->head_size;
+  const int kvh = h / (a->num_heads / a->num_kv_heads);
+  const int n = a->q_start[s + 1] - a->q_start[s];
+  const int j = row - a->q_start[s];
+  const int p = a->context_lens[s] - n + j; /* position of this query token */
+  const size_t q_base = ((size_t)row * a->num_heads + h) * d;
+  double* o = a->out + q_base;
+  const double ks = (a->kv_dtype == OR_E4M3) ? (double)a->k_scale[kvh] : 1.0;
+  const double vs = (a->kv_dtype == OR_E4M3) ? (double)a->v_scale[kvh] : 1.0;
+  for (int i = 0; i < d; ++i) o[i] = 0.0;
+  for (int t = 0; t <= p; ++t) {
+    int blk = a->block_tables[(size_t)s * a->max_blocks_per_seq + t / a->block_size];
+    if (blk < 0 || blk >= a->num_blocks) return OR_BAD_BLOCK;
+    size_t k_base = (((size_t)blk * a->block_size + t % a->block_size) * a->num_kv_heads + kvh) * d;
+    double dot = 0.0;
+    for (int i = 0; i < d; ++i)
+      dot += element(a->query, a->q_dtype, q_base + i) * (element(a->key_cache, a->kv_dtype, k_base + i) * ks);
+    z[t] = a->scale * dot;
+  }
+  double m = z[0];
+  for (int t = 1; t <= p; ++t)
+    if (z[t] > m) m = z[t];
+  double denom = 0.0;
+  for (int t = 0; t <= p; ++t) denom += exp(z[t] - m);
+  for (int t = 0; t <= p; ++t) {
+    int blk = a->block_tables[(size_t)s * a->max_blocks_per_seq + t / a->block_size];
+    size_t v_base = (((size_t)blk * a->block_size + t % a->block_size) * a->num_kv_heads + kvh) * d;
+    double w = exp(z[t] - m) / denom;
+    for (int i = 0; i < d; ++i) o[i] += w * (element(a->value_cache, a->kv_dtype, v_base + i) * vs);
+  }
+  return OR_OK;
+}
+
+static void* prefill_worker(void* arg) {
+  or_prefill_job* a = (or_prefill_job*)arg;
+  int max_len = 1;
+  for (int s = 0; s < a->num_seqs; ++s)
+    if (a->context_lens[s] > max_len) max_len = a->context_lens[s];
+  double* z = (double*)malloc(sizeof(double) * (size_t)max_len);
+  if (!z) {
+    a->status = OR_NO_MEMORY;
+    return NULL;
+  }
+  const long rows = a->q_start[a->num_seqs];
+  const long total = rows * a->num_heads;
+  int s = 0;
+  for (long item = a->thread_index; item < total; item += a->num_threads) {
+    int row = (int)(item / a->num_heads), h = (int)(item % a->num_heads);
+    while (a->q_start[s + 1] <= row) ++s; /* rows are visited in increasing order */
+    int st = prefill_one(a, s, row, h, z);
+    if (st != OR_OK) {
+      a->status = st;
+      break;
+    }
+  }
+  free(z);
+  return NULL;
+}
+
+int or_paged_prefill(double* out, const void* query, int q_dtype, const void* key_cache,
+                     const void* value_cache, int kv_dtype, const float* k_scale, const float* v_scale,
+                     const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                     const int32_t* q_start, int num_seqs, int num_heads, int num_kv_heads, int head_size,
+                     int block_size, int num_blocks, double scale, int num_threads) {
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens || !q_start) return OR_BAD_ARG;
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return OR_BAD_ARG;
+  if (head_size <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq < 0) return OR_BAD_ARG;
+  if (q_dtype != OR_F16 && q_dtype != OR_BF16) return OR_BAD_ARG;
+  if (kv_dtype != OR_F16 && kv_dtype != OR_BF16 && kv_dtype != OR_E4M3) return OR_BAD_ARG;
+  if (kv_dtype == OR_E4M3 && (!k_scale || !v_scale)) return OR_BAD_ARG;
+  if (q_start[0] != 0) return OR_BAD_ARG;
+  for (int s = 0; s < num_seqs; ++s) {
+    int n = q_start[s + 1] - q_start[s];
+    if (n < 0 || n > context_lens[s]) return OR_BAD_ARG; /* a chunk lies inside its context */
+    if ((long)context_lens[s] > (long)max_blocks_per_seq * block_size) return OR_BAD_ARG;
+  }
+  if (num_threads < 1) num_threads = 1;
+  or_prefill_job base = {out, query, q_dtype, key_cache, value_cache, kv_dtype, k_scale, v_scale,
+                         block_tables, max_blocks_per_seq, context_lens, q_start, num_seqs, num_heads,
+                         num_kv_heads, head_size, block_size, num_blocks, scale, num_threads, 0, OR_OK};
+  or_prefill_job* jobs = (or_prefill_job*)malloc(sizeof(or_prefill_job) * (size_t)num_threads);
+  pthread_t* threads = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)num_threads);
+  if (!jobs || !threads) {
+    free(jobs);
+    free(threads);
+    return OR_NO_MEMORY;
+  }
+  int started = 0;
+  for (int t = 0; t < num_threads; ++t) {
+    jobs[t] = base;
+    jobs[t].thread_index = t;
+  }
+  for (int t = 1; t < num_threads; ++t) {
+    if (pthread_create(&threads[t], NULL, prefill_worker, &jobs[t]) != 0) break;
+    started = t;
+  }
+  for (int t = started + 1; t < num_threads; ++t) prefill_worker(&jobs[t]);
+  prefill_worker(&jobs[0]);
+  for (int t = 1; t <= started; ++t) pthread_join(threads[t], NULL);
+  int status = OR_OK;
+  for (int t = 0; t < num_threads; ++t)
+    if (jobs[t].status != OR_OK) status = jobs[t].status;
+  free(jobs);
+  free(threads);
+  return status;
+}
