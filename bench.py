@@ -214,7 +214,7 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--op", default="decode", choices=["decode", "swap", "layers"],
+    ap.add_argument("--op", default="decode", choices=["decode", "swap", "layers", "plan"],
                     help="decode: the decode step (default); swap: swap_blocks host<->device throughput")
     ap.add_argument("--workload", default="7b", choices=list(W.CONFIGS))
     ap.add_argument("--partition-size", type=int, default=None,
@@ -235,9 +235,9 @@ def main():
         args.partition_size = cfg.partition_size
     world, rank, local = dist_setup(args)
 
-    if args.op in ("swap", "layers"):
+    if args.op in ("swap", "layers", "plan"):
         if rank == 0:
-            (run_swap if args.op == "swap" else run_layers)(args, cfg)
+            {"swap": run_swap, "layers": run_layers, "plan": run_plan}[args.op](args, cfg)
         if world > 1:
             torch.distributed.destroy_process_group()
         return
@@ -509,6 +509,53 @@ def run_layers(args, cfg, num_layers=32, pool_blocks=2048, cow_pairs=64):
                          "frac": round(gbs(total, t_fused) / peak, 3) if peak else None, "traffic": None,
                          "peak_source": "measured" if peak else None},
             "clocks": clocks.summary(), "gpu_launches": 2 * args.steps}
+    print(json.dumps(line), flush=True)
+
+
+def run_plan(args, cfg, plan_steps=200):
+    """Host cost of the block manager per decode step: the workload's batch is admitted (prompts of
+    its context lengths), then plan_steps decode plans (one new token for every sequence: slots,
+    copy-on-write pairs, block tables, lengths, written into pinned buffers) are timed on the host
+    clock. Beside it the oracle's manager doing the same steps (the reference arm of this part)."""
+    from pagedattention_paged_kv_attention_b200.block_manager import BlockManager
+    from oracle.block_manager import BlockManagerOracle
+    lens = W._lengths(cfg, np.random.default_rng(W.sub_seeds(cfg.seed)[0]), cfg.num_seqs).tolist()
+    S, bs = len(lens), cfg.block_size
+    grow = plan_steps + args.warmup
+    need = sum(-(-(L + grow) // bs) for L in lens)
+    max_blocks = max(-(-(L + grow) // bs) for L in lens)
+    ids = list(range(S))
+
+    def admit(bm):
+        for i, L in enumerate(lens):
+            bm.add_sequence(i, int(L))
+
+    bm = BlockManager(need + 16, bs)
+    admit(bm)
+    out = (torch.empty(S, dtype=torch.int64).pin_memory(), torch.empty((S, 2), dtype=torch.int64).pin_memory(),
+           torch.empty((S, max_blocks), dtype=torch.int32).pin_memory(), torch.empty(S, dtype=torch.int32).pin_memory())
+    for _ in range(args.warmup):
+        bm.plan_decode(ids, max_blocks, 0, out)
+    t0 = time.perf_counter()
+    for _ in range(plan_steps):
+        bm.plan_decode(ids, max_blocks, 0, out)
+    t_native = (time.perf_counter() - t0) / plan_steps
+    ref = BlockManagerOracle(need + 16, bs)
+    admit(ref)
+    ref_steps = max(1, plan_steps // 10)
+    t0 = time.perf_counter()
+    for _ in range(ref_steps):
+        ref.append_slots(ids)
+        ref.block_tables(ids, max_blocks)
+    t_ref = (time.perf_counter() - t0) / ref_steps
+    line = {"metric": "block-manager decode plan: sequences planned per second", "value": round(S / t_native),
+            "unit": "seq/s", "impl": "ours", "n_gpus": 1, "steps": plan_steps, "warmup": args.warmup, "ms_per_step": round(t_native * 1e3, 4), "higher_is_better": True, "dtype": "int64",
+            "data": "synthetic",
+            "config": {"workload": f"{cfg.name} batch: {S} sequences, context {min(lens)}..{max(lens)}, block "
+                                   f"{bs}, one token per sequence per step into pinned buffers"},
+            "cpu_baseline": {"value": round(S / t_ref), "unit": "seq/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{ref_steps} steps of the oracle's manager on the same batch"},
+            "gpu_launches": 0}
     print(json.dumps(line), flush=True)
 
 

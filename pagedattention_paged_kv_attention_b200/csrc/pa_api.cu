@@ -16,6 +16,7 @@
 #include <unordered_set>
 
 #include "pa_cache_ops.cuh"
+#include "pa_host_util.h"
 #include "pa_launch.cuh"
 #include "pagedattn.h"
 
@@ -26,9 +27,13 @@ constexpr int kPlanItemsPerCta = 16;     // work items per persistent CTA the au
 constexpr int kMinAutoPartition = 256;
 constexpr int kMaxAutoPartition = 1024;
 
-bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-int ceil_div(int a, int b) { return (a + b - 1) / b; }
+using pa_host::aligned;
+using pa_host::ceil_div;
+using pa_host::elem_bytes;
+using pa_host::is_16bit;
+using pa_host::is_dtype;
+using pa_host::round_up;
+using pa_host::tensor_map_encoder;
 
 // Query heads handled per CTA (the kernel template's G) and CTAs per kv head.
 void group_tiling(int group, int* g_tile, int* subgroups) {
@@ -72,19 +77,6 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_size, int
   return w;
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // 4-D view of a cache; box = one 128-byte chunk of the rows of 8 consecutive tokens for 8 consecutive
 // kv heads of one block (heads past the last one read as zeros), written to shared memory with the
 // 128-byte swizzle.
@@ -108,9 +100,6 @@ bool encode_cache_map(CUtensorMap* map, const void* cache, int elem_bytes, int h
   return r == CUDA_SUCCESS;
 }
 
-bool is_16bit(pa_dtype t) { return t == PA_F16 || t == PA_BF16; }
-bool is_dtype(pa_dtype t) { return t == PA_F16 || t == PA_BF16 || t == PA_FP8_E4M3; }
-int elem_bytes(pa_dtype t) { return t == PA_FP8_E4M3 ? 1 : 2; }
 bool supported_block_size(int bs) { return bs == 8 || bs == 16 || bs == 32 || bs == 64; }
 
 }  // namespace
