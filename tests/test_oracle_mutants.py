@@ -82,9 +82,13 @@ def test_unmutated_oracle_passes_the_selection():
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_planted_mistake_is_caught(tmp_path, name, old, new):
     text = open(SRC).read()
-    assert text.count(old) == 1, f"mutation anchor for {name} not unique"
+    # The mistakes are planted in the codecs and the decode definition, which come before the
+    # decode worker; later functions (prefill, cache operations) are left as they are.
+    cut = text.index("static void* attention_worker(")
+    head, tail = text[:cut], text[cut:]
+    assert head.count(old) == 1, f"mutation anchor for {name} not unique"
     src = tmp_path / "mutant.c"
-    src.write_text(text.replace(old, new))
+    src.write_text(head.replace(old, new) + tail)
     lib = tmp_path / f"libmutant_{name}.so"
     subprocess.run(["gcc", "-std=c11", "-O1", "-fPIC", "-shared", "-pthread", "-o", str(lib), str(src), "-lm"],
                    check=True)
