@@ -163,6 +163,37 @@ PA_API pa_status pa_paged_attention_static(void* out, const void* query, pa_dtyp
                                     unsigned int* device_error_out, pa_stream_t stream);
 
 /*
+ * Causal paged prefill attention: a chunk of new query tokens per sequence attends to its prefix in
+ * the paged cache (page "PagedAttention 与连续批处理：LLM Serving 的底层架构拆解": prefill is the
+ * compute-bound phase, section "对 agent 开发者的启示", and a token attends to the tokens before it,
+ * section "PagedAttention：把显存做成虚拟内存"; formula of the tutorial page "企业官网建设流程全解析",
+ * sec. 2.2). Sequence s owns query rows q_start[s] .. q_start[s+1]-1 (n_s rows); its cache holds
+ * context_lens[s] = L_s >= n_s tokens INCLUDING the chunk's own keys and values (write them with
+ * pa_reshape_and_cache first), and the chunk is the last n_s of them. For query j of the chunk at
+ * position p = L_s - n_s + j and every head h (kv head h / (num_heads / num_kv_heads)):
+ *     out[q_start[s] + j][h][:] = softmax_t<=p(scale * q . k_t) . v_t       (fp32 accumulation)
+ * Runs on the tcgen05 tensor cores: 128 query rows (128/G tokens x G grouped heads) per CTA.
+ *
+ *  out, query     [num_q_tokens][num_heads][head_size], q_dtype (PA_F16 / PA_BF16); 16-byte aligned.
+ *  key_cache,
+ *  value_cache    [num_blocks][block_size][num_kv_heads][head_size], kv_dtype == q_dtype.
+ *  block_tables   [num_seqs][max_blocks_per_seq] int32; context_lens [num_seqs] int32;
+ *  q_start        [num_seqs + 1] int32, non-decreasing, q_start[0] = 0, q_start[num_seqs] = num_q_tokens.
+ *  max_q_len      >= max_s n_s (sizes the grid; tiles past a sequence's chunk exit at once).
+ *  workspace      >= PA_WORKSPACE_HEADER_BYTES, zeroed once; its first word is the device error word
+ *                 (read with pa_get_device_error).
+ * Supported: head_size 64 or 128; block_size 8, 16, 32, 64 or 128; num_heads / num_kv_heads dividing
+ * 128. A chunk outside its context (n_s > L_s, or L_s beyond the block table) sets
+ * PA_DEVERR_CONTEXT_LEN and NaNs its rows; a block id outside the pool sets PA_DEVERR_BLOCK_ID.
+ */
+PA_API pa_status pa_paged_prefill(void* out, const void* query, pa_dtype q_dtype, const void* key_cache,
+                                  const void* value_cache, pa_dtype kv_dtype, const int32_t* block_tables,
+                                  int max_blocks_per_seq, const int32_t* context_lens, const int32_t* q_start,
+                                  int num_seqs, int num_q_tokens, int num_heads, int num_kv_heads, int head_size,
+                                  int block_size, int num_blocks, int max_q_len, float scale, void* workspace,
+                                  size_t workspace_bytes, pa_stream_t stream);
+
+/*
  * Write new tokens into their physical slots ([V] "PagedAttention的破局思路": blocks are filled as the
  * sequence grows). For token i with slot = slot_mapping[i] in [0, num_blocks*block_size):
  *     key_cache[slot / block_size][slot % block_size][h][:] = key[i][h][:]   (same for value)

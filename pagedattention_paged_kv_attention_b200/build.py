@@ -18,7 +18,7 @@ LIBRARY = os.path.join(HERE, "libpagedattn.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 SOURCES = ["pa_api.cu", "pa_attention_bf16.cu", "pa_attention_f16.cu", "pa_static_workspace.cu",
-           "pa_block_manager.cpp"]
+           "pa_prefill.cu", "pa_block_manager.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

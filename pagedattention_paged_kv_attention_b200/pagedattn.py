@@ -24,7 +24,7 @@ EXPORTS = (
     "pa_paged_attention_partition_size", "pa_paged_attention_workspace_size", "pa_paged_attention",
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_copy_blocks_check", "pa_get_device_error",
     "pa_clear_device_error", "pa_status_string", "pa_paged_attention_static", "pa_selftest_wait_timeout",
-    "pa_swap_blocks", "pa_reshape_and_cache_layers", "pa_copy_blocks_layers",
+    "pa_swap_blocks", "pa_reshape_and_cache_layers", "pa_copy_blocks_layers", "pa_paged_prefill",
     # include/pa_block_manager.h
     "pa_bm_create", "pa_bm_destroy", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_append_slots",
     "pa_bm_block_tables", "pa_bm_plan_decode", "pa_bm_free_sequence", "pa_bm_swap_out", "pa_bm_swap_in",
@@ -49,6 +49,9 @@ lib.pa_paged_attention.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _p, _
 lib.pa_paged_attention_static.restype = _i
 lib.pa_paged_attention_static.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i,
                                           _f, _i, _p, _p]
+lib.pa_paged_prefill.restype = _i
+lib.pa_paged_prefill.argtypes = [_p, _p, _i, _p, _p, _i, _p, _i, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _sz,
+                                 _p]
 lib.pa_reshape_and_cache.restype = _i
 lib.pa_reshape_and_cache.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 lib.pa_copy_blocks.restype = _i
@@ -159,6 +162,20 @@ def paged_attention(out, query, key_cache, value_cache, block_tables, context_le
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "pa_paged_attention")
     return out
+
+
+def paged_prefill(out, query, key_cache, value_cache, block_tables, context_lens, q_start, scale, max_q_len,
+                  workspace, stream=None):
+    """Causal prefill: out[T,H,d] for query chunks query[T,H,d] (rows q_start[s]..q_start[s+1]-1 of
+    sequence s, the last rows of its context_lens[s] cached tokens) over key/value_cache[NB,bs,Hkv,d]."""
+    T, H, d = query.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    st = lib.pa_paged_prefill(_ptr(out), _ptr(query), dtype_code(query.dtype), _ptr(key_cache), _ptr(value_cache),
+                              dtype_code(key_cache.dtype), _ptr(block_tables), block_tables.shape[1],
+                              _ptr(context_lens), _ptr(q_start), context_lens.shape[0], T, H, Hkv, d, bs, NB,
+                              int(max_q_len), float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream))
+    _check(st, "pa_paged_prefill")
 
 
 def paged_attention_static(out, query, key_cache, value_cache, block_tables, context_lens, scale,

@@ -278,3 +278,170 @@ def ideal_bytes(context_lens, num_kv_heads: int, head_size: int, kv_elem_bytes: 
     ids = int(((lens + block_size - 1) // block_size).sum()) * 4
     q = len(lens) * num_heads * head_size * q_elem_bytes
     return {"kv": kv, "block_ids": ids, "query": q, "out": q, "total": kv + ids + 2 * q}
+
+
+# ------------------------------------------------------------------------------------------------
+# Prefill (a chunk of new query tokens per sequence, causal over its prefix).
+#
+# Recipe: context lengths as above (explicit or uniform); each sequence's chunk is its last
+# n_s = min(chunk, L_s) tokens (chunk None: the whole prompt, n_s = L_s); the pool holds every context
+# token except the chunk's, whose slots are NaN until the step writes them (the chunk's keys and values
+# are returned as new_key/new_value with their slot_mapping, in row order); the query rows are the
+# chunks back to back (q_start the prefix sums of n_s); N(0,1) values drawn in logical order; random
+# block placement over a pool of ceil(1.2 x needed) blocks plus a NaN poison block for padding.
+# ------------------------------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class PrefillConfig:
+    name: str
+    description: str
+    num_seqs: int
+    num_heads: int
+    num_kv_heads: int
+    head_size: int
+    block_size: int
+    dtype: str
+    seed: int
+    context_lens: Optional[Sequence[int]] = None
+    len_range: Optional[tuple] = None
+    chunk: Optional[int] = None                    # None: the whole prompt is the chunk
+    scale: Optional[float] = None
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.head_size)
+
+
+PREFILL_CONFIGS = {
+    "prefill_tiny": PrefillConfig(
+        name="prefill_tiny",
+        description="small prefill: 3 prompts of 37, 128 and 200 tokens, 8 q / 2 kv heads, head_size 128, "
+                    "block_size 16, bf16",
+        num_seqs=3, num_heads=8, num_kv_heads=2, head_size=128, block_size=16, dtype="bf16", seed=11,
+        context_lens=(37, 128, 200)),
+    "prefill_7b": PrefillConfig(
+        name="prefill_7b",
+        description="7B-shape prompt prefill: 16 prompts U[1024,4096] tokens, 32 q / 32 kv heads, head_size 128, "
+                    "block_size 16, bf16, causal",
+        num_seqs=16, num_heads=32, num_kv_heads=32, head_size=128, block_size=16, dtype="bf16", seed=12,
+        len_range=(1024, 4096)),
+    "prefill_70b_gqa": PrefillConfig(
+        name="prefill_70b_gqa",
+        description="70B-shape GQA prompt prefill: 16 prompts U[1024,4096] tokens, 64 q / 8 kv heads, "
+                    "head_size 128, block_size 16, bf16, causal",
+        num_seqs=16, num_heads=64, num_kv_heads=8, head_size=128, block_size=16, dtype="bf16", seed=13,
+        len_range=(1024, 4096)),
+    "chunked_prefill": PrefillConfig(
+        name="chunked_prefill",
+        description="chunked prefill: 32 sequences with contexts U[2048,8192], the last 512 tokens of each as "
+                    "the chunk, 32 q / 8 kv heads, head_size 128, block_size 16, bf16",
+        num_seqs=32, num_heads=32, num_kv_heads=8, head_size=128, block_size=16, dtype="bf16", seed=14,
+        len_range=(2048, 8192), chunk=512),
+}
+
+
+@dataclasses.dataclass
+class PrefillWorkload:
+    cfg: PrefillConfig
+    context_lens: torch.Tensor      # int32 [S]
+    q_start: torch.Tensor           # int32 [S + 1]
+    block_tables: torch.Tensor      # int32 [S, max_blocks]
+    num_blocks: int
+    query: torch.Tensor             # [T, H, d]
+    key_values: torch.Tensor        # [NB, bs, Hkv, d]; the chunks' slots are NaN
+    value_values: torch.Tensor
+    new_key: torch.Tensor           # [T, Hkv, d]: the chunks' keys, row order
+    new_value: torch.Tensor
+    slot_mapping: torch.Tensor      # int64 [T]
+
+    @property
+    def max_q_len(self) -> int:
+        q = self.q_start
+        return int((q[1:] - q[:-1]).max().item()) if q.numel() > 1 else 0
+
+    def causal_pairs(self) -> int:
+        """(query row, visible key) pairs per head: sum over sequences of n(L-n) + n(n+1)/2."""
+        L = self.context_lens.to(torch.int64)
+        n = (self.q_start[1:] - self.q_start[:-1]).to(torch.int64)
+        return int((n * (L - n) + n * (n + 1) // 2).sum().item())
+
+
+def make_prefill_workload(cfg: PrefillConfig, seed: Optional[int] = None, device="cpu",
+                          num_seqs: Optional[int] = None,
+                          context_lens: Optional[Sequence[int]] = None,
+                          chunk_lens: Optional[Sequence[int]] = None) -> PrefillWorkload:
+    seed = cfg.seed if seed is None else seed
+    s_lens, s_perm, s_q, s_k, s_v, _, _, _ = sub_seeds(seed)
+    bs, Hkv, H, d = cfg.block_size, cfg.num_kv_heads, cfg.num_heads, cfg.head_size
+    if context_lens is not None:
+        lens = np.array(context_lens, dtype=np.int64)
+    elif cfg.context_lens is not None:
+        lens = np.array(cfg.context_lens, dtype=np.int64)
+    else:
+        lo, hi = cfg.len_range
+        lens = np.random.default_rng(s_lens).integers(lo, hi + 1, size=cfg.num_seqs, dtype=np.int64)
+    if num_seqs is not None:
+        lens = lens[:num_seqs]
+    S = len(lens)
+    if chunk_lens is not None:
+        n = np.array(chunk_lens, dtype=np.int64)
+    else:
+        n = lens.copy() if cfg.chunk is None else np.minimum(lens, cfg.chunk)
+    assert np.all(n <= lens) and np.all(n >= 0)
+    nblocks = (lens + bs - 1) // bs
+    needed = int(nblocks.sum())
+    NB = max(int(math.ceil(1.2 * needed)), needed + 1)
+    perm = np.random.default_rng(s_perm).permutation(NB)
+    used, poison = perm[:needed], int(perm[needed])
+    max_blocks = int(max(1, nblocks.max() if S else 1))
+    tables = np.full((S, max_blocks), poison, dtype=np.int64)
+    cursor = 0
+    for s in range(S):
+        tables[s, :nblocks[s]] = used[cursor:cursor + nblocks[s]]
+        cursor += int(nblocks[s])
+
+    tdtype = _TORCH_DTYPES[cfg.dtype]
+    nan_bits = _NAN_BITS[cfg.dtype]
+    dev = torch.device(device)
+
+    def gen(sd):
+        g = torch.Generator(device=dev)
+        g.manual_seed(sd)
+        return g
+
+    q_start = np.concatenate([[0], np.cumsum(n)]).astype(np.int64)
+    T = int(q_start[-1])
+    query = torch.randn((T, H, d), generator=gen(s_q), device=dev, dtype=torch.float32).to(tdtype)
+    used_t = torch.from_numpy(used.astype(np.int64)).to(dev)
+    pools = []
+    for s_vals in (s_k, s_v):
+        pool = torch.empty((NB, bs, Hkv, d), dtype=tdtype, device=dev)
+        pool.view(torch.int16).fill_(nan_bits)
+        pool[used_t] = torch.randn((needed, bs, Hkv, d), generator=gen(s_vals), device=dev,
+                                   dtype=torch.float32).to(tdtype)
+        pools.append(pool)
+    key_pool, value_pool = pools
+
+    # The chunk rows: slots of positions L-n .. L-1, their values taken out of the pool and poisoned there.
+    tables_t = torch.from_numpy(tables).to(dev)
+    seq_of_row = torch.from_numpy(np.repeat(np.arange(S), n)).to(dev)
+    pos = torch.from_numpy(np.concatenate([np.arange(L - k, L) for L, k in zip(lens, n)]) if T else
+                           np.zeros(0, np.int64)).to(dev)
+    blk = tables_t[seq_of_row, pos // bs]
+    off = pos % bs
+    new_key = key_pool[blk, off].clone()
+    new_value = value_pool[blk, off].clone()
+    key_pool[blk, off] = torch.full_like(new_key.view(torch.int16), nan_bits).view(tdtype)
+    value_pool[blk, off] = torch.full_like(new_value.view(torch.int16), nan_bits).view(tdtype)
+    # Tails of last blocks past each context stay NaN from the fill (they were drawn, so re-poison).
+    for s in range(S):
+        L = int(lens[s])
+        if L % bs:
+            b_last = int(tables[s, (L - 1) // bs])
+            key_pool[b_last, L % bs:].view(torch.int16).fill_(nan_bits)
+            value_pool[b_last, L % bs:].view(torch.int16).fill_(nan_bits)
+    return PrefillWorkload(
+        cfg=cfg, context_lens=torch.from_numpy(lens.astype(np.int32)).to(dev),
+        q_start=torch.from_numpy(q_start.astype(np.int32)).to(dev),
+        block_tables=torch.from_numpy(tables.astype(np.int32)).to(dev), num_blocks=NB,
+        query=query, key_values=key_pool, value_values=value_pool, new_key=new_key, new_value=new_value,
+        slot_mapping=(blk * bs + off).to(torch.int64))
