@@ -214,9 +214,11 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--op", default="decode", choices=["decode", "swap", "layers", "plan"],
-                    help="decode: the decode step (default); swap: swap_blocks host<->device throughput")
-    ap.add_argument("--workload", default="7b", choices=list(W.CONFIGS))
+    ap.add_argument("--op", default="decode", choices=["decode", "prefill", "swap", "layers", "plan"],
+                    help="decode: the decode step (default); prefill: the causal prefill step; swap: swap_blocks "
+                         "host<->device; layers: multi-layer cache ops; plan: the block manager's decode plan")
+    ap.add_argument("--workload", default=None, choices=list(W.CONFIGS) + list(W.PREFILL_CONFIGS),
+                    help="default: 7b (decode ops), prefill_7b (--op prefill)")
     ap.add_argument("--partition-size", type=int, default=None,
                     help="tokens per split-K partition (default: the workload's, else the library's choice)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -227,6 +229,14 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
+    if args.workload is None:
+        args.workload = "prefill_7b" if args.op == "prefill" else "7b"
+    if args.op == "prefill":
+        world, rank, local = dist_setup(args)
+        run_prefill(args, W.PREFILL_CONFIGS[args.workload], world, rank)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     cfg = W.CONFIGS[args.workload]
     if args.pool_blocks is not None:
         import dataclasses
@@ -377,6 +387,190 @@ def main():
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+
+
+def run_prefill(args, cfg, world, rank):
+    """The prefill step: reshape_and_cache of every chunk's keys and values, then causal paged prefill
+    attention. value = causal attention FLOPs (4 * d per visible (query head, key) pair) / device step
+    time; each rank runs its own batch (weak scaling). The roofline is the attention call's FLOPs over
+    its event-timed duration against the measured dense bf16 tensor peak."""
+    if args.impl == "reference":
+        return run_prefill_reference(args, cfg, world, rank)
+    from pagedattention_paged_kv_attention_b200 import pagedattn as P
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = W.make_prefill_workload(cfg, seed=cfg.seed + 1000 * rank, device=dev, num_seqs=args.num_seqs)
+    H, d = cfg.num_heads, cfg.head_size
+    flops = 4.0 * d * H * w.causal_pairs()
+    key_cache, value_cache = w.key_values, w.value_values
+    out = torch.empty_like(w.query)
+    ws = torch.zeros(64, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    mq = w.max_q_len
+
+    def step(q, nk, nv, slots, tables, lens, qs, o, ev=None):
+        P.reshape_and_cache(nk, nv, key_cache, value_cache, slots)
+        if ev is not None:
+            ev[0].record(stream)
+        P.paged_prefill(o, q, key_cache, value_cache, tables, lens, qs, cfg.softmax_scale, mq, ws)
+        if ev is not None:
+            ev[1].record(stream)
+
+    inputs = (w.query, w.new_key, w.new_value, w.slot_mapping, w.block_tables, w.context_lens, w.q_start)
+    for _ in range(args.warmup):
+        step(*inputs, out)
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_selector(dev)) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            step(*inputs, out, events[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = start.elapsed_time(stop) / args.steps
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in events]))
+    assert P.get_device_error(ws) == 0, "device error word set"
+    max_ms = reduce_max(step_ms, world, dev)
+    total_flops = reduce_sum(flops, world, dev)
+    value = total_flops / (max_ms * 1e-3) / 1e12
+
+    # end to end: pinned host inputs in, output back to pinned host memory
+    host_in = [t.cpu().pin_memory() for t in inputs]
+    dev_in = [torch.empty_like(t) for t in inputs]
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for dst, src in zip(dev_in, host_in):
+            dst.copy_(src, non_blocking=True)
+        step(*dev_in, out)
+        host_out.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(a0.elapsed_time(a1) / args.steps, world, dev)
+    e2e_value = total_flops / (e2e_ms * 1e-3) / 1e12
+
+    if rank != 0:
+        return
+    peaks = measured_peaks()
+    peak = peaks.get("bf16_tflops") if peaks else 1590.0
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    T = w.query.shape[0]
+    line = {"metric": "paged prefill attention: causal TFLOP/s", "value": round(value, 2), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+            "data": "synthetic",
+            "config": {"workload": cfg.description, "name": cfg.name, "num_seqs": cfg.num_seqs, "query_tokens": T,
+                       "causal_pairs_per_head": w.causal_pairs(), "num_heads": H, "num_kv_heads": cfg.num_kv_heads,
+                       "head_size": d, "block_size": cfg.block_size,
+                       "l2": f"inputs larger than L2: {(w.query.numel() * 2 * 2 + key_cache.numel() * 4) / 1e9:.2f} GB "
+                             "of query, output and K/V per step vs 126 MB L2",
+                       "parallelism": f"dp{world} (independent batches)"},
+            "tokens_per_s": round(reduce_sum(float(T), world, dev) / (max_ms * 1e-3), 1),
+            "roofline": {"kernel": "paged_prefill_kernel (pa_paged_prefill call)", "bound": "tensor",
+                         "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4),
+                         "peak_source": "measured bf16 burst" if peaks else "fallback",
+                         "flops_per_launch": flops, "avg_launch_ms": round(attn_ms, 4), "traffic": None},
+            "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+            "gpu_launches": 2 * args.steps, "clocks": clocks.summary()}
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = prefill_cpu_baseline(cfg, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def _prefill_sample(cfg, rows_wanted):
+    """Sampled query rows of the prefill workload as one-token chunks over truncated contexts (the
+    oracle's cost per row is its prefix length), with their FLOPs."""
+    import dataclasses
+    w = W.make_prefill_workload(cfg, num_seqs=min(cfg.num_seqs, 2))
+    rng = np.random.default_rng(cfg.seed)
+    q_start = w.q_start.numpy()
+    lens = w.context_lens.numpy()
+    rows = np.sort(rng.choice(w.query.shape[0], size=min(rows_wanted, w.query.shape[0]), replace=False))
+    seq = np.searchsorted(q_start, rows, side="right") - 1
+    n = q_start[seq + 1] - q_start[seq]
+    pos = lens[seq] - n + (rows - q_start[seq])
+    kc, vc = bits16(w.key_values), bits16(w.value_values)
+    import oracle
+    oracle.reshape_and_cache(bits16(w.new_key), bits16(w.new_value), cfg.dtype, kc, vc, cfg.dtype,
+                             w.slot_mapping.numpy())
+    inp = dict(query_bits=bits16(w.query)[rows], q_dtype=cfg.dtype, key_cache=kc, value_cache=vc,
+               kv_dtype=cfg.dtype, block_tables=w.block_tables.numpy()[seq], context_lens=(pos + 1).astype(np.int32),
+               q_start=np.arange(len(rows) + 1, dtype=np.int32), scale=cfg.softmax_scale)
+    flops = 4.0 * cfg.head_size * cfg.num_heads * float((pos + 1).sum())
+    return inp, flops, len(rows)
+
+
+def prefill_cpu_baseline(cfg, seconds):
+    import oracle
+    rows = 4
+    while True:
+        inp, flops, n = _prefill_sample(cfg, rows)
+        t0 = time.perf_counter()
+        oracle.paged_prefill(**inp)
+        dt = time.perf_counter() - t0
+        if dt >= seconds / 3 or rows >= 4096:
+            break
+        rows = min(4096, max(rows * 2, int(rows * seconds / 3 / max(dt, 1e-3))))
+    reps, total = 0, 0.0
+    while total < seconds * 2 / 3 or reps == 0:
+        t0 = time.perf_counter()
+        oracle.paged_prefill(**inp)
+        total += time.perf_counter() - t0
+        reps += 1
+    t = total / reps
+    return {"value": round(flops / t / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.default_threads(),
+            "kind": "oracle", "sample": f"{n} random query rows of the workload's first sequences, each over its "
+                                        f"whole prefix, {reps} timed passes of {t:.2f} s, fp64"}
+
+
+def run_prefill_reference(args, cfg, world, rank):
+    """The oracle's prefill on a bounded sample, timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+    rows = 4
+    while True:
+        inp, flops, n = _prefill_sample(cfg, rows)
+        t0 = time.perf_counter()
+        oracle.paged_prefill(**inp)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 or rows >= 4096:
+            break
+        rows = min(4096, max(rows * 2, int(rows * 1.0 / max(dt, 1e-3))))
+    for _ in range(args.warmup):
+        oracle.paged_prefill(**inp)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.paged_prefill(**inp)
+        times.append(time.perf_counter() - t0)
+    t = float(np.mean(times))
+    value = flops / t / 1e12
+    sample = f"{n} random query rows of the workload, each over its whole prefix, fp64 oracle"
+    line = {"metric": "paged prefill attention: causal TFLOP/s", "value": round(value, 6), "unit": "TFLOP/s",
+            "impl": "reference", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t * 1e3, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "config": {"workload": cfg.description, "name": cfg.name},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.default_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
 
 
 def run_swap(args, cfg, num_blocks=1024):
