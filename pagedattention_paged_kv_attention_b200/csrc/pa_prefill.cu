@@ -91,7 +91,7 @@ extern "C" pa_status pa_paged_prefill(void* out, const void* query, pa_dtype q_d
     return PA_ERR_UNSUPPORTED;
   if (group > pa::pf::kRows || pa::pf::kRows % group != 0) return PA_ERR_UNSUPPORTED;
   const int tile_tokens = pa::pf::kRows / group;
-  const int q_tiles = ceil_div(max_q_len, tile_tokens);
+  const int q_pairs = ceil_div(max_q_len, tile_tokens * pa::pf::kTiles);
   if (num_seqs > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
 
   CUtensorMap tq, tk, tv;
@@ -114,9 +114,9 @@ extern "C" pa_status pa_paged_prefill(void* out, const void* query, pa_dtype q_d
   a.tile_tokens = tile_tokens;
   a.block_size = block_size;
   a.num_blocks = num_blocks;
-  a.num_q_tiles = q_tiles;
+  a.num_pairs = q_pairs;
   a.scale_log2 = scale * kLog2e;
-  const dim3 grid(static_cast<unsigned>(q_tiles), static_cast<unsigned>(num_kv_heads),
+  const dim3 grid(static_cast<unsigned>(q_pairs), static_cast<unsigned>(num_kv_heads),
                   static_cast<unsigned>(num_seqs));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;

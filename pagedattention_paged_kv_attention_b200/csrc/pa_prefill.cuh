@@ -7,16 +7,20 @@
 // section "PagedAttention：把显存做成虚拟内存"; softmax(QK^T * scale) V from the tutorial page
 // "企业官网建设流程全解析", sec. 2.2; the block table indirection from sec. 2.1).
 //
-// One CTA per (128-row query tile, kv head, sequence). A tile's 128 rows are 128/G query tokens x the
-// G query heads that share the kv head, so grouped heads reuse every K/V tile. Per 128-token KV tile:
-//   warp 0      TMA: the query tile once; K and V boxes of one block x one kv head x 64 columns,
-//               straight from the paged cache through the block table, into a 2-stage ring;
-//   warp 1      one thread issues S = Q K^T (M 128, N 128) into TMEM, then O_tile = P V (M 128, N d)
-//               into TMEM, and commits each to an mbarrier; the warp owns the TMEM allocation;
-//   warps 4..7  thread r owns row r (TMEM lane r): reads its S row, applies the causal mask, keeps the
-//               online-softmax max/sum in fp32, writes P (16-bit, 128-byte swizzled K-major) to shared
-//               memory for the PV MMA, and accumulates O_tile into fp32 registers with the rescale;
-//               at the end it normalises and stores the row.
+// One CTA per (pair of 128-row query tiles A and B, kv head, sequence). A tile's 128 rows are 128/G
+// query tokens x the G query heads that share the kv head, so grouped heads reuse every K/V tile, and
+// the two tiles share the K/V stream. Per 128-key tile j:
+//   warp 0        TMA: both query tiles once; K and V boxes of one block x one kv head x 64 columns,
+//                 straight from the paged cache through the block table, into a 2-stage ring;
+//   warp 1        one thread issues, per tile X, S_X = Q_X K^T (M 128, N 128) into TMEM and
+//                 O_X += P_X V (M 128, N d) with P read from TMEM, in the order
+//                 S_A(0) S_B(0) | PV_A(j) S_A(j+1) PV_B(j) S_B(j+1) | ..., so that each softmax
+//                 warpgroup works on its S while the tensor cores run the other tile's pair;
+//   warps 4..7    softmax of tile A, warps 8..11 of tile B: thread r owns row r (TMEM lane r); it reads
+//                 its S row, applies the causal mask, computes P = exp2(S * scale * log2e - m) against
+//                 a running max m that is raised only when a row's maximum exceeds it by more than 8
+//                 (then O and the sum are rescaled in place), and writes P (16-bit pairs) over S for the
+//                 PV MMA; at the end it normalises O and stores the row.
 // Every wait is bounded; a timed-out wait records PA_DEVERR_TIMEOUT and the CTA winds down (waiting,
 // bounded, for its own copies and MMAs) before it frees TMEM.
 #pragma once
@@ -30,13 +34,15 @@
 namespace pa {
 namespace pf {
 
-constexpr int kRows = 128;      // query rows per CTA (M of both MMAs)
+constexpr int kRows = 128;      // query rows per tile (M of both MMAs)
+constexpr int kTiles = 2;       // query tiles per CTA
 constexpr int kKvTile = 128;    // keys per KV tile (N of QK^T, K of PV)
 constexpr int kStages = 2;      // K/V ring depth
-constexpr int kThreads = 256;   // warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-7 softmax
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kTmemS = 0;    // S: columns [0, 128)
-constexpr uint32_t kTmemO = 128;  // O tile: columns [128, 128 + d)
+constexpr int kThreads = 384;   // warp 0 TMA, warp 1 MMA, warps 2-3 idle, warps 4-7 / 8-11 softmax
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemTile = 256;  // per query tile: S (and P over it) in [0, 128), O in [128, 128 + d)
+constexpr uint32_t kTmemO = 128;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8 between rescales
 
 struct PrefillArgs {
   void* out;                    // [T][H][d]
@@ -45,7 +51,7 @@ struct PrefillArgs {
   const int32_t* q_start;       // [S + 1]
   unsigned int* error_word;
   int max_blocks_per_seq, num_seqs, num_q_tokens, num_heads, num_kv_heads, group, tile_tokens, block_size,
-      num_blocks, num_q_tiles;
+      num_blocks, num_pairs;
   float scale_log2;             // scale * log2(e)
 };
 
@@ -53,18 +59,20 @@ template <int D>
 struct Layout {
   static constexpr int kChunks = D / 64;                        // 128-byte column chunks of a d row
   static constexpr uint32_t kTileChunk = kRows * 128;           // one chunk of a 128-row tile
-  static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kP = kQ + kChunks * kTileChunk;     // P: 128 rows x 128 keys = 2 chunks
-  static constexpr uint32_t kKV = kP + 2 * kTileChunk;
+  static constexpr uint32_t kQ = 0;                             // tile X at kQ + X * kQTile
+  static constexpr uint32_t kQTile = kChunks * kTileChunk;
+  static constexpr uint32_t kKV = kQ + kTiles * kQTile;
   static constexpr uint32_t kK = 0;                             // inside a stage
   static constexpr uint32_t kV = kChunks * kKvTile * 128;
   static constexpr uint32_t kStage = 2 * kChunks * kKvTile * 128;
   static constexpr uint32_t kBars = kKV + kStages * kStage;
-  static constexpr uint32_t kBytes = kBars + 256 + 1024;        // barriers and flags, alignment slack
+  // Barriers and flags, alignment slack; at least 120 KB so that one CTA holds an SM (and with it
+  // all 512 TMEM columns: a second CTA's allocation would wait for the first to finish).
+  static constexpr uint32_t kBytes = (kBars + 256 + 1024) > 120u * 1024 ? (kBars + 256 + 1024) : 120u * 1024;
 };
 
 struct Bars {
-  uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full, p_full, o_full, o_empty, mma_done;
+  uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[kTiles], p_full[kTiles], o_final[kTiles], mma_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -121,24 +129,24 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* b = reinterpret_cast<Bars*>(sm + L::kBars);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q_tile = a.num_q_tiles - 1 - static_cast<int>(blockIdx.x);  // longest prefixes first
+  const int pair = a.num_pairs - 1 - static_cast<int>(blockIdx.x);  // longest prefixes first
   const int kvh = blockIdx.y, s = blockIdx.z;
   const int G = a.group;
 
-  // ---- the tile's extent; every condition below is uniform over the CTA ----
+  // ---- the tiles' extent; every condition below is uniform over the CTA ----
   const int q0 = a.q_start[s];
   const int n = a.q_start[s + 1] - q0;
   const int ctx = a.context_lens[s];
-  const int tok0 = q_tile * a.tile_tokens;
+  const int tok0 = pair * kTiles * a.tile_tokens;  // first token of tile A; tile B follows
   if (n <= 0 || tok0 >= n || q0 < 0) {
-    if (q_tile == 0 && threadIdx.x == 0 && (n < 0 || q0 < 0)) atomicOr(a.error_word, PA_DEVERR_CONTEXT_LEN);
+    if (pair == 0 && threadIdx.x == 0 && (n < 0 || q0 < 0)) atomicOr(a.error_word, PA_DEVERR_CONTEXT_LEN);
     return;
   }
   if (n > ctx || q0 + n > a.num_q_tokens ||
       static_cast<long long>(ctx) > static_cast<long long>(a.max_blocks_per_seq) * a.block_size) {
     // A chunk must lie inside its context and inside the query array: flag it, NaN the rows.
     if (threadIdx.x == 0) atomicOr(a.error_word, PA_DEVERR_CONTEXT_LEN);
-    if (threadIdx.x < kRows && q0 + n <= a.num_q_tokens) {
+    if (threadIdx.x < kTiles * kRows && q0 + n <= a.num_q_tokens) {
       const int tok = tok0 + static_cast<int>(threadIdx.x) / G;
       if (tok < n) {
         T* o = static_cast<T*>(a.out) +
@@ -149,8 +157,21 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
     }
     return;
   }
-  const int p_max = ctx - n + min(n, tok0 + a.tile_tokens) - 1;  // last key any row of the tile needs
-  const int nkv = p_max / kKvTile + 1;
+  // Per tile: first token, KV tiles needed (0 when the tile lies past the chunk).
+  int tile_tok0[kTiles], nkv_t[kTiles];
+  int p_max = 0;
+#pragma unroll
+  for (int x = 0; x < kTiles; ++x) {
+    tile_tok0[x] = tok0 + x * a.tile_tokens;
+    if (tile_tok0[x] < n) {
+      const int pm = ctx - n + min(n, tile_tok0[x] + a.tile_tokens) - 1;  // last key the tile needs
+      nkv_t[x] = pm / kKvTile + 1;
+      p_max = max(p_max, pm);
+    } else {
+      nkv_t[x] = 0;
+    }
+  }
+  const int nkv = p_max / kKvTile + 1;  // = nkv_t of the last active tile
 
   // ---- set-up: barriers (thread 0), TMEM (warp 1) ----
   if (threadIdx.x == 0) {
@@ -159,10 +180,11 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
       mbar_init(&b->kv_full[i], 1);
       mbar_init(&b->kv_empty[i], 1);
     }
-    mbar_init(&b->s_full, 1);
-    mbar_init(&b->p_full, kRows);
-    mbar_init(&b->o_full, 1);
-    mbar_init(&b->o_empty, kRows);
+    for (int x = 0; x < kTiles; ++x) {
+      mbar_init(&b->s_full[x], 1);
+      mbar_init(&b->p_full[x], kRows);
+      mbar_init(&b->o_final[x], 1);
+    }
     mbar_init(&b->mma_done, 1);
     b->abort = 0;
     fence_mbar_init();
@@ -183,9 +205,12 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
     const int bs = a.block_size;
     const int32_t* table = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
     if (lane == 0) {
-      mbar_arrive_expect_tx(&b->q_full, L::kChunks * L::kTileChunk);
-      for (int c = 0; c < L::kChunks; ++c)
-        tma_load_3d(sm + L::kQ + c * L::kTileChunk, &tq, &b->q_full, c * 64, kvh * G, q0 + tok0);
+      const int tiles = (nkv_t[1] > 0) ? 2 : 1;
+      mbar_arrive_expect_tx(&b->q_full, tiles * L::kQTile);
+      for (int x = 0; x < tiles; ++x)
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(sm + L::kQ + x * L::kQTile + c * L::kTileChunk, &tq, &b->q_full, c * 64, kvh * G,
+                      q0 + tile_tok0[x]);
     }
     for (int j = 0; j < nkv; ++j) {
       const int stage = j % kStages;
@@ -218,137 +243,173 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
       if (issued[i] > 0) mbar_wait(&b->kv_full[i], (issued[i] - 1) & 1, err);
   } else if (warp == 1) {
     // ================================ MMA issuer ================================
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = mma_idesc_f16<T>(kRows, kKvTile, false);
-      constexpr uint32_t idesc_o = mma_idesc_f16<T>(kRows, D, true);
-      const uint32_t q_addr = smem_u32(sm + L::kQ), p_addr = smem_u32(sm + L::kP);
-      bool ok = wait_or_abort(b, &b->q_full, 0, err);
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int stage = j % kStages;
-        const uint32_t k_addr = smem_u32(sm + L::kKV + stage * L::kStage + L::kK);
-        const uint32_t v_addr = smem_u32(sm + L::kKV + stage * L::kStage + L::kV);
-        if (!(ok = wait_or_abort(b, &b->kv_full[stage], (j / kStages) & 1, err))) break;
-        tc_fence_after();
+    constexpr uint32_t idesc_s = mma_idesc_f16<T>(kRows, kKvTile, false);
+    constexpr uint32_t idesc_o = mma_idesc_f16<T>(kRows, D, true);
+    auto kv_addr = [&](int j, uint32_t part) { return smem_u32(sm + L::kKV + (j % kStages) * L::kStage + part); };
+    auto issue_s = [&](int x, int j) {  // S_x = Q_x K_j^T over d in steps of 16
+      const uint32_t q_addr = smem_u32(sm + L::kQ + x * L::kQTile), k_addr = kv_addr(j, L::kK);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {  // S = Q K^T over d in steps of 16
-          const uint32_t qo = (k >> 2) * L::kTileChunk + (k & 3) * 32;
-          const uint32_t ko = (k >> 2) * (kKvTile * 128) + (k & 3) * 32;
-          mma_f16_ss(tmem + kTmemS, smem_desc_sw128(q_addr + qo, 16, 1024), smem_desc_sw128(k_addr + ko, 16, 1024),
-                     idesc_s, k > 0);
-        }
-        mma_commit(&b->s_full);
-        if (!(ok = wait_or_abort(b, &b->p_full, j & 1, err))) break;
-        if (j > 0 && !(ok = wait_or_abort(b, &b->o_empty, (j - 1) & 1, err))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < kKvTile / 16; ++k) {  // O_tile = P V over keys in steps of 16
-          const uint32_t po = (k >> 2) * L::kTileChunk + (k & 3) * 32;
-          const uint32_t vo = k * 16 * 128;
-          mma_f16_ss(tmem + kTmemO, smem_desc_sw128(p_addr + po, 16, 1024),
-                     smem_desc_sw128(v_addr + vo, kKvTile * 128, 1024), idesc_o, k > 0);
-        }
-        mma_commit(&b->o_full);
-        mma_commit(&b->kv_empty[stage]);
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t qo = (k >> 2) * L::kTileChunk + (k & 3) * 32;
+        const uint32_t ko = (k >> 2) * (kKvTile * 128) + (k & 3) * 32;
+        mma_f16_ss(tmem + x * kTmemTile, smem_desc_sw128(q_addr + qo, 16, 1024),
+                   smem_desc_sw128(k_addr + ko, 16, 1024), idesc_s, k > 0);
       }
-      // Wind-down: every MMA issued above has completed before TMEM can be freed.
+      mma_commit(&b->s_full[x]);
+    };
+    auto issue_pv = [&](int x, int j) {  // O_x += P_x V_j over keys in steps of 16, P from TMEM
+      const uint32_t v_addr = kv_addr(j, L::kV);
+#pragma unroll
+      for (int k = 0; k < kKvTile / 16; ++k)
+        mma_f16_ts(tmem + x * kTmemTile + kTmemO, tmem + x * kTmemTile + 8 * k,
+                   smem_desc_sw128(v_addr + k * 16 * 128, kKvTile * 128, 1024), idesc_o, (j > 0 || k > 0) ? 1u : 0u);
+    };
+    bool ok = warp_wait_or_abort(b, &b->q_full, 0, err) && warp_wait_or_abort(b, &b->kv_full[0], 0, err);
+    if (ok) {
+      tc_fence_after();
+      if (lane == 0)
+        for (int x = 0; x < kTiles; ++x)
+          if (nkv_t[x] > 0) issue_s(x, 0);
+      __syncwarp();
+    }
+    for (int j = 0; ok && j < nkv; ++j) {
+      if (j + 1 < nkv && !(ok = warp_wait_or_abort(b, &b->kv_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, err)))
+        break;
+      if (j == nkv - 1) {
+        // Keys past the last one any row needs (not loaded, or past the context) must not reach PV
+        // as stale or NaN values: zero those V rows of the last tile before its PV MMAs.
+        const int cut = p_max + 1 - j * kKvTile;
+        if (cut < kKvTile) {
+          uint8_t* vb = sm + L::kKV + (j % kStages) * L::kStage + L::kV;
+          const int units = (kKvTile - cut) * 8;
+          for (int c = 0; c < L::kChunks; ++c)
+            for (int u = lane; u < units; u += 32)
+              *reinterpret_cast<uint4*>(vb + c * (kKvTile * 128) + cut * 128 + u * 16) = make_uint4(0, 0, 0, 0);
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+      }
+      for (int x = 0; x < kTiles; ++x) {
+        if (j >= nkv_t[x]) continue;
+        if (!(ok = warp_wait_or_abort(b, &b->p_full[x], j & 1, err))) break;
+        tc_fence_after();
+        if (lane == 0) {
+          issue_pv(x, j);
+          if (j + 1 < nkv_t[x])
+            issue_s(x, j + 1);
+          else
+            mma_commit(&b->o_final[x]);
+        }
+        __syncwarp();
+      }
+      if (lane == 0) mma_commit(&b->kv_empty[j % kStages]);
+      __syncwarp();
+    }
+    // Wind-down: every MMA issued above has completed before TMEM can be freed.
+    if (lane == 0) {
       mma_commit(&b->mma_done);
       mbar_wait(&b->mma_done, 0, err);
     }
     __syncwarp();
   } else if (warp >= 4) {
     // ================================ softmax / epilogue ================================
-    const int r = threadIdx.x - 128;                // row == TMEM lane
-    const int tok = tok0 + r / G;
-    const bool row_valid = tok < n;
-    const int pos = ctx - n + min(tok, n - 1);      // rows past the chunk reuse its last position
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(r & ~31) << 16);
-    const float sl2 = a.scale_log2;
-    float o[D];
-#pragma unroll
-    for (int i = 0; i < D; ++i) o[i] = 0.f;
-    float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      if (!(ok = warp_wait_or_abort(b, &b->s_full, j & 1, err))) break;
-      tc_fence_after();
-      const int base = j * kKvTile;
-      // Pass 1: the row maximum over the keys this row may see.
-      float mx = -INFINITY;
+    const int x = (warp - 4) >> 2;                  // query tile of this warpgroup
+    const int r = threadIdx.x - 128 - x * kRows;    // row == TMEM lane
+    const int nkv_x = nkv_t[x];
+    if (nkv_x > 0) {
+      const int tok = tile_tok0[x] + r / G;
+      const bool row_valid = tok < n;
+      const int pos = ctx - n + min(tok, n - 1);    // rows past the chunk reuse its last position
+      const uint32_t t_s = tmem + x * kTmemTile + (static_cast<uint32_t>(r & ~31) << 16);
+      const uint32_t t_o = t_s + kTmemO;
+      const float sl2 = a.scale_log2;
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nkv_x; ++j) {
+        if (!(ok = warp_wait_or_abort(b, &b->s_full[x], j & 1, err))) break;
+        tc_fence_after();
+        const int base = j * kKvTile;
+        // Pass 1: the row maximum over the keys this row may see.
+        float mx = -INFINITY;
 #pragma unroll 1
-      for (int c = 0; c < kKvTile / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(t_lane + kTmemS + 32 * c, v);
-        tmem_wait_ld(v);
+        for (int c = 0; c < kKvTile / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(t_s + 32 * c, v);
+          tmem_wait_ld(v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (base + 32 * c + i <= pos) mx = fmaxf(mx, __uint_as_float(v[i]));
-      }
-      const float m_new = fmaxf(m, mx * sl2);
-      const float alpha = ex2(m - m_new);           // 0 on the first tile (m = -inf)
-      // The last tile holds keys past the tile's last needed key (unloaded or past the context):
-      // zero those V rows so that 0 * (stale or NaN) cannot reach the PV product.
-      if (j == nkv - 1) {
-        const int cut = p_max + 1 - base;
-        if (cut < kKvTile) {
-          const int stage = j % kStages;
-          if (!(ok = warp_wait_or_abort(b, &b->kv_full[stage], (j / kStages) & 1, err))) break;
-          uint8_t* vb = sm + L::kKV + stage * L::kStage + L::kV;
-          const int units = (kKvTile - cut) * 8;
-          for (int c = 0; c < L::kChunks; ++c)
-            for (int u = r; u < units; u += kRows)
-              *reinterpret_cast<uint4*>(vb + c * (kKvTile * 128) + cut * 128 + u * 16) = make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < 32; ++i)
+            if (base + 32 * c + i <= pos) mx = fmaxf(mx, __uint_as_float(v[i]));
         }
-      }
-      // Pass 2: P = exp2(S * scale * log2e - m), rounded to 16 bits; the sum uses the rounded values.
-      float lsum = 0.f;
+        const float m_cand = mx * sl2;
+        if (j == 0) {
+          m = m_cand;                               // O is written fresh by the first PV
+        } else {
+          // S_x(j) was issued after PV_x(j-1), so O holds every earlier tile and may be rescaled.
+          const bool raise = m_cand > m + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, raise)) {
+            const float alpha = raise ? ex2(m - m_cand) : 1.f;
 #pragma unroll 1
-      for (int c = 0; c < kKvTile / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(t_lane + kTmemS + 32 * c, v);
-        tmem_wait_ld(v);
-        uint32_t w[16];
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t v[32];
+              tmem_ld32(t_o + 32 * c, v);
+              tmem_wait_ld(v);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int t = base + 32 * c + 2 * i;
-          const float p0 = (t <= pos) ? ex2(fmaf(__uint_as_float(v[2 * i]), sl2, -m_new)) : 0.f;
-          const float p1 = (t + 1 <= pos) ? ex2(fmaf(__uint_as_float(v[2 * i + 1]), sl2, -m_new)) : 0.f;
-          w[i] = pack_pair<T>(p0, p1);
-          const float2 back = unpack_pair<T>(w[i]);
-          lsum += back.x + back.y;
+              for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+              tmem_st32(t_o + 32 * c, v);
+            }
+            tmem_wait_st();
+            if (raise) {
+              l *= alpha;
+              m = m_cand;
+            }
+          }
         }
-        uint8_t* prow = sm + L::kP + (c >> 1) * L::kTileChunk + r * 128;
+        // Pass 2: P = exp2(S * scale * log2e - m), rounded to 16 bits and written over S; the sum
+        // uses the rounded values.
+        float lsum = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < kKvTile / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(t_s + 32 * c, v);
+          tmem_wait_ld(v);
+          uint32_t w[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int unit = ((c & 1) * 4 + q) ^ (r & 7);
-          *reinterpret_cast<uint4*>(prow + unit * 16) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          for (int i = 0; i < 16; ++i) {
+            const int t = base + 32 * c + 2 * i;
+            const float p0 = (t <= pos) ? ex2(fmaf(__uint_as_float(v[2 * i]), sl2, -m)) : 0.f;
+            const float p1 = (t + 1 <= pos) ? ex2(fmaf(__uint_as_float(v[2 * i + 1]), sl2, -m)) : 0.f;
+            w[i] = pack_pair<T>(p0, p1);
+            const float2 back = unpack_pair<T>(w[i]);
+            lsum += back.x + back.y;
+          }
+          tmem_st16(t_s + 16 * c, w);               // columns already read (16c < 32c + 32)
+        }
+        l += lsum;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&b->p_full[x]);
+      }
+      if (ok) ok = warp_wait_or_abort(b, &b->o_final[x], 0, err);
+      if (ok) {
+        tc_fence_after();
+        const float inv = 1.f / l;
+        T* dst = static_cast<T*>(a.out) + (static_cast<size_t>(q0 + min(tok, n - 1)) * a.num_heads + kvh * G + r % G) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(t_o + 32 * c, v);
+          tmem_wait_ld(v);
+          if (row_valid) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8)
+              *reinterpret_cast<uint4*>(dst + 32 * c + i) = make_uint4(
+                  pack_pair<T>(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv),
+                  pack_pair<T>(__uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv),
+                  pack_pair<T>(__uint_as_float(v[i + 4]) * inv, __uint_as_float(v[i + 5]) * inv),
+                  pack_pair<T>(__uint_as_float(v[i + 6]) * inv, __uint_as_float(v[i + 7]) * inv));
+          }
         }
       }
-      l = l * alpha + lsum;
-      m = m_new;
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&b->p_full);
-      if (!(ok = warp_wait_or_abort(b, &b->o_full, j & 1, err))) break;
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(t_lane + kTmemO + 32 * c, v);
-        tmem_wait_ld(v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[32 * c + i] = fmaf(o[32 * c + i], alpha, __uint_as_float(v[i]));
-      }
-      tc_fence_before();
-      mbar_arrive(&b->o_empty);
-    }
-    if (ok && row_valid) {
-      const float inv = 1.f / l;
-      T* dst = static_cast<T*>(a.out) + (static_cast<size_t>(q0 + tok) * a.num_heads + kvh * G + r % G) * D;
-#pragma unroll
-      for (int i = 0; i < D; i += 8)
-        *reinterpret_cast<uint4*>(dst + i) =
-            make_uint4(pack_pair<T>(o[i] * inv, o[i + 1] * inv), pack_pair<T>(o[i + 2] * inv, o[i + 3] * inv),
-                       pack_pair<T>(o[i + 4] * inv, o[i + 5] * inv), pack_pair<T>(o[i + 6] * inv, o[i + 7] * inv));
     }
   }
 
