@@ -182,8 +182,8 @@ PA_API pa_status pa_paged_attention_static(void* out, const void* query, pa_dtyp
  *  max_q_len      >= max_s n_s (sizes the grid; tiles past a sequence's chunk exit at once).
  *  workspace      >= PA_WORKSPACE_HEADER_BYTES, zeroed once; its first word is the device error word
  *                 (read with pa_get_device_error).
- * Supported: head_size 64 or 128; block_size 8, 16, 32, 64 or 128; num_heads / num_kv_heads dividing
- * 128. A chunk outside its context (n_s > L_s, or L_s beyond the block table) sets
+ * scale must be positive and finite. Supported: head_size 64 or 128; block_size 8, 16, 32, 64 or 128;
+ * num_heads / num_kv_heads dividing 128. A chunk outside its context (n_s > L_s, or L_s beyond the block table) sets
  * PA_DEVERR_CONTEXT_LEN and NaNs its rows; a block id outside the pool sets PA_DEVERR_BLOCK_ID.
  */
 PA_API pa_status pa_paged_prefill(void* out, const void* query, pa_dtype q_dtype, const void* key_cache,

@@ -74,7 +74,7 @@ extern "C" pa_status pa_paged_prefill(void* out, const void* query, pa_dtype q_d
                                       void* workspace, size_t workspace_bytes, pa_stream_t stream) {
   if (num_seqs < 0 || num_q_tokens < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
       head_size <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_q_len < 0 ||
-      !std::isfinite(scale))
+      !std::isfinite(scale) || !(scale > 0.f))
     return PA_ERR_INVALID_ARGUMENT;
   if (!is_dtype(q_dtype) || !is_dtype(kv_dtype) || !is_16bit(q_dtype)) return PA_ERR_INVALID_ARGUMENT;
   if (num_seqs == 0 || num_q_tokens == 0 || max_q_len == 0) return PA_OK;  // nothing to compute

@@ -43,6 +43,12 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemTile = 256;  // per query tile: S (and P over it) in [0, 128), O in [128, 128 + d)
 constexpr uint32_t kTmemO = 128;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8 between rescales
+// Bit i set: in every 32-key chunk of an S row, the pair of keys (2i, 2i+1) has its exponentials
+// computed on the FMA pipe (ex2_fma2) instead of MUFU.
+#ifndef PA_PREFILL_POLY_MASK
+#define PA_PREFILL_POLY_MASK 0x0000
+#endif
+constexpr unsigned kPolyMask = PA_PREFILL_POLY_MASK;
 
 struct PrefillArgs {
   void* out;                    // [T][H][d]
@@ -72,15 +78,43 @@ struct Layout {
 };
 
 struct Bars {
-  uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[kTiles], p_full[kTiles], o_final[kTiles], mma_done;
+  uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages], s_full[kTiles],
+      p_full[kTiles], o_final[kTiles], mma_done;
   uint32_t tmem_base;
   int abort;
 };
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x for a pair of values on the FMA/ALU pipes (packed f32x2 arithmetic), so that the MUFU unit is
+// not the only one computing the softmax exponentials. Range reduction x = n + f with n = round(x)
+// (adding and subtracting 1.5 * 2^23 rounds to an integer held in the low mantissa bits) and f in
+// [-1/2, 1/2]; 2^f by a cubic whose coefficients were fitted here to minimise the relative error on
+// that interval (max 7.5e-5, below the 16-bit rounding of P); n is added to the exponent field. x is
+// clamped at -126 so that the result stays a non-negative float (a masked score, -inf, gives about
+// 1e-38 instead of 0).
+__device__ __forceinline__ float2 ex2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 r = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(r, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(0.05517113208770752f, 0.05517113208770752f), f,
+                        make_float2(0.24261008203029633f, 0.24261008203029633f));
+  p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+  p = __ffma2_rn(p, f, make_float2(0.9999281167984009f, 0.9999281167984009f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 // A bounded wait that gives up at once after any role of the CTA has given up.
@@ -177,8 +211,10 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
   if (threadIdx.x == 0) {
     mbar_init(&b->q_full, 1);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&b->kv_full[i], 1);
-      mbar_init(&b->kv_empty[i], 1);
+      mbar_init(&b->k_full[i], 1);
+      mbar_init(&b->k_empty[i], 1);
+      mbar_init(&b->v_full[i], 1);
+      mbar_init(&b->v_empty[i], 1);
     }
     for (int x = 0; x < kTiles; ++x) {
       mbar_init(&b->s_full[x], 1);
@@ -198,10 +234,9 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = b->tmem_base;
   unsigned int* err = a.error_word;
-
   if (warp == 0) {
     // ================================ TMA producer ================================
-    int issued[kStages] = {0, 0};
+    int issued[2 * kStages] = {0, 0, 0, 0};
     const int bs = a.block_size;
     const int32_t* table = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
     if (lane == 0) {
@@ -212,9 +247,10 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
           tma_load_3d(sm + L::kQ + x * L::kQTile + c * L::kTileChunk, &tq, &b->q_full, c * 64, kvh * G,
                       q0 + tile_tok0[x]);
     }
+    // K and V of a tile go to separate rings: a K slot is freed once both query tiles' S MMAs have
+    // read it, long before the PV MMAs release the V slot, so the next K arrives early.
     for (int j = 0; j < nkv; ++j) {
       const int stage = j % kStages;
-      if (j >= kStages && !warp_wait_or_abort(b, &b->kv_empty[stage], ((j / kStages) - 1) & 1, err)) break;
       const int first = j * kKvTile;
       const int ntok = min(kKvTile, p_max + 1 - first);
       const int nblk = (ntok + bs - 1) / bs;
@@ -226,21 +262,32 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
         if (!ok) atomicOr(err, PA_DEVERR_BLOCK_ID);
       }
       const unsigned okmask = __ballot_sync(0xffffffffu, ok);
+      const uint32_t bytes = __popc(okmask) * bs * 128 * L::kChunks;
       uint8_t* st = sm + L::kKV + stage * L::kStage;
-      if (lane == 0) mbar_arrive_expect_tx(&b->kv_full[stage], __popc(okmask) * bs * 128 * L::kChunks * 2);
-      __syncwarp();
-      if (ok) {
-        for (int c = 0; c < L::kChunks; ++c) {
-          const uint32_t off = c * (kKvTile * 128) + lane * bs * 128;
-          tma_load_4d(st + L::kK + off, &tk, &b->kv_full[stage], c * 64, 0, kvh, blk);
-          tma_load_4d(st + L::kV + off, &tv, &b->kv_full[stage], c * 64, 0, kvh, blk);
+      bool go = true;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {  // 0: K, 1: V
+        uint64_t* full = part == 0 ? &b->k_full[stage] : &b->v_full[stage];
+        uint64_t* empty = part == 0 ? &b->k_empty[stage] : &b->v_empty[stage];
+        if (j >= kStages && !warp_wait_or_abort(b, empty, ((j / kStages) - 1) & 1, err)) {
+          go = false;
+          break;
         }
+        if (lane == 0) mbar_arrive_expect_tx(full, bytes);
+        __syncwarp();
+        if (ok)
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_4d(st + (part == 0 ? L::kK : L::kV) + c * (kKvTile * 128) + lane * bs * 128,
+                        part == 0 ? &tk : &tv, full, c * 64, 0, kvh, blk);
+        ++issued[part * kStages + stage];
       }
-      ++issued[stage];
+      if (!go) break;
     }
-    // Wind-down: the last load issued into each stage has landed (immediate unless the CTA aborted).
-    for (int i = 0; i < kStages; ++i)
-      if (issued[i] > 0) mbar_wait(&b->kv_full[i], (issued[i] - 1) & 1, err);
+    // Wind-down: the last load issued into each slot has landed (immediate unless the CTA aborted).
+    for (int part = 0; part < 2; ++part)
+      for (int i = 0; i < kStages; ++i)
+        if (issued[part * kStages + i] > 0)
+          mbar_wait(part == 0 ? &b->k_full[i] : &b->v_full[i], (issued[part * kStages + i] - 1) & 1, err);
   } else if (warp == 1) {
     // ================================ MMA issuer ================================
     constexpr uint32_t idesc_s = mma_idesc_f16<T>(kRows, kKvTile, false);
@@ -264,17 +311,18 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
         mma_f16_ts(tmem + x * kTmemTile + kTmemO, tmem + x * kTmemTile + 8 * k,
                    smem_desc_sw128(v_addr + k * 16 * 128, kKvTile * 128, 1024), idesc_o, (j > 0 || k > 0) ? 1u : 0u);
     };
-    bool ok = warp_wait_or_abort(b, &b->q_full, 0, err) && warp_wait_or_abort(b, &b->kv_full[0], 0, err);
+    bool ok = warp_wait_or_abort(b, &b->q_full, 0, err) && warp_wait_or_abort(b, &b->k_full[0], 0, err);
     if (ok) {
       tc_fence_after();
-      if (lane == 0)
+      if (lane == 0) {
         for (int x = 0; x < kTiles; ++x)
           if (nkv_t[x] > 0) issue_s(x, 0);
+        mma_commit(&b->k_empty[0]);
+      }
       __syncwarp();
     }
     for (int j = 0; ok && j < nkv; ++j) {
-      if (j + 1 < nkv && !(ok = warp_wait_or_abort(b, &b->kv_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, err)))
-        break;
+      if (!(ok = warp_wait_or_abort(b, &b->v_full[j % kStages], (j / kStages) & 1, err))) break;
       if (j == nkv - 1) {
         // Keys past the last one any row needs (not loaded, or past the context) must not reach PV
         // as stale or NaN values: zero those V rows of the last tile before its PV MMAs.
@@ -289,20 +337,28 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
         }
         __syncwarp();
       }
+      bool next_k = false;  // K_{j+1} waited for
       for (int x = 0; x < kTiles; ++x) {
         if (j >= nkv_t[x]) continue;
         if (!(ok = warp_wait_or_abort(b, &b->p_full[x], j & 1, err))) break;
         tc_fence_after();
-        if (lane == 0) {
-          issue_pv(x, j);
-          if (j + 1 < nkv_t[x])
-            issue_s(x, j + 1);
-          else
-            mma_commit(&b->o_final[x]);
+        if (lane == 0) issue_pv(x, j);
+        if (j + 1 < nkv_t[x]) {
+          if (!next_k && !(ok = warp_wait_or_abort(b, &b->k_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, err)))
+            break;
+          next_k = true;
+          tc_fence_after();
+          if (lane == 0) issue_s(x, j + 1);
+        } else if (lane == 0) {
+          mma_commit(&b->o_final[x]);
         }
         __syncwarp();
       }
-      if (lane == 0) mma_commit(&b->kv_empty[j % kStages]);
+      if (!ok) break;
+      if (lane == 0) {
+        mma_commit(&b->v_empty[j % kStages]);
+        if (next_k) mma_commit(&b->k_empty[(j + 1) % kStages]);
+      }
       __syncwarp();
     }
     // Wind-down: every MMA issued above has completed before TMEM can be freed.
@@ -320,6 +376,7 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
       const int tok = tile_tok0[x] + r / G;
       const bool row_valid = tok < n;
       const int pos = ctx - n + min(tok, n - 1);    // rows past the chunk reuse its last position
+      const int pos_lane0 = __shfl_sync(0xffffffffu, pos, 0);
       const uint32_t t_s = tmem + x * kTmemTile + (static_cast<uint32_t>(r & ~31) << 16);
       const uint32_t t_o = t_s + kTmemO;
       const float sl2 = a.scale_log2;
@@ -329,18 +386,27 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
         if (!(ok = warp_wait_or_abort(b, &b->s_full[x], j & 1, err))) break;
         tc_fence_after();
         const int base = j * kKvTile;
-        // Pass 1: the row maximum over the keys this row may see.
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < kKvTile / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(t_s + 32 * c, v);
-          tmem_wait_ld(v);
+        // The whole S row at once: four loads in flight, then one wait.
+        uint32_t v[kKvTile / 32][32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (base + 32 * c + i <= pos) mx = fmaxf(mx, __uint_as_float(v[i]));
+        for (int c = 0; c < kKvTile / 32; ++c) tmem_ld32(t_s + 32 * c, v[c]);
+#pragma unroll
+        for (int c = 0; c < kKvTile / 32; ++c) tmem_wait_ld(v[c]);
+        // Causal mask: keys past this row's position become -inf (then exp2 gives 0). Only chunks that
+        // reach past the warp's first row position need it (positions rise with the lane).
+        float mxs[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // independent chains
+#pragma unroll
+        for (int c = 0; c < kKvTile / 32; ++c) {
+          if (base + 32 * c + 31 > pos_lane0) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (base + 32 * c + i > pos) v[c][i] = __float_as_uint(-INFINITY);
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            mxs[(i >> 1) & 3] = fmax3(mxs[(i >> 1) & 3], __uint_as_float(v[c][i]), __uint_as_float(v[c][i + 1]));
         }
-        const float m_cand = mx * sl2;
+        const float m_cand = fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])) * sl2;
         if (j == 0) {
           m = m_cand;                               // O is written fresh by the first PV
         } else {
@@ -349,41 +415,41 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
           if (__any_sync(0xffffffffu, raise)) {
             const float alpha = raise ? ex2(m - m_cand) : 1.f;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t v[32];
-              tmem_ld32(t_o + 32 * c, v);
-              tmem_wait_ld(v);
+            for (int c = 0; c < D / 8; ++c) {      // 8 columns at a time: the S row stays in registers
+              uint32_t o[8];
+              tmem_ld8(t_o + 8 * c, o);
+              tmem_wait_ld8(o);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-              tmem_st32(t_o + 32 * c, v);
+              for (int i = 0; i < 8; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st8(t_o + 8 * c, o);
             }
-            tmem_wait_st();
             if (raise) {
               l *= alpha;
               m = m_cand;
             }
           }
         }
-        // Pass 2: P = exp2(S * scale * log2e - m), rounded to 16 bits and written over S; the sum
-        // uses the rounded values.
-        float lsum = 0.f;
-#pragma unroll 1
+        // P = exp2(S * scale * log2e - m), written over S as 16-bit pairs (columns 16c .. 16c+15 were
+        // read above); the row sum is kept in fp32.
+        float2 ls[4];                               // independent chains
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ls[i] = make_float2(0.f, 0.f);
+        const float2 sl2x2 = make_float2(sl2, sl2), negm = make_float2(-m, -m);
+#pragma unroll
         for (int c = 0; c < kKvTile / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(t_s + 32 * c, v);
-          tmem_wait_ld(v);
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int t = base + 32 * c + 2 * i;
-            const float p0 = (t <= pos) ? ex2(fmaf(__uint_as_float(v[2 * i]), sl2, -m)) : 0.f;
-            const float p1 = (t + 1 <= pos) ? ex2(fmaf(__uint_as_float(v[2 * i + 1]), sl2, -m)) : 0.f;
-            w[i] = pack_pair<T>(p0, p1);
-            const float2 back = unpack_pair<T>(w[i]);
-            lsum += back.x + back.y;
+            const float2 xy = __ffma2_rn(make_float2(__uint_as_float(v[c][2 * i]), __uint_as_float(v[c][2 * i + 1])),
+                                         sl2x2, negm);
+            const float2 p = ((kPolyMask >> i) & 1u) ? ex2_fma2(xy) : make_float2(ex2(xy.x), ex2(xy.y));
+            w[i] = pack_pair<T>(p.x, p.y);
+            ls[i & 3] = __fadd2_rn(ls[i & 3], p);
           }
-          tmem_st16(t_s + 16 * c, w);               // columns already read (16c < 32c + 32)
+          tmem_st16(t_s + 16 * c, w);
         }
+        const float2 l2 = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
+        const float lsum = l2.x + l2.y;
         l += lsum;
         tmem_wait_st();
         tc_fence_before();
