@@ -43,12 +43,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemTile = 256;  // per query tile: S (and P over it) in [0, 128), O in [128, 128 + d)
 constexpr uint32_t kTmemO = 128;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8 between rescales
-// Bit i set: in every 32-key chunk of an S row, the pair of keys (2i, 2i+1) has its exponentials
-// computed on the FMA pipe (ex2_fma2) instead of MUFU.
-#ifndef PA_PREFILL_POLY_MASK
-#define PA_PREFILL_POLY_MASK 0x0000
-#endif
-constexpr unsigned kPolyMask = PA_PREFILL_POLY_MASK;
 
 struct PrefillArgs {
   void* out;                    // [T][H][d]
@@ -94,27 +88,6 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x for a pair of values on the FMA/ALU pipes (packed f32x2 arithmetic), so that the MUFU unit is
-// not the only one computing the softmax exponentials. Range reduction x = n + f with n = round(x)
-// (adding and subtracting 1.5 * 2^23 rounds to an integer held in the low mantissa bits) and f in
-// [-1/2, 1/2]; 2^f by a cubic whose coefficients were fitted here to minimise the relative error on
-// that interval (max 7.5e-5, below the 16-bit rounding of P); n is added to the exponent field. x is
-// clamped at -126 so that the result stays a non-negative float (a masked score, -inf, gives about
-// 1e-38 instead of 0).
-__device__ __forceinline__ float2 ex2_fma2(float2 x) {
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
-  const float2 r = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __ffma2_rn(r, make_float2(-1.f, -1.f), x);
-  float2 p = __ffma2_rn(make_float2(0.05517113208770752f, 0.05517113208770752f), f,
-                        make_float2(0.24261008203029633f, 0.24261008203029633f));
-  p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
-  p = __ffma2_rn(p, f, make_float2(0.9999281167984009f, 0.9999281167984009f));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 // A bounded wait that gives up at once after any role of the CTA has given up.
@@ -442,7 +415,7 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
           for (int i = 0; i < 16; ++i) {
             const float2 xy = __ffma2_rn(make_float2(__uint_as_float(v[c][2 * i]), __uint_as_float(v[c][2 * i + 1])),
                                          sl2x2, negm);
-            const float2 p = ((kPolyMask >> i) & 1u) ? ex2_fma2(xy) : make_float2(ex2(xy.x), ex2(xy.y));
+            const float2 p = make_float2(ex2(xy.x), ex2(xy.y));
             w[i] = pack_pair<T>(p.x, p.y);
             ls[i & 3] = __fadd2_rn(ls[i & 3], p);
           }
