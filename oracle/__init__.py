@@ -20,9 +20,9 @@ import numpy as np
 
 from . import build as _build
 
-F16, BF16, E4M3 = 0, 1, 2
+F16, BF16, E4M3, E4M3_BLOCK = 0, 1, 2, 3   # E4M3_BLOCK: E4M3 codes, one scale per (block, kv head)
 _DTYPE_CODES = {"f16": F16, "fp16": F16, "float16": F16, "bf16": BF16, "bfloat16": BF16,
-                "fp8_e4m3": E4M3, "e4m3": E4M3}
+                "fp8_e4m3": E4M3, "e4m3": E4M3, "fp8_e4m3_block": E4M3_BLOCK}
 
 _default = None
 
@@ -289,3 +289,21 @@ def quantize_e4m3(values_bits, in_dtype, scale_per_head):
     if any(statuses):
         raise OracleError(f"quantize_e4m3 failed with statuses {statuses}")
     return out.reshape(vb.shape)
+
+
+def quantize_e4m3_blocks(pool_bits, in_dtype, scale_per_block):
+    """E4M3 codes of a whole pool [NB, bs, Hkv, d] of 16-bit values with one scale per (block, kv
+    head) ([NB, Hkv]): the same arithmetic as writing every slot through reshape_and_cache into a
+    per-block-scaled E4M3 cache."""
+    vb = _c(pool_bits, np.uint16)
+    NB, bs, Hkv, d = vb.shape
+    sc = _c(np.repeat(_c(scale_per_block, np.float32), bs, axis=0), np.float32)   # one row per slot
+    rows = vb.reshape(NB * bs, Hkv, d)
+    out = np.zeros((NB * bs, 1, Hkv, d), np.uint8)
+    scratch = np.zeros_like(out)
+    sm = np.arange(NB * bs, dtype=np.int64)
+    st = lib().or_reshape_and_cache(_ptr(rows), _ptr(rows), dtype_code(in_dtype), _ptr(out), _ptr(scratch),
+                                    E4M3_BLOCK, _ptr(sc), _ptr(sc), _ptr(sm), NB * bs, Hkv, d, 1, NB * bs)
+    if st:
+        raise OracleError(f"quantize_e4m3_blocks failed with status {st}")
+    return out.reshape(NB, bs, Hkv, d)

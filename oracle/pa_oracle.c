@@ -34,7 +34,9 @@
  *    ((blk*block_size + off)*num_kv_heads + h)*head_size + i;
  *  - grouped-query heads: query head h reads kv head h / (num_heads / num_kv_heads);
  *  - a context of length 0 gives an all-zero output row;
- *  - FP8 values dequantise as code_value * scale[kv_head]; quantisation is
+ *  - FP8 values dequantise as code_value * scale[kv_head] (per-head format), or code_value *
+ *    scale[block][kv_head] (per-block format: [T] sec. 3.2 stores blocks in FP8 one by one, so each
+ *    block may carry its own scale); quantisation is
  *    code = nearest E4M3 value to (float)x / scale (IEEE single division), ties to the even code,
  *    magnitudes >= 448 (and infinities) saturate to +-448, every NaN maps to the canonical NaN code
  *    0x7F (the OCP spec does not fix the sign of a NaN produced by a conversion);
@@ -47,7 +49,8 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { OR_F16 = 0, OR_BF16 = 1, OR_E4M3 = 2 };
+/* OR_E4M3_BLOCK: E4M3 codes like OR_E4M3, with one scale per (block, kv head) instead of per kv head. */
+enum { OR_F16 = 0, OR_BF16 = 1, OR_E4M3 = 2, OR_E4M3_BLOCK = 3 };
 
 enum {
   OR_OK = 0,
@@ -159,6 +162,14 @@ static double element(const void* base, int dtype, size_t index) {
   }
 }
 
+/* Dequantisation scale of kv head kvh for a token in physical block blk: 1 for 16-bit caches, the
+ * kv head's scale for the per-head E4M3 format, the (block, kv head) scale for the per-block one. */
+static double kv_scale(const float* scale, int kv_dtype, int blk, int num_kv_heads, int kvh) {
+  if (kv_dtype == OR_E4M3) return (double)scale[kvh];
+  if (kv_dtype == OR_E4M3_BLOCK) return (double)scale[(size_t)blk * num_kv_heads + kvh];
+  return 1.0;
+}
+
 /* ------------------------------------------------------------------------------------------------
  * Paged decode attention, by definition ([T] sec. 2.2 formula; indirection per [T] sec. 2.1,
  * [V] "PagedAttention的破局思路", [C] "PagedAttention：把显存做成虚拟内存").
@@ -198,15 +209,13 @@ static int attend_one(const or_attention_job* a, int s, int h, double* z) {
   for (int i = 0; i < d; ++i) o[i] = 0.0;
   if (L == 0) return OR_OK;
 
-  const double ks = (a->kv_dtype == OR_E4M3) ? (double)a->k_scale[kvh] : 1.0;
-  const double vs = (a->kv_dtype == OR_E4M3) ? (double)a->v_scale[kvh] : 1.0;
-
   /* Scores. */
   for (int t = 0; t < L; ++t) {
     int blk = a->block_tables[(size_t)s * a->max_blocks_per_seq + t / a->block_size];
     int off = t % a->block_size;
     if (blk < 0 || blk >= a->num_blocks) return OR_BAD_BLOCK;
     size_t k_base = (((size_t)blk * a->block_size + off) * a->num_kv_heads + kvh) * d;
+    const double ks = kv_scale(a->k_scale, a->kv_dtype, blk, a->num_kv_heads, kvh);
     double dot = 0.0;
     for (int i = 0; i < d; ++i)
       dot += element(a->query, a->q_dtype, q_base + i) * (element(a->key_cache, a->kv_dtype, k_base + i) * ks);
@@ -223,6 +232,7 @@ static int attend_one(const or_attention_job* a, int s, int h, double* z) {
     int blk = a->block_tables[(size_t)s * a->max_blocks_per_seq + t / a->block_size];
     int off = t % a->block_size;
     size_t v_base = (((size_t)blk * a->block_size + off) * a->num_kv_heads + kvh) * d;
+    const double vs = kv_scale(a->v_scale, a->kv_dtype, blk, a->num_kv_heads, kvh);
     double w = exp(z[t] - m) / denom;
     for (int i = 0; i < d; ++i) o[i] += w * (element(a->value_cache, a->kv_dtype, v_base + i) * vs);
   }
@@ -261,8 +271,8 @@ int or_paged_attention(double* out, const void* query, int q_dtype, const void* 
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return OR_BAD_ARG;
   if (head_size <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq < 0) return OR_BAD_ARG;
   if (q_dtype != OR_F16 && q_dtype != OR_BF16) return OR_BAD_ARG;
-  if (kv_dtype != OR_F16 && kv_dtype != OR_BF16 && kv_dtype != OR_E4M3) return OR_BAD_ARG;
-  if (kv_dtype == OR_E4M3 && (!k_scale || !v_scale)) return OR_BAD_ARG;
+  if (kv_dtype != OR_F16 && kv_dtype != OR_BF16 && kv_dtype != OR_E4M3 && kv_dtype != OR_E4M3_BLOCK) return OR_BAD_ARG;
+  if ((kv_dtype == OR_E4M3 || kv_dtype == OR_E4M3_BLOCK) && (!k_scale || !v_scale)) return OR_BAD_ARG;
   for (int s = 0; s < num_seqs; ++s)
     if (context_lens[s] < 0 || (long)context_lens[s] > (long)max_blocks_per_seq * block_size) return OR_BAD_ARG;
   if (num_threads < 1) num_threads = 1;
@@ -301,7 +311,8 @@ int or_paged_attention(double* out, const void* query, int q_dtype, const void* 
 /* ------------------------------------------------------------------------------------------------
  * Writing new tokens into their slots ([V] "PagedAttention的破局思路": blocks are filled as the
  * sequence grows). Token i of key/value [T][Hkv][d] goes to slot slot_mapping[i], i.e. block
- * slot / bs, offset slot % bs. E4M3 caches store or_e4m3_from_float((float)x / scale[h]).
+ * slot / bs, offset slot % bs. E4M3 caches store or_e4m3_from_float((float)x / scale), with scale the
+ * kv head's (scale[h]) or, in the per-block format, the slot's block's (scale[block][h]).
  * --------------------------------------------------------------------------------------------- */
 int or_reshape_and_cache(const void* key, const void* value, int in_dtype, void* key_cache,
                          void* value_cache, int kv_dtype, const float* k_scale, const float* v_scale,
@@ -309,8 +320,9 @@ int or_reshape_and_cache(const void* key, const void* value, int in_dtype, void*
                          int head_size, int block_size, int64_t num_blocks) {
   if (!key || !value || !key_cache || !value_cache || !slot_mapping) return OR_BAD_ARG;
   if (in_dtype != OR_F16 && in_dtype != OR_BF16) return OR_BAD_ARG;
-  if (kv_dtype != in_dtype && kv_dtype != OR_E4M3) return OR_BAD_ARG;
-  if (kv_dtype == OR_E4M3 && (!k_scale || !v_scale)) return OR_BAD_ARG;
+  const int fp8 = kv_dtype == OR_E4M3 || kv_dtype == OR_E4M3_BLOCK;
+  if (kv_dtype != in_dtype && !fp8) return OR_BAD_ARG;
+  if (fp8 && (!k_scale || !v_scale)) return OR_BAD_ARG;
   for (int64_t i = 0; i < num_tokens; ++i) {
     int64_t slot = slot_mapping[i];
     if (slot < 0 || slot >= num_blocks * block_size) continue;
@@ -326,8 +338,9 @@ int or_reshape_and_cache(const void* key, const void* value, int in_dtype, void*
           /* The input value is exact in float; the division is IEEE single precision. */
           float kx = (float)element(key, in_dtype, src);
           float vx = (float)element(value, in_dtype, src);
-          float ky = kx / k_scale[h];
-          float vy = vx / v_scale[h];
+          size_t sidx = (kv_dtype == OR_E4M3_BLOCK) ? (size_t)blk * num_kv_heads + h : (size_t)h;
+          float ky = kx / k_scale[sidx];
+          float vy = vx / v_scale[sidx];
           ((uint8_t*)key_cache)[dst] = or_e4m3_from_float(ky);
           ((uint8_t*)value_cache)[dst] = or_e4m3_from_float(vy);
         }
@@ -345,7 +358,7 @@ int or_copy_blocks(void* key_cache, void* value_cache, int kv_dtype, const int64
                    int64_t num_pairs, int num_kv_heads, int head_size, int block_size,
                    int64_t num_blocks) {
   if (!key_cache || !value_cache || (!block_mapping && num_pairs > 0)) return OR_BAD_ARG;
-  size_t elem = (kv_dtype == OR_E4M3) ? 1 : 2;
+  size_t elem = (kv_dtype == OR_E4M3 || kv_dtype == OR_E4M3_BLOCK) ? 1 : 2;
   size_t block_bytes = (size_t)block_size * num_kv_heads * head_size * elem;
   for (int64_t p = 0; p < num_pairs; ++p) {
     int64_t src = block_mapping[2 * p], dst = block_mapping[2 * p + 1];
@@ -367,7 +380,7 @@ int or_swap_blocks(void* dst_key_cache, void* dst_value_cache, const void* src_k
                    int64_t src_num_blocks, int64_t dst_num_blocks) {
   if (!dst_key_cache || !dst_value_cache || !src_key_cache || !src_value_cache || (!block_mapping && num_pairs > 0))
     return OR_BAD_ARG;
-  size_t elem = (kv_dtype == OR_E4M3) ? 1 : 2;
+  size_t elem = (kv_dtype == OR_E4M3 || kv_dtype == OR_E4M3_BLOCK) ? 1 : 2;
   size_t block_bytes = (size_t)block_size * num_kv_heads * head_size * elem;
   for (int64_t p = 0; p < num_pairs; ++p) {
     int64_t src = block_mapping[2 * p], dst = block_mapping[2 * p + 1];

@@ -34,8 +34,8 @@ MUTANTS = [
     ("fp8_subnormal_exponent", "v = ldexp((double)mantissa, -9);", "v = ldexp((double)mantissa, -10);"),
     ("fp8_bias", "v = ldexp(1.0 + mantissa / 8.0, exponent - 7);", "v = ldexp(1.0 + mantissa / 8.0, exponent - 8);"),
     ("fp8_ties_away", "pick = (lo % 2 == 0) ? lo : hi;", "pick = hi;"),
-    ("fp8_k_scale_dropped", "const double ks = (a->kv_dtype == OR_E4M3) ? (double)a->k_scale[kvh] : 1.0;",
-     "const double ks = 1.0;"),
+    ("fp8_k_scale_dropped", "(element(a->key_cache, a->kv_dtype, k_base + i) * ks);",
+     "(element(a->key_cache, a->kv_dtype, k_base + i));"),
     ("bf16_bias", "v = ldexp(1.0 + fraction / 128.0, exponent - 127);", "v = ldexp(1.0 + fraction / 128.0, exponent - 126);"),
 ]
 
