@@ -174,16 +174,15 @@ def run_reference(args, cfg, world, rank):
     n, dt = 1, 0.0
     while True:
         w = W.make_workload(cfg, seed=cfg.seed, num_seqs=n, prefilled=True)
-        inp = dict(query_bits=bits16(w.query), q_dtype=cfg.dtype, key_cache=bits16(w.key_values),
-                   value_cache=bits16(w.value_values), kv_dtype=cfg.kv_dtype, block_tables=w.block_tables.numpy(),
-                   context_lens=w.context_lens.numpy(), scale=cfg.softmax_scale)
+        inp = oracle_inputs(cfg, w)
         t0 = time.perf_counter()
         oracle.paged_attention(**inp)
         dt = time.perf_counter() - t0
         if dt >= 0.5 or n >= cfg.num_seqs:
             break
         n = min(cfg.num_seqs, max(n * 2, int(n * 1.0 / max(dt, 1e-3))))
-    kv = W.ideal_bytes(w.context_lens.numpy(), cfg.num_kv_heads, cfg.head_size, 2, cfg.block_size,
+    kv = W.ideal_bytes(w.context_lens.numpy(), cfg.num_kv_heads, cfg.head_size,
+                       1 if cfg.kv_dtype.startswith("fp8") else 2, cfg.block_size,
                        cfg.num_heads, 2)["kv"]
     for _ in range(args.warmup):
         oracle.paged_attention(**inp)
@@ -263,10 +262,10 @@ def main():
     dev = torch.device("cuda", local)
     w = W.make_workload(cfg, seed=cfg.seed + 1000 * rank, device=dev, num_seqs=args.num_seqs)
     S, H, d = w.query.shape
-    kv_bytes = 1 if cfg.kv_dtype == "fp8_e4m3" else 2
+    kv_bytes = 1 if cfg.kv_dtype.startswith("fp8") else 2
     ks = vs = None
     key_cache, value_cache = w.key_values, w.value_values
-    if cfg.kv_dtype == "fp8_e4m3":
+    if cfg.kv_dtype.startswith("fp8"):
         # The product's own quantiser fills the FP8 pools from the drawn values.
         NB, bs, Hkv, _ = key_cache.shape
         ks, vs = w.k_scale.to(dev), w.v_scale.to(dev)
@@ -753,6 +752,22 @@ def run_plan(args, cfg, plan_steps=200):
     print(json.dumps(line), flush=True)
 
 
+def oracle_inputs(cfg, w):
+    """The workload as oracle arrays (FP8 pools quantised by the oracle's own encoder)."""
+    import oracle
+    kb, vb = bits16(w.key_values), bits16(w.value_values)
+    ks = vs = None
+    if cfg.kv_dtype == "fp8_e4m3":
+        ks, vs = w.k_scale.cpu().numpy(), w.v_scale.cpu().numpy()
+        kb, vb = oracle.quantize_e4m3(kb, cfg.dtype, ks), oracle.quantize_e4m3(vb, cfg.dtype, vs)
+    elif cfg.kv_dtype == "fp8_e4m3_block":
+        ks, vs = w.k_scale.cpu().numpy(), w.v_scale.cpu().numpy()
+        kb, vb = oracle.quantize_e4m3_blocks(kb, cfg.dtype, ks), oracle.quantize_e4m3_blocks(vb, cfg.dtype, vs)
+    return dict(query_bits=bits16(w.query), q_dtype=cfg.dtype, key_cache=kb, value_cache=vb, kv_dtype=cfg.kv_dtype,
+                block_tables=w.block_tables.cpu().numpy(), context_lens=w.context_lens.cpu().numpy(),
+                scale=cfg.softmax_scale, k_scale=ks, v_scale=vs)
+
+
 def cpu_baseline(cfg, seconds):
     """The oracle (as it stands) on a bounded sample of the same workload, on the host cores."""
     import dataclasses
@@ -761,9 +776,7 @@ def cpu_baseline(cfg, seconds):
     n = 1
     while True:
         w = W.make_workload(cfg, seed=cfg.seed, num_seqs=n, prefilled=True)
-        inp = dict(query_bits=bits16(w.query), q_dtype=cfg.dtype, key_cache=bits16(w.key_values),
-                   value_cache=bits16(w.value_values), kv_dtype=cfg.kv_dtype, block_tables=w.block_tables.numpy(),
-                   context_lens=w.context_lens.numpy(), scale=cfg.softmax_scale)
+        inp = oracle_inputs(cfg, w)
         t0 = time.perf_counter()
         oracle.paged_attention(**inp)
         dt = time.perf_counter() - t0
@@ -777,7 +790,8 @@ def cpu_baseline(cfg, seconds):
         total += time.perf_counter() - t0
         reps += 1
     t = total / reps
-    kv = W.ideal_bytes(w.context_lens.numpy(), cfg.num_kv_heads, cfg.head_size, 2, cfg.block_size,
+    kv = W.ideal_bytes(w.context_lens.numpy(), cfg.num_kv_heads, cfg.head_size,
+                       1 if cfg.kv_dtype.startswith("fp8") else 2, cfg.block_size,
                        cfg.num_heads, 2)["kv"]
     return {"value": round(kv / t / 1e9, 4), "unit": "GB/s", "cores": oracle.default_threads(), "kind": "oracle",
             "sample": f"{n} of {cfg.num_seqs} sequences ({int(w.context_lens.sum())} context tokens), "

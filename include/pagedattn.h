@@ -69,7 +69,15 @@ typedef enum pa_status {
 typedef enum pa_dtype {
   PA_F16 = 0,                           /* IEEE binary16 */
   PA_BF16 = 1,                          /* bfloat16 */
-  PA_FP8_E4M3 = 2                       /* OCP FP8 E4M3 (bias 7, max 448, no infinities) */
+  PA_FP8_E4M3 = 2,                      /* OCP FP8 E4M3 (bias 7, max 448, no infinities); k_scale and
+                                           v_scale hold one fp32 scale per kv head: [num_kv_heads] */
+  PA_FP8_E4M3_BLOCK = 3                 /* the same E4M3 codes with one scale per (block, kv head):
+                                           k_scale, v_scale are [num_blocks][num_kv_heads] (tutorial
+                                           page "企业官网建设流程全解析", sec. 3.2: blocks are stored in
+                                           FP8 one by one, so each carries its own scale). Copying a
+                                           block (copy_blocks, swap_blocks) does not copy its scales:
+                                           the caller keeps them with the block. Attention with this
+                                           format needs num_heads / num_kv_heads >= 2. */
 } pa_dtype;
 
 /* Bits of the device error word (pa_get_device_error). */

@@ -32,6 +32,8 @@ using pa_host::ceil_div;
 using pa_host::elem_bytes;
 using pa_host::is_16bit;
 using pa_host::is_dtype;
+using pa_host::is_fp8;
+using pa_host::scale_block_stride;
 using pa_host::round_up;
 using pa_host::tensor_map_encoder;
 
@@ -151,9 +153,11 @@ pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dtype, con
   if (!aligned(out, 16) || !aligned(query, 16) || !aligned(key_cache, 16) || !aligned(value_cache, 16) ||
       !aligned(workspace, 16) || !aligned(block_tables, 4) || !aligned(context_lens, 4))
     return PA_ERR_INVALID_ARGUMENT;
-  const bool fp8 = kv_dtype == PA_FP8_E4M3;
+  const bool fp8 = is_fp8(kv_dtype);
   if (fp8 && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4))) return PA_ERR_INVALID_ARGUMENT;
   if (!fp8 && kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;
+  // Per-block scales are applied per 8-token box in the tensor-core path (grouped query heads).
+  if (kv_dtype == PA_FP8_E4M3_BLOCK && num_heads / num_kv_heads < 2) return PA_ERR_UNSUPPORTED;
   if (head_size != 64 && head_size != 128) return PA_ERR_UNSUPPORTED;
   if (fp8 && head_size != 128) return PA_ERR_UNSUPPORTED;
   if (!supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
@@ -204,6 +208,7 @@ pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dtype, con
   a.num_partitions = partitions;
   a.num_items = static_cast<unsigned int>(items);
   a.scale_log2 = scale * pa::kLog2e;
+  a.scale_block_stride = scale_block_stride(kv_dtype, num_kv_heads);
   const int grid = static_cast<int>(std::min<unsigned long long>(static_cast<unsigned long long>(sms), items));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = q_dtype == PA_BF16 ? pa::launch_attention_bf16(tk, tv, a, fp8, head_size, g_tile, grid, st)
@@ -223,9 +228,10 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dtype in_d
   if (!aligned(key, 16) || !aligned(value, 16) || !aligned(key_cache, 16) || !aligned(value_cache, 16) ||
       !aligned(slot_mapping, 8))
     return PA_ERR_INVALID_ARGUMENT;
-  const bool fp8 = kv_dtype == PA_FP8_E4M3;
+  const bool fp8 = is_fp8(kv_dtype);
   if (fp8 && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4))) return PA_ERR_INVALID_ARGUMENT;
   if (!fp8 && kv_dtype != in_dtype) return PA_ERR_UNSUPPORTED;
+  const int sstride = scale_block_stride(kv_dtype, num_kv_heads);
   if (head_size % 8 != 0) return PA_ERR_UNSUPPORTED;
   if (num_tokens == 0) return PA_OK;
   const int row = num_kv_heads * head_size;
@@ -237,23 +243,23 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dtype in_d
       pa::reshape_and_cache_kernel<__nv_bfloat16, __nv_fp8_e4m3><<<grid, threads, 0, st>>>(
           static_cast<const __nv_bfloat16*>(key), static_cast<const __nv_bfloat16*>(value),
           static_cast<__nv_fp8_e4m3*>(key_cache), static_cast<__nv_fp8_e4m3*>(value_cache), k_scale, v_scale,
-          slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+          slot_mapping, num_kv_heads, head_size, block_size, num_blocks, sstride);
     else
       pa::reshape_and_cache_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, threads, 0, st>>>(
           static_cast<const __nv_bfloat16*>(key), static_cast<const __nv_bfloat16*>(value),
           static_cast<__nv_bfloat16*>(key_cache), static_cast<__nv_bfloat16*>(value_cache), k_scale, v_scale,
-          slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+          slot_mapping, num_kv_heads, head_size, block_size, num_blocks, sstride);
   } else {
     if (fp8)
       pa::reshape_and_cache_kernel<__half, __nv_fp8_e4m3><<<grid, threads, 0, st>>>(
           static_cast<const __half*>(key), static_cast<const __half*>(value), static_cast<__nv_fp8_e4m3*>(key_cache),
           static_cast<__nv_fp8_e4m3*>(value_cache), k_scale, v_scale, slot_mapping, num_kv_heads, head_size,
-          block_size, num_blocks);
+          block_size, num_blocks, sstride);
     else
       pa::reshape_and_cache_kernel<__half, __half><<<grid, threads, 0, st>>>(
           static_cast<const __half*>(key), static_cast<const __half*>(value), static_cast<__half*>(key_cache),
           static_cast<__half*>(value_cache), k_scale, v_scale, slot_mapping, num_kv_heads, head_size, block_size,
-          num_blocks);
+          num_blocks, sstride);
   }
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -289,9 +295,10 @@ pa_status pa_reshape_and_cache_layers(const void* const* keys, const void* const
   if (!aligned(keys, 8) || !aligned(values, 8) || !aligned(key_caches, 8) || !aligned(value_caches, 8) ||
       !aligned(slot_mapping, 8))
     return PA_ERR_INVALID_ARGUMENT;
-  const bool fp8 = kv_dtype == PA_FP8_E4M3;
+  const bool fp8 = is_fp8(kv_dtype);
   if (fp8 && (!k_scales || !v_scales || !aligned(k_scales, 8) || !aligned(v_scales, 8))) return PA_ERR_INVALID_ARGUMENT;
   if (!fp8 && kv_dtype != in_dtype) return PA_ERR_UNSUPPORTED;
+  const int sstride = scale_block_stride(kv_dtype, num_kv_heads);
   if (head_size % 8 != 0 || num_layers > 65535) return PA_ERR_UNSUPPORTED;
   if (num_tokens == 0 || num_layers == 0) return PA_OK;
   const int row = num_kv_heads * head_size;
@@ -303,17 +310,17 @@ pa_status pa_reshape_and_cache_layers(const void* const* keys, const void* const
   if (in_dtype == PA_BF16) {
     if (fp8)
       pa::reshape_and_cache_layers_kernel<__nv_bfloat16, __nv_fp8_e4m3><<<grid, threads, 0, st>>>(
-          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks, sstride);
     else
       pa::reshape_and_cache_layers_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, threads, 0, st>>>(
-          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks, sstride);
   } else {
     if (fp8)
       pa::reshape_and_cache_layers_kernel<__half, __nv_fp8_e4m3><<<grid, threads, 0, st>>>(
-          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks, sstride);
     else
       pa::reshape_and_cache_layers_kernel<__half, __half><<<grid, threads, 0, st>>>(
-          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks, sstride);
   }
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -94,6 +94,7 @@ struct AttnArgs {
   int num_partitions;
   unsigned int num_items;       // num_partitions * num_seqs * head_blocks * subgroups
   float scale_log2;             // softmax scale * log2(e)
+  int scale_block_stride;       // FP8 scales: 0 = per kv head, num_kv_heads = per (block, kv head)
 };
 
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
@@ -143,6 +144,8 @@ struct StageMsg {
   int ntok;    // valid tokens in the stage
   int flags;   // kMsgFirst | kMsgLast | kMsgBadBlock
   int pad;
+  int blk[2];  // physical block of each 8-token box (for per-block scales; 0 when not loaded)
+  int pad2[2];
 };
 
 struct ItemInfo {
@@ -409,12 +412,20 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
               aborted = true;
               break;
             }
+            // Block of box 0 and box 1 (their lanes' ids) for per-block scales; unloaded or invalid
+            // boxes report block 0, a valid index whose scales meet only zero weights or NaN rows.
+            const int safe_blk = (mine && blk < args.num_blocks) ? blk : 0;
+            const int blk0 = __shfl_sync(0xffffffffu, safe_blk, 0);
+            const int blk1 = __shfl_sync(0xffffffffu, safe_blk, (2 * S::kChunks) & 31);
             if (lane == 0) {
               StageMsg m;
               m.item = local;
               m.ntok = ntok;
               m.flags = (k == 0 ? kMsgFirst : 0) | (k == n_stages - 1 ? kMsgLast : 0) | (bad ? kMsgBadBlock : 0);
               m.pad = 0;
+              m.blk[0] = blk0;
+              m.blk[1] = S::kGroups > 1 ? blk1 : blk0;
+              m.pad2[0] = m.pad2[1] = 0;
               msgs[slot] = m;
               if (bad) atomicOr(err, PA_DEVERR_BLOCK_ID);
               mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nbox * 2 * S::kChunks * S::kBoxBytes));
@@ -443,7 +454,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
       bool ok = true;
       if (lane == 0) ok = mbar_wait(&empty[slot], (static_cast<uint32_t>(issued / kStages) & 1u) ^ 1u, err);
       if (__shfl_sync(0xffffffffu, ok, 0) && lane == 0) {
-        msgs[slot] = StageMsg{-1, 0, 0, 0};
+        msgs[slot] = StageMsg{-1, 0, 0, 0, {0, 0}, {0, 0}};
         mbar_arrive(&full[slot]);
       }
       ++issued;
@@ -583,14 +594,27 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             }
           }
         }
-        // Scores of query head lane/4 for tokens 8*gr + 2*t4 and 8*gr + 2*t4 + 1.
-        const float zscale = (EB == 1) ? args.scale_log2 * args.k_scale[inf.kvh0 + cw] : args.scale_log2;
+        // Scores of query head lane/4 for tokens 8*gr + 2*t4 and 8*gr + 2*t4 + 1. FP8 scales: K's scales
+        // the scores of its box, V's the weights that enter P V of its box (per-block scales), or the
+        // output (per-head scales).
+        float zs[NG], vsb[NG];
+#pragma unroll
+        for (int gr = 0; gr < NG; ++gr) {
+          zs[gr] = args.scale_log2;
+          vsb[gr] = 1.0f;
+          if constexpr (EB == 1) {
+            const int kvh = inf.kvh0 + cw;
+            const int si = args.scale_block_stride ? m.blk[gr] * args.scale_block_stride + kvh : kvh;
+            zs[gr] *= __ldg(args.k_scale + si);
+            if (args.scale_block_stride) vsb[gr] = __ldg(args.v_scale + si);
+          }
+        }
         float sv[NG][2];
         float cm = -INFINITY;
 #pragma unroll
         for (int gr = 0; gr < NG; ++gr) {
-          sv[gr][0] = gr * kBoxTokens + 2 * t4 < nvalid ? sacc[gr][0] * zscale : -INFINITY;
-          sv[gr][1] = gr * kBoxTokens + 2 * t4 + 1 < nvalid ? sacc[gr][1] * zscale : -INFINITY;
+          sv[gr][0] = gr * kBoxTokens + 2 * t4 < nvalid ? sacc[gr][0] * zs[gr] : -INFINITY;
+          sv[gr][1] = gr * kBoxTokens + 2 * t4 + 1 < nvalid ? sacc[gr][1] * zs[gr] : -INFINITY;
           cm = fmaxf(cm, fmaxf(sv[gr][0], sv[gr][1]));
         }
         cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
@@ -601,10 +625,14 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         float psum = 0.f;
 #pragma unroll
         for (int gr = 0; gr < NG; ++gr) {
-          pfrag[gr] = pack2<MmaT>(fast_exp2(sv[gr][0] - m_new), fast_exp2(sv[gr][1] - m_new));
+          const float p0 = fast_exp2(sv[gr][0] - m_new), p1 = fast_exp2(sv[gr][1] - m_new);
+          pfrag[gr] = pack2<MmaT>(p0, p1);
           // The sum uses the rounded weights that enter P V, so the weights of the output sum to one.
           const float2 pr = unpack2<MmaT>(pfrag[gr]);
           psum += pr.x + pr.y;
+          // Per-block V scales ride on the weights of their box (the sum keeps the unscaled ones).
+          if constexpr (EB == 1)
+            if (args.scale_block_stride) pfrag[gr] = pack2<MmaT>(pr.x * vsb[gr], pr.y * vsb[gr]);
         }
         l_run = l_run * alpha + psum;
         m_run = m_new;
@@ -750,7 +778,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
         const int g = lane >> 2, t4 = lane & 3;
         if (g < inf.heads) {
-          float r = ((EB == 1) ? args.v_scale[inf.kvh0 + cw] : 1.0f) / l_tot;
+          float r = ((EB == 1 && !args.scale_block_stride) ? args.v_scale[inf.kvh0 + cw] : 1.0f) / l_tot;
           if (poisoned) r = __int_as_float(0x7fc00000);
           const int h = (inf.kvh0 + cw) * args.group + inf.h_sub + g;
           const size_t rowi = (static_cast<size_t>(inf.s) * args.num_heads + h) * args.num_partitions + inf.part;

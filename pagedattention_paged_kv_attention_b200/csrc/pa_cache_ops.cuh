@@ -19,7 +19,8 @@ __device__ __forceinline__ void reshape_and_cache_token(const IT* __restrict__ k
                                                         const float* __restrict__ k_scale,
                                                         const float* __restrict__ v_scale,
                                                         const int64_t* __restrict__ slot_mapping, int num_kv_heads,
-                                                        int head_size, int block_size, int num_blocks) {
+                                                        int head_size, int block_size, int num_blocks,
+                                                        int scale_stride) {
   const int64_t token = blockIdx.x;
   const int64_t slot = slot_mapping[token];
   if (slot < 0 || slot >= static_cast<int64_t>(num_blocks) * block_size) return;
@@ -36,9 +37,10 @@ __device__ __forceinline__ void reshape_and_cache_token(const IT* __restrict__ k
       *reinterpret_cast<uint4*>(key_cache + dst_base + e) = kin;
       *reinterpret_cast<uint4*>(value_cache + dst_base + e) = vin;
     } else {
-      // E4M3: code = cvt.rn.satfinite(x / scale), the division correctly rounded (IEEE).
+      // E4M3: code = cvt.rn.satfinite(x / scale), the division correctly rounded (IEEE); the scale is
+      // the kv head's, or with per-block scales (scale_stride = num_kv_heads) the slot's block's.
       const int h = e / head_size;
-      const float ks = k_scale[h], vs = v_scale[h];
+      const float ks = k_scale[blk * scale_stride + h], vs = v_scale[blk * scale_stride + h];
       const IT* kx = reinterpret_cast<const IT*>(&kin);
       const IT* vx = reinterpret_cast<const IT*>(&vin);
       uint32_t kout[2], vout[2];
@@ -69,9 +71,9 @@ __global__ void __launch_bounds__(256)
 reshape_and_cache_kernel(const IT* __restrict__ key, const IT* __restrict__ value, KVT* __restrict__ key_cache,
                          KVT* __restrict__ value_cache, const float* __restrict__ k_scale,
                          const float* __restrict__ v_scale, const int64_t* __restrict__ slot_mapping,
-                         int num_kv_heads, int head_size, int block_size, int num_blocks) {
+                         int num_kv_heads, int head_size, int block_size, int num_blocks, int scale_stride) {
   reshape_and_cache_token<IT, KVT>(key, value, key_cache, value_cache, k_scale, v_scale, slot_mapping, num_kv_heads,
-                                   head_size, block_size, num_blocks);
+                                   head_size, block_size, num_blocks, scale_stride);
 }
 
 // All layers in one launch: grid (tokens, layers); per-layer pointers come from device arrays.
@@ -81,12 +83,12 @@ reshape_and_cache_layers_kernel(const void* const* __restrict__ keys, const void
                                 void* const* __restrict__ key_caches, void* const* __restrict__ value_caches,
                                 const float* const* __restrict__ k_scales, const float* const* __restrict__ v_scales,
                                 const int64_t* __restrict__ slot_mapping, int num_kv_heads, int head_size,
-                                int block_size, int num_blocks) {
+                                int block_size, int num_blocks, int scale_stride) {
   const int layer = blockIdx.y;
   reshape_and_cache_token<IT, KVT>(static_cast<const IT*>(keys[layer]), static_cast<const IT*>(values[layer]),
                                    static_cast<KVT*>(key_caches[layer]), static_cast<KVT*>(value_caches[layer]),
                                    k_scales ? k_scales[layer] : nullptr, v_scales ? v_scales[layer] : nullptr,
-                                   slot_mapping, num_kv_heads, head_size, block_size, num_blocks);
+                                   slot_mapping, num_kv_heads, head_size, block_size, num_blocks, scale_stride);
 }
 
 // One CTA per (pair, key|value): copy one contiguous block of `block_bytes` (a multiple of 16).

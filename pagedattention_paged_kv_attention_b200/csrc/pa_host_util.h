@@ -17,8 +17,11 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 inline bool is_16bit(pa_dtype t) { return t == PA_F16 || t == PA_BF16; }
-inline bool is_dtype(pa_dtype t) { return t == PA_F16 || t == PA_BF16 || t == PA_FP8_E4M3; }
-inline int elem_bytes(pa_dtype t) { return t == PA_FP8_E4M3 ? 1 : 2; }
+inline bool is_fp8(pa_dtype t) { return t == PA_FP8_E4M3 || t == PA_FP8_E4M3_BLOCK; }
+inline bool is_dtype(pa_dtype t) { return t == PA_F16 || t == PA_BF16 || is_fp8(t); }
+inline int elem_bytes(pa_dtype t) { return is_fp8(t) ? 1 : 2; }
+// Scale index stride per block: 0 for per-kv-head scales, num_kv_heads for per-(block, kv head) ones.
+inline int scale_block_stride(pa_dtype t, int num_kv_heads) { return t == PA_FP8_E4M3_BLOCK ? num_kv_heads : 0; }
 
 inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;

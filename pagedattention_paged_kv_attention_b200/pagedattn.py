@@ -15,7 +15,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIBRARY_PATH = os.path.join(_HERE, "libpagedattn.so")
 
 PA_OK, PA_ERR_INVALID_ARGUMENT, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL, PA_ERR_CUDA, PA_ERR_OUT_OF_BLOCKS = range(6)
-PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
+PA_F16, PA_BF16, PA_FP8_E4M3, PA_FP8_E4M3_BLOCK = 0, 1, 2, 3
 PA_DEVERR_BLOCK_ID, PA_DEVERR_CONTEXT_LEN, PA_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 WORKSPACE_HEADER_BYTES = 256
 
@@ -122,6 +122,15 @@ def dtype_code(t: torch.dtype) -> int:
     raise ValueError(f"unsupported dtype {t}")
 
 
+def cache_code(cache: torch.Tensor, k_scale=None) -> int:
+    """The cache format: 16-bit, or E4M3 with per-kv-head scales ([Hkv]) or per-(block, kv head)
+    scales ([num_blocks, Hkv])."""
+    code = dtype_code(cache.dtype)
+    if code == PA_FP8_E4M3 and k_scale is not None and k_scale.dim() == 2:
+        return PA_FP8_E4M3_BLOCK
+    return code
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -157,7 +166,7 @@ def paged_attention(out, query, key_cache, value_cache, block_tables, context_le
     NB, bs, Hkv, d2 = key_cache.shape
     st = lib.pa_paged_attention(
         _ptr(out), _ptr(query), dtype_code(query.dtype), _ptr(key_cache), _ptr(value_cache),
-        dtype_code(key_cache.dtype), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), block_tables.shape[1],
+        cache_code(key_cache, k_scale), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), block_tables.shape[1],
         _ptr(context_lens), S, H, Hkv, d, bs, NB, int(max_context_len), float(scale), int(partition_size),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "pa_paged_attention")
@@ -188,7 +197,7 @@ def paged_attention_static(out, query, key_cache, value_cache, block_tables, con
     NB, bs, Hkv, d2 = key_cache.shape
     st = lib.pa_paged_attention_static(
         _ptr(out), _ptr(query), dtype_code(query.dtype), _ptr(key_cache), _ptr(value_cache),
-        dtype_code(key_cache.dtype), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), block_tables.shape[1],
+        cache_code(key_cache, k_scale), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), block_tables.shape[1],
         _ptr(context_lens), S, H, Hkv, d, bs, NB, int(max_context_len), float(scale), int(partition_size),
         _ptr(device_error_out), _stream(stream))
     _check(st, "pa_paged_attention_static")
@@ -200,7 +209,7 @@ def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, k_scale=
     T, Hkv, d = key.shape
     NB, bs = key_cache.shape[0], key_cache.shape[1]
     st = lib.pa_reshape_and_cache(_ptr(key), _ptr(value), dtype_code(key.dtype), _ptr(key_cache),
-                                  _ptr(value_cache), dtype_code(key_cache.dtype), _ptr(k_scale), _ptr(v_scale),
+                                  _ptr(value_cache), cache_code(key_cache, k_scale), _ptr(k_scale), _ptr(v_scale),
                                   _ptr(slot_mapping), T, Hkv, d, bs, NB, _stream(stream))
     _check(st, "pa_reshape_and_cache")
 
@@ -228,7 +237,8 @@ def reshape_and_cache_layers(keys, values, key_caches, value_caches, slot_mappin
     ks = pointer_array(k_scales) if k_scales is not None else None
     vs = pointer_array(v_scales) if v_scales is not None else None
     st = lib.pa_reshape_and_cache_layers(*[_ptr(a) for a in arrays[:2]], dtype_code(keys[0].dtype),
-                                         *[_ptr(a) for a in arrays[2:]], dtype_code(key_caches[0].dtype), _ptr(ks),
+                                         *[_ptr(a) for a in arrays[2:]],
+                                         cache_code(key_caches[0], k_scales[0] if k_scales is not None else None), _ptr(ks),
                                          _ptr(vs), _ptr(slot_mapping), T, L, Hkv, d, bs, NB, _stream(stream))
     _check(st, "pa_reshape_and_cache_layers")
     return arrays  # keep the pointer arrays alive until the stream has used them

@@ -10,7 +10,7 @@ import torch
 import oracle
 from helpers import bits16
 
-TOLERANCE = {"f16": 2e-3, "bf16": 1e-2, "fp8_e4m3": 3e-2}   # max-abs, per cache dtype
+TOLERANCE = {"f16": 2e-3, "bf16": 1e-2, "fp8_e4m3": 3e-2, "fp8_e4m3_block": 3e-2}   # max-abs, per cache format
 MANTISSA_BITS = {"f16": 10, "bf16": 7}
 
 
@@ -31,6 +31,9 @@ def initial_pools(w):
     if cfg.kv_dtype == "fp8_e4m3":
         kb = oracle.quantize_e4m3(kb, cfg.dtype, w.k_scale.numpy())
         vb = oracle.quantize_e4m3(vb, cfg.dtype, w.v_scale.numpy())
+    elif cfg.kv_dtype == "fp8_e4m3_block":
+        kb = oracle.quantize_e4m3_blocks(kb, cfg.dtype, w.k_scale.numpy())
+        vb = oracle.quantize_e4m3_blocks(vb, cfg.dtype, w.v_scale.numpy())
     return kb, vb
 
 
@@ -49,7 +52,7 @@ def oracle_step(w, kc, vc, write_new=True, copy=True):
 
 
 def to_device_pool(arr, cfg):
-    if cfg.kv_dtype == "fp8_e4m3":
+    if cfg.kv_dtype.startswith("fp8"):
         return torch.from_numpy(arr).cuda()                       # uint8 codes
     t = torch.from_numpy(arr.view(np.int16)).cuda()
     return t.view(torch.bfloat16 if cfg.kv_dtype == "bf16" else torch.float16)

@@ -50,7 +50,7 @@ class Config:
     head_size: int
     block_size: int
     dtype: str                      # query / output / new-token dtype: "f16" or "bf16"
-    kv_dtype: str                   # "f16", "bf16" or "fp8_e4m3"
+    kv_dtype: str                   # "f16", "bf16", "fp8_e4m3" (per-kv-head scales) or "fp8_e4m3_block"
     seed: int
     context_lens: Optional[Sequence[int]] = None   # explicit lengths
     len_range: Optional[tuple] = None              # uniform [lo, hi]
@@ -97,6 +97,13 @@ CONFIGS = {
                     "with per-kv-head fp32 scale, reshape_and_cache of 256 tokens + copy_blocks of 64 pairs",
         num_seqs=256, num_heads=32, num_kv_heads=8, head_size=128, block_size=16, dtype="bf16",
         kv_dtype="fp8_e4m3", seed=5, len_range=(1, 512), shared_prefix_tokens=1024, cow_pairs=64),
+    "shared_prefix_fp8_block": Config(
+        name="shared_prefix_fp8_block",
+        description="the shared-prefix serving batch with an FP8-E4M3 cache scaled per (block, kv head): 256 "
+                    "seqs, 1024-token shared prefix + suffixes U[1,512], 32 q / 8 kv heads, head_size 128, "
+                    "block_size 16, reshape_and_cache of 256 tokens + copy_blocks of 64 pairs",
+        num_seqs=256, num_heads=32, num_kv_heads=8, head_size=128, block_size=16, dtype="bf16",
+        kv_dtype="fp8_e4m3_block", seed=6, len_range=(1, 512), shared_prefix_tokens=1024, cow_pairs=64),
 }
 
 
@@ -122,7 +129,7 @@ class Workload:
     new_value: torch.Tensor
     slot_mapping: torch.Tensor      # int64 [S]
     cow_mapping: torch.Tensor       # int64 [N, 2]
-    k_scale: Optional[torch.Tensor]  # float32 [Hkv] (FP8 only)
+    k_scale: Optional[torch.Tensor]  # float32 [Hkv], or [num_blocks, Hkv] for per-block scales (FP8 only)
     v_scale: Optional[torch.Tensor]
 
     @property
@@ -197,8 +204,9 @@ def make_workload(cfg: Config, seed: Optional[int] = None, device="cpu", num_seq
         cursor += n_priv
 
     tdtype = _TORCH_DTYPES[cfg.dtype]
-    store_dtype = tdtype if cfg.kv_dtype == "fp8_e4m3" else _TORCH_DTYPES[cfg.kv_dtype]
-    store_key = cfg.dtype if cfg.kv_dtype == "fp8_e4m3" else cfg.kv_dtype
+    fp8 = cfg.kv_dtype.startswith("fp8")
+    store_dtype = tdtype if fp8 else _TORCH_DTYPES[cfg.kv_dtype]
+    store_key = cfg.dtype if fp8 else cfg.kv_dtype
     dev = torch.device(device)
 
     def gen(s):
@@ -243,6 +251,19 @@ def make_workload(cfg: Config, seed: Optional[int] = None, device="cpu", num_seq
         v_amax = value_pool[used_t].float().abs().amax(dim=(0, 1, 3))
         k_scale = (k_amax / FP8_MAX).to(torch.float32)
         v_scale = (v_amax / FP8_MAX).to(torch.float32)
+    elif cfg.kv_dtype == "fp8_e4m3_block":
+        # One scale per (block, kv head): max |x| over the block's drawn values of that head / 448;
+        # blocks without data get 1; copy-on-write destinations carry their source block's scales.
+        scales = []
+        for pool in (key_pool, value_pool):
+            sc = torch.ones((NB, Hkv), dtype=torch.float32, device=dev)
+            amax = pool[used_t].float().abs().amax(dim=(1, 3))
+            sc[used_t] = torch.where(amax > 0, amax / FP8_MAX, torch.ones_like(amax))
+            if cfg.cow_pairs:
+                src = torch.from_numpy(used[:cfg.cow_pairs].astype(np.int64)).to(dev)
+                sc[torch.from_numpy(cow_dst.astype(np.int64)).to(dev)] = sc[src]
+            scales.append(sc)
+        k_scale, v_scale = scales
 
     # Poison the tail of each sequence's last block (from L-1, or from L when prefilled).
     for s in range(S):
