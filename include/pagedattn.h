@@ -34,9 +34,10 @@
  * Token t of sequence s is stored in physical block block_tables[s][t / block_size] at offset
  * t % block_size ([T] sec. 2.1; [V] "PagedAttention的破局思路").
  *
- * Supported set: head_size in {64, 128}; block_size in {8, 16, 32, 64}; num_heads % num_kv_heads == 0;
- * query/output dtype PA_F16 or PA_BF16; cache dtype equal to the query dtype, or PA_FP8_E4M3 with
- * head_size 128. Anything else returns PA_ERR_UNSUPPORTED.
+ * Supported set (decode attention): head_size in {64, 128}; block_size in {8, 16, 32, 64};
+ * num_heads % num_kv_heads == 0; num_blocks < 2^27; query/output dtype PA_F16 or PA_BF16; cache dtype
+ * equal to the query dtype, or PA_FP8_E4M3 / PA_FP8_E4M3_BLOCK with head_size 128 (the per-block format
+ * also needs num_heads / num_kv_heads >= 2). Anything else returns PA_ERR_UNSUPPORTED.
  */
 #ifndef PAGEDATTN_H_
 #define PAGEDATTN_H_

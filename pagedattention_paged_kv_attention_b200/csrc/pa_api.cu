@@ -161,6 +161,7 @@ pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dtype, con
   if (head_size != 64 && head_size != 128) return PA_ERR_UNSUPPORTED;
   if (fp8 && head_size != 128) return PA_ERR_UNSUPPORTED;
   if (!supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+  if (num_blocks >= (1 << 27)) return PA_ERR_UNSUPPORTED;  // block ids ride in 28 bits of a stage message
   const int ps = plan_partition(num_seqs, num_heads, num_kv_heads, max_context_len, partition_size);
   if (ps <= 0) return PA_ERR_INVALID_ARGUMENT;
   const int partitions = std::max(1, ceil_div(max_context_len, ps));

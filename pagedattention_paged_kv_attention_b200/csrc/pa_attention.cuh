@@ -67,6 +67,7 @@ constexpr int kWsDone = 2;
 
 // Stage message flags.
 constexpr int kMsgFirst = 1;
+constexpr int kMsgBlkShift = 4;  // StageMsg.flags: bits 0-3 flags, bits 4-31 box 0's block id
 constexpr int kMsgLast = 2;
 constexpr int kMsgBadBlock = 4;
 
@@ -143,10 +144,8 @@ struct StageMsg {
   int item;    // CTA-local item sequence number, -1 = no more work
   int ntok;    // valid tokens in the stage
   int flags;   // kMsgFirst | kMsgLast | kMsgBadBlock
-  int pad;
-  int blk[2];  // physical block of each 8-token box (for per-block scales; 0 when not loaded)
-  int pad2[2];
-};
+  int blk1;    // physical blocks of the stage's two 8-token boxes, for per-block scales (0 when a box
+};             // is not loaded); box 0's is carried in flags >> kMsgBlkShift
 
 struct ItemInfo {
   int s, part, kvh0, h_sub, heads, write_final, pad0, pad1;  // h_sub: first query-head offset in a group
@@ -250,7 +249,9 @@ __device__ __forceinline__ bool context_len_invalid(int L, const AttnArgs& a) {
   return L < 0 || L > a.max_blocks_per_seq * a.block_size || L > a.num_partitions * a.partition_size;
 }
 
-template <typename QT, typename KVT, int D, int G>
+// BS: FP8 cache with per-(block, kv head) scales (args.scale_block_stride != 0); a separate
+// instantiation so that the per-head FP8 path carries none of its work.
+template <typename QT, typename KVT, int D, int G, bool BS>
 __global__ void __launch_bounds__(kThreads, 1)
 paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                      const AttnArgs args) {
@@ -414,18 +415,19 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             }
             // Block of box 0 and box 1 (their lanes' ids) for per-block scales; unloaded or invalid
             // boxes report block 0, a valid index whose scales meet only zero weights or NaN rows.
-            const int safe_blk = (mine && blk < args.num_blocks) ? blk : 0;
-            const int blk0 = __shfl_sync(0xffffffffu, safe_blk, 0);
-            const int blk1 = __shfl_sync(0xffffffffu, safe_blk, (2 * S::kChunks) & 31);
+            int blk0 = 0, blk1 = 0;
+            if constexpr (BS) {
+              const int safe_blk = (mine && blk < args.num_blocks) ? blk : 0;
+              blk0 = __shfl_sync(0xffffffffu, safe_blk, 0);
+              blk1 = __shfl_sync(0xffffffffu, safe_blk, (2 * S::kChunks) & 31);
+            }
             if (lane == 0) {
               StageMsg m;
               m.item = local;
               m.ntok = ntok;
               m.flags = (k == 0 ? kMsgFirst : 0) | (k == n_stages - 1 ? kMsgLast : 0) | (bad ? kMsgBadBlock : 0);
-              m.pad = 0;
-              m.blk[0] = blk0;
-              m.blk[1] = S::kGroups > 1 ? blk1 : blk0;
-              m.pad2[0] = m.pad2[1] = 0;
+              m.flags |= blk0 << kMsgBlkShift;
+              m.blk1 = S::kGroups > 1 ? blk1 : blk0;
               msgs[slot] = m;
               if (bad) atomicOr(err, PA_DEVERR_BLOCK_ID);
               mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nbox * 2 * S::kChunks * S::kBoxBytes));
@@ -454,7 +456,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
       bool ok = true;
       if (lane == 0) ok = mbar_wait(&empty[slot], (static_cast<uint32_t>(issued / kStages) & 1u) ^ 1u, err);
       if (__shfl_sync(0xffffffffu, ok, 0) && lane == 0) {
-        msgs[slot] = StageMsg{-1, 0, 0, 0, {0, 0}, {0, 0}};
+        msgs[slot] = StageMsg{-1, 0, 0, 0};
         mbar_arrive(&full[slot]);
       }
       ++issued;
@@ -483,6 +485,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     float o[S::kNBlocks][4];      // tensor-core path: output accumulator fragments
     bool poisoned = false;
     bool active = false;  // this warp's kv head exists in the current item
+    float zitem = 0.f;    // per-head FP8: scale_log2 * k_scale of this warp's kv head for the item
     ItemInfo inf{};
 
     for (int j = 0;; ++j) {
@@ -499,8 +502,9 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         active = inf.kvh0 + cw < args.num_kv_heads;
         float qscale = args.scale_log2;
         if constexpr (EB == 1) {
-          if (active) qscale *= args.k_scale[inf.kvh0 + cw];
+          if (active && !BS) qscale *= args.k_scale[inf.kvh0 + cw];
         }
+        zitem = qscale;
         const QT* qs = reinterpret_cast<const QT*>(smem + Lay::kQuery + qb * Lay::kQueryOne) + cw * G * D;
         if constexpr (S::kMma) {
           const int g = lane >> 2, t4 = lane & 3;
@@ -600,13 +604,15 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         float zs[NG], vsb[NG];
 #pragma unroll
         for (int gr = 0; gr < NG; ++gr) {
-          zs[gr] = args.scale_log2;
+          zs[gr] = zitem;
           vsb[gr] = 1.0f;
-          if constexpr (EB == 1) {
-            const int kvh = inf.kvh0 + cw;
-            const int si = args.scale_block_stride ? m.blk[gr] * args.scale_block_stride + kvh : kvh;
-            zs[gr] *= __ldg(args.k_scale + si);
-            if (args.scale_block_stride) vsb[gr] = __ldg(args.v_scale + si);
+          if constexpr (BS) {
+            {
+              const int blk = gr == 0 ? (m.flags >> kMsgBlkShift) : m.blk1;
+              const int si = blk * args.scale_block_stride + inf.kvh0 + cw;
+              zs[gr] = args.scale_log2 * __ldg(args.k_scale + si);
+              vsb[gr] = __ldg(args.v_scale + si);
+            }
           }
         }
         float sv[NG][2];
@@ -631,8 +637,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           const float2 pr = unpack2<MmaT>(pfrag[gr]);
           psum += pr.x + pr.y;
           // Per-block V scales ride on the weights of their box (the sum keeps the unscaled ones).
-          if constexpr (EB == 1)
-            if (args.scale_block_stride) pfrag[gr] = pack2<MmaT>(pr.x * vsb[gr], pr.y * vsb[gr]);
+          if constexpr (BS) pfrag[gr] = pack2<MmaT>(pr.x * vsb[gr], pr.y * vsb[gr]);
         }
         l_run = l_run * alpha + psum;
         m_run = m_new;
@@ -778,7 +783,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 2);
         const int g = lane >> 2, t4 = lane & 3;
         if (g < inf.heads) {
-          float r = ((EB == 1 && !args.scale_block_stride) ? args.v_scale[inf.kvh0 + cw] : 1.0f) / l_tot;
+          float r = ((EB == 1 && !BS) ? args.v_scale[inf.kvh0 + cw] : 1.0f) / l_tot;
           if (poisoned) r = __int_as_float(0x7fc00000);
           const int h = (inf.kvh0 + cw) * args.group + inf.h_sub + g;
           const size_t rowi = (static_cast<size_t>(inf.s) * args.num_heads + h) * args.num_partitions + inf.part;

@@ -9,12 +9,12 @@
 
 namespace pa {
 
-template <typename QT, typename KVT, int D, int G>
+template <typename QT, typename KVT, int D, int G, bool BS = false>
 cudaError_t launch_attention_one(const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a, int grid,
                                  cudaStream_t stream) {
   constexpr int EB = Elem<KVT>::kBytes;
   constexpr size_t smem = Layout<QT, D, G, EB>::kAllocBytes;
-  auto kernel = paged_attention_main<QT, KVT, D, G>;
+  auto kernel = paged_attention_main<QT, KVT, D, G, BS>;
   // The attribute is per device; setting it on every call costs a few microseconds of host time at
   // most and keeps multi-device processes correct.
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -35,7 +35,13 @@ template <typename QT, typename KVT>
 cudaError_t launch_attention(const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a, int D, int G,
                              int grid, cudaStream_t stream) {
   if constexpr (sizeof(KVT) == 1) {
-    if (D == 128) {
+    if (D == 128 && a.scale_block_stride != 0) {  // per-block scales: grouped heads only
+      switch (G) {
+        case 2: return launch_attention_one<QT, KVT, 128, 2, true>(tk, tv, a, grid, stream);
+        case 4: return launch_attention_one<QT, KVT, 128, 4, true>(tk, tv, a, grid, stream);
+        case 8: return launch_attention_one<QT, KVT, 128, 8, true>(tk, tv, a, grid, stream);
+      }
+    } else if (D == 128) {
       switch (G) {
         case 1: return launch_attention_one<QT, KVT, 128, 1>(tk, tv, a, grid, stream);
         case 2: return launch_attention_one<QT, KVT, 128, 2>(tk, tv, a, grid, stream);
