@@ -116,17 +116,6 @@ __device__ __forceinline__ uint32_t pack_pair<__half>(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
-template <typename T>
-__device__ __forceinline__ float2 unpack_pair(uint32_t w);
-template <>
-__device__ __forceinline__ float2 unpack_pair<__nv_bfloat16>(uint32_t w) {
-  return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w));
-}
-template <>
-__device__ __forceinline__ float2 unpack_pair<__half>(uint32_t w) {
-  return __half22float2(*reinterpret_cast<__half2*>(&w));
-}
-
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 1)
 paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
