@@ -36,8 +36,8 @@
  *
  * Supported set (decode attention): head_size in {64, 128}; block_size in {8, 16, 32, 64};
  * num_heads % num_kv_heads == 0; num_blocks < 2^27; query/output dtype PA_F16 or PA_BF16; cache dtype
- * equal to the query dtype, or PA_FP8_E4M3 / PA_FP8_E4M3_BLOCK with head_size 128 (the per-block format
- * also needs num_heads / num_kv_heads >= 2). Anything else returns PA_ERR_UNSUPPORTED.
+ * equal to the query dtype, or PA_FP8_E4M3 / PA_FP8_E4M3_BLOCK with head_size 128. Anything else returns
+ * PA_ERR_UNSUPPORTED.
  */
 #ifndef PAGEDATTN_H_
 #define PAGEDATTN_H_
@@ -77,8 +77,7 @@ typedef enum pa_dtype {
                                            page "企业官网建设流程全解析", sec. 3.2: blocks are stored in
                                            FP8 one by one, so each carries its own scale). Copying a
                                            block (copy_blocks, swap_blocks) does not copy its scales:
-                                           the caller keeps them with the block. Attention with this
-                                           format needs num_heads / num_kv_heads >= 2. */
+                                           the caller keeps them with the block. */
 } pa_dtype;
 
 /* Bits of the device error word (pa_get_device_error). */

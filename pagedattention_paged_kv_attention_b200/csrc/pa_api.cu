@@ -156,8 +156,6 @@ pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dtype, con
   const bool fp8 = is_fp8(kv_dtype);
   if (fp8 && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4))) return PA_ERR_INVALID_ARGUMENT;
   if (!fp8 && kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;
-  // Per-block scales are applied per 8-token box in the tensor-core path (grouped query heads).
-  if (kv_dtype == PA_FP8_E4M3_BLOCK && num_heads / num_kv_heads < 2) return PA_ERR_UNSUPPORTED;
   if (head_size != 64 && head_size != 128) return PA_ERR_UNSUPPORTED;
   if (fp8 && head_size != 128) return PA_ERR_UNSUPPORTED;
   if (!supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;

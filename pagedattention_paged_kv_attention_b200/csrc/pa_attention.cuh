@@ -695,6 +695,17 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         const int nvalid = m.ntok;
         const uint8_t* ktile = smem + Lay::kRing + slot * S::kStageBytes;
         const uint8_t* vtile = ktile + S::kTileBytes;
+        // Per-block FP8 scales of the stage's two 8-token boxes (K scales the scores, V the weights).
+        float ksb[2] = {1.f, 1.f}, vsb2[2] = {1.f, 1.f};
+        if constexpr (BS) {
+#pragma unroll
+          for (int bx = 0; bx < 2; ++bx) {
+            const int blk = bx == 0 ? (m.flags >> kMsgBlkShift) : m.blk1;
+            const int si = blk * args.scale_block_stride + inf.kvh0 + cw;
+            ksb[bx] = __ldg(args.k_scale + si);
+            vsb2[bx] = __ldg(args.v_scale + si);
+          }
+        }
         // ---- scores ----
         float sc[S::kIters];
 #pragma unroll
@@ -717,7 +728,8 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           float v[G];
 #pragma unroll
           for (int g = 0; g < G; ++g) v[g] = pacc[g].x + pacc[g].y;
-          const float z = reduce_scatter<G, S::kLog2NS>(v, lane);
+          float z = reduce_scatter<G, S::kLog2NS>(v, lane);
+          if constexpr (BS) z *= ksb[t / kBoxTokens];
           sc[it] = t < nvalid ? z : -INFINITY;
         }
         // ---- online softmax (per head g_lane) ----
@@ -763,6 +775,10 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             } else {
 #pragma unroll
               for (int g = 0; g < G; ++g) p[g] = pw[t * G + g];
+            }
+            if constexpr (BS) {
+#pragma unroll
+              for (int g = 0; g < G; ++g) p[g] *= vsb2[t / kBoxTokens];
             }
 #pragma unroll
             for (int g = 0; g < G; ++g) {
@@ -835,7 +851,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             }
         }
         // l and m of head g live on the primary lanes with tslot 0 (lane g << (log2 NS - log2 G)).
-        const float vscale = (EB == 1) ? args.v_scale[inf.kvh0 + cw] : 1.0f;
+        const float vscale = (EB == 1 && !BS) ? args.v_scale[inf.kvh0 + cw] : 1.0f;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const int src = g << (S::kLog2NS - S::kLog2G);

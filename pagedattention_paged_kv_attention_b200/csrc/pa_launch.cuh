@@ -35,8 +35,9 @@ template <typename QT, typename KVT>
 cudaError_t launch_attention(const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a, int D, int G,
                              int grid, cudaStream_t stream) {
   if constexpr (sizeof(KVT) == 1) {
-    if (D == 128 && a.scale_block_stride != 0) {  // per-block scales: grouped heads only
+    if (D == 128 && a.scale_block_stride != 0) {  // per-block scales
       switch (G) {
+        case 1: return launch_attention_one<QT, KVT, 128, 1, true>(tk, tv, a, grid, stream);
         case 2: return launch_attention_one<QT, KVT, 128, 2, true>(tk, tv, a, grid, stream);
         case 4: return launch_attention_one<QT, KVT, 128, 4, true>(tk, tv, a, grid, stream);
         case 8: return launch_attention_one<QT, KVT, 128, 8, true>(tk, tv, a, grid, stream);

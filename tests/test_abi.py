@@ -79,7 +79,7 @@ def call_attention(P, **over):
     (dict(kv_dtype=0), 2),                                                   # f16 cache with bf16 query
     (dict(kv_dtype=2, k_scale=16, v_scale=16, head_size=64), 2),
     (dict(kv_dtype=3), 1),                                                   # per-block FP8 without scales
-    (dict(kv_dtype=3, k_scale=16, v_scale=16, num_kv_heads=8), 2),          # per-block FP8 needs grouped heads
+    (dict(kv_dtype=3, k_scale=16, v_scale=16, head_size=64), 2),            # per-block FP8: head size 128 only
     (dict(kv_dtype=4, k_scale=16, v_scale=16), 1),                          # no such cache format
     (dict(workspace_bytes=255), 3), (dict(max_context_len=4096, partition_size=64, workspace_bytes=1024), 3),
     (dict(num_seqs=0), 0),                                                   # empty batch: nothing to do

@@ -83,7 +83,7 @@ for bs in (8, 16, 32):
         CASES.append(("fp8_e4m3", "bf16", 128, bs, H, Hkv))
         CASES.append(("fp8_e4m3", "f16", 128, bs, H, Hkv))
 for bs in (8, 16, 32):
-    for (H, Hkv) in ((8, 2), (32, 4), (64, 8), (12, 3)):
+    for (H, Hkv) in ((8, 2), (32, 4), (64, 8), (12, 3), (8, 8), (6, 1)):
         CASES.append(("fp8_e4m3_block", "bf16", 128, bs, H, Hkv))
     CASES.append(("fp8_e4m3_block", "f16", 128, bs, 16, 2))
 for (H, Hkv) in ((8, 8), (16, 2)):
