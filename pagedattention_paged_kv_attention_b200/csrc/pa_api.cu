@@ -237,30 +237,20 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dtype in_d
   const int threads = static_cast<int>(std::min<size_t>(256, round_up(static_cast<size_t>(ceil_div(row, 8)), 32)));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const dim3 grid(static_cast<unsigned>(num_tokens));
-  if (in_dtype == PA_BF16) {
-    if (fp8)
-      pa::reshape_and_cache_kernel<__nv_bfloat16, __nv_fp8_e4m3><<<grid, threads, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(key), static_cast<const __nv_bfloat16*>(value),
-          static_cast<__nv_fp8_e4m3*>(key_cache), static_cast<__nv_fp8_e4m3*>(value_cache), k_scale, v_scale,
-          slot_mapping, num_kv_heads, head_size, block_size, num_blocks, sstride);
-    else
-      pa::reshape_and_cache_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, threads, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(key), static_cast<const __nv_bfloat16*>(value),
-          static_cast<__nv_bfloat16*>(key_cache), static_cast<__nv_bfloat16*>(value_cache), k_scale, v_scale,
-          slot_mapping, num_kv_heads, head_size, block_size, num_blocks, sstride);
-  } else {
-    if (fp8)
-      pa::reshape_and_cache_kernel<__half, __nv_fp8_e4m3><<<grid, threads, 0, st>>>(
-          static_cast<const __half*>(key), static_cast<const __half*>(value), static_cast<__nv_fp8_e4m3*>(key_cache),
-          static_cast<__nv_fp8_e4m3*>(value_cache), k_scale, v_scale, slot_mapping, num_kv_heads, head_size,
-          block_size, num_blocks, sstride);
-    else
-      pa::reshape_and_cache_kernel<__half, __half><<<grid, threads, 0, st>>>(
-          static_cast<const __half*>(key), static_cast<const __half*>(value), static_cast<__half*>(key_cache),
-          static_cast<__half*>(value_cache), k_scale, v_scale, slot_mapping, num_kv_heads, head_size, block_size,
-          num_blocks, sstride);
-  }
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const auto launch = [&](auto in_tag, auto cache_tag) {
+    using IT = decltype(in_tag);
+    using KVT = decltype(cache_tag);
+    return pa_host::launch_overlapped(pa::reshape_and_cache_kernel<IT, KVT>, grid, dim3(threads), 0, st,
+                                      static_cast<const IT*>(key), static_cast<const IT*>(value),
+                                      static_cast<KVT*>(key_cache), static_cast<KVT*>(value_cache), k_scale, v_scale,
+                                      slot_mapping, num_kv_heads, head_size, block_size, num_blocks, sstride);
+  };
+  cudaError_t e;
+  if (in_dtype == PA_BF16)
+    e = fp8 ? launch(__nv_bfloat16{}, __nv_fp8_e4m3{}) : launch(__nv_bfloat16{}, __nv_bfloat16{});
+  else
+    e = fp8 ? launch(__half{}, __nv_fp8_e4m3{}) : launch(__half{}, __half{});
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_copy_blocks(void* key_cache, void* value_cache, pa_dtype kv_dtype, const int64_t* block_mapping,
@@ -276,9 +266,11 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, pa_dtype kv_dtype, 
   if (block_bytes % 16 != 0) return PA_ERR_UNSUPPORTED;
   if (num_pairs == 0) return PA_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  pa::copy_blocks_kernel<<<dim3(static_cast<unsigned>(num_pairs), 2), 256, 0, st>>>(
-      static_cast<uint8_t*>(key_cache), static_cast<uint8_t*>(value_cache), block_mapping, block_bytes, num_blocks);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const cudaError_t e = pa_host::launch_overlapped(pa::copy_blocks_kernel, dim3(static_cast<unsigned>(num_pairs), 2),
+                                                   dim3(256), 0, st, static_cast<uint8_t*>(key_cache),
+                                                   static_cast<uint8_t*>(value_cache), block_mapping, block_bytes,
+                                                   num_blocks);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_reshape_and_cache_layers(const void* const* keys, const void* const* values, pa_dtype in_dtype,

@@ -287,6 +287,10 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     }
     fence_mbar_init();
   }
+  // Everything above touched shared memory only; from here on the previous kernel's writes (the new
+  // tokens in the cache, a reset workspace) must be visible.
+  grid_dependency_wait();
+  grid_dependents_launch();
   __syncthreads();
 
   if (warp == 0) {
@@ -902,6 +906,8 @@ template <typename QT, int D>
 __global__ void __launch_bounds__(kReduceWarps * 32)
 paged_attention_reduce(const AttnArgs args) {
   constexpr int kPer = D / 32;  // elements per lane: 4 for d = 128, 2 for d = 64
+  grid_dependency_wait();
+  grid_dependents_launch();
   const int lane = threadIdx.x & 31;
   const long row = static_cast<long>(blockIdx.x) * kReduceWarps + (threadIdx.x >> 5);
   if (row >= static_cast<long>(args.num_seqs) * args.num_heads) return;

@@ -72,6 +72,8 @@ reshape_and_cache_kernel(const IT* __restrict__ key, const IT* __restrict__ valu
                          KVT* __restrict__ value_cache, const float* __restrict__ k_scale,
                          const float* __restrict__ v_scale, const int64_t* __restrict__ slot_mapping,
                          int num_kv_heads, int head_size, int block_size, int num_blocks, int scale_stride) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   reshape_and_cache_token<IT, KVT>(key, value, key_cache, value_cache, k_scale, v_scale, slot_mapping, num_kv_heads,
                                    head_size, block_size, num_blocks, scale_stride);
 }
@@ -95,6 +97,8 @@ reshape_and_cache_layers_kernel(const void* const* __restrict__ keys, const void
 __global__ void __launch_bounds__(256)
 copy_blocks_kernel(uint8_t* __restrict__ key_cache, uint8_t* __restrict__ value_cache,
                    const int64_t* __restrict__ block_mapping, int64_t block_bytes, int num_blocks) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   const int pair = blockIdx.x;
   const int64_t src = block_mapping[2 * pair];
   const int64_t dst = block_mapping[2 * pair + 1];

@@ -13,6 +13,19 @@
 namespace pa {
 
 // ------------------------------------------------------------------------------------------------
+// Programmatic dependent launch. A kernel launched with programmatic stream serialisation may be
+// scheduled while the kernel before it in the stream is still running; grid_dependency_wait() returns
+// once that kernel has completed and its memory operations are visible, so every global access comes
+// after it. grid_dependents_launch() lets the next such kernel be scheduled (its own wait still holds
+// it until this grid completes). Both are no-ops for a kernel launched without the attribute.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------------------------------
 // Shared-memory addresses and mbarriers.
 // ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -8,6 +8,7 @@
 
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "pagedattn.h"
 
@@ -34,6 +35,26 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
   return fn;
+}
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled while the previous kernel
+// in the stream is still running. Every kernel launched this way begins with grid_dependency_wait()
+// (pa_device.cuh) before any global-memory access, so stream order holds for memory and only the
+// launch latency and the shared-memory prologue overlap the previous kernel.
+template <typename... Params, typename... Args>
+cudaError_t launch_overlapped(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace pa_host

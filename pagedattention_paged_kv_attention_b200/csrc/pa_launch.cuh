@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include "pa_attention.cuh"
+#include "pa_host_util.h"
 
 namespace pa {
 
@@ -19,14 +20,13 @@ cudaError_t launch_attention_one(const CUtensorMap& tk, const CUtensorMap& tv, c
   // most and keeps multi-device processes correct.
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kernel<<<grid, kThreads, smem, stream>>>(tk, tv, a);
-  e = cudaGetLastError();
+  e = pa_host::launch_overlapped(kernel, dim3(grid), dim3(kThreads), smem, stream, tk, tv, a);
   if (e != cudaSuccess) return e;
   if (a.num_partitions > 1) {
     const long rows = static_cast<long>(a.num_heads) * a.num_seqs;
-    paged_attention_reduce<QT, D>
-        <<<static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps), kReduceWarps * 32, 0, stream>>>(a);
-    e = cudaGetLastError();
+    e = pa_host::launch_overlapped(paged_attention_reduce<QT, D>,
+                                   dim3(static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps)),
+                                   dim3(kReduceWarps * 32), 0, stream, a);
   }
   return e;
 }
