@@ -135,6 +135,33 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+_I32, _I64, _F32 = (torch.int32,), (torch.int64,), (torch.float32,)
+
+
+def _arg(t, name, dtypes=None, dim=None, cuda=True):
+    """The pointer of a tensor argument, after the checks the C ABI cannot make from a pointer: a dense
+    row-major layout, the element type the call reads, the rank, and (for kernel operands) residence
+    on a CUDA device. None passes through as a null pointer."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if dim is not None and t.dim() not in ((dim,) if isinstance(dim, int) else dim):
+        raise ValueError(f"{name}: expected {dim} dimensions, got shape {tuple(t.shape)}")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name}: expected dtype {' or '.join(map(str, dtypes))}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous (the library reads a dense row-major layout)")
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _same(a, b, what):
+    if a.shape != b.shape or a.dtype != b.dtype:
+        raise ValueError(f"{what}: shapes/dtypes differ ({tuple(a.shape)} {a.dtype} vs {tuple(b.shape)} {b.dtype})")
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -164,11 +191,15 @@ def paged_attention(out, query, key_cache, value_cache, block_tables, context_le
     """out[S,H,d] = paged decode attention of query[S,H,d] over key/value_cache[NB,bs,Hkv,d]."""
     S, H, d = query.shape
     NB, bs, Hkv, d2 = key_cache.shape
+    _same(out, query, "out/query")
+    _same(key_cache, value_cache, "key_cache/value_cache")
     st = lib.pa_paged_attention(
-        _ptr(out), _ptr(query), dtype_code(query.dtype), _ptr(key_cache), _ptr(value_cache),
-        cache_code(key_cache, k_scale), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), block_tables.shape[1],
-        _ptr(context_lens), S, H, Hkv, d, bs, NB, int(max_context_len), float(scale), int(partition_size),
-        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+        _arg(out, "out"), _arg(query, "query"), dtype_code(query.dtype), _arg(key_cache, "key_cache"),
+        _arg(value_cache, "value_cache"), cache_code(key_cache, k_scale), _arg(k_scale, "k_scale", _F32, (1, 2)),
+        _arg(v_scale, "v_scale", _F32, (1, 2)), _arg(block_tables, "block_tables", _I32, 2), block_tables.shape[1],
+        _arg(context_lens, "context_lens", _I32, 1), S, H, Hkv, d, bs, NB, int(max_context_len), float(scale),
+        int(partition_size), _arg(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream))
     _check(st, "pa_paged_attention")
     return out
 
@@ -179,11 +210,15 @@ def paged_prefill(out, query, key_cache, value_cache, block_tables, context_lens
     sequence s, the last rows of its context_lens[s] cached tokens) over key/value_cache[NB,bs,Hkv,d]."""
     T, H, d = query.shape
     NB, bs, Hkv, _ = key_cache.shape
-    st = lib.pa_paged_prefill(_ptr(out), _ptr(query), dtype_code(query.dtype), _ptr(key_cache), _ptr(value_cache),
-                              dtype_code(key_cache.dtype), _ptr(block_tables), block_tables.shape[1],
-                              _ptr(context_lens), _ptr(q_start), context_lens.shape[0], T, H, Hkv, d, bs, NB,
-                              int(max_q_len), float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                              _stream(stream))
+    _same(out, query, "out/query")
+    _same(key_cache, value_cache, "key_cache/value_cache")
+    st = lib.pa_paged_prefill(_arg(out, "out"), _arg(query, "query"), dtype_code(query.dtype),
+                              _arg(key_cache, "key_cache"), _arg(value_cache, "value_cache"),
+                              dtype_code(key_cache.dtype), _arg(block_tables, "block_tables", _I32, 2),
+                              block_tables.shape[1], _arg(context_lens, "context_lens", _I32, 1),
+                              _arg(q_start, "q_start", _I32, 1), context_lens.shape[0], T, H, Hkv, d, bs, NB,
+                              int(max_q_len), float(scale), _arg(workspace, "workspace"),
+                              workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "pa_paged_prefill")
 
 
@@ -195,11 +230,15 @@ def paged_attention_static(out, query, key_cache, value_cache, block_tables, con
     tensor of one element that receives the device error word."""
     S, H, d = query.shape
     NB, bs, Hkv, d2 = key_cache.shape
+    _same(out, query, "out/query")
+    _same(key_cache, value_cache, "key_cache/value_cache")
     st = lib.pa_paged_attention_static(
-        _ptr(out), _ptr(query), dtype_code(query.dtype), _ptr(key_cache), _ptr(value_cache),
-        cache_code(key_cache, k_scale), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), block_tables.shape[1],
-        _ptr(context_lens), S, H, Hkv, d, bs, NB, int(max_context_len), float(scale), int(partition_size),
-        _ptr(device_error_out), _stream(stream))
+        _arg(out, "out"), _arg(query, "query"), dtype_code(query.dtype), _arg(key_cache, "key_cache"),
+        _arg(value_cache, "value_cache"), cache_code(key_cache, k_scale), _arg(k_scale, "k_scale", _F32, (1, 2)),
+        _arg(v_scale, "v_scale", _F32, (1, 2)), _arg(block_tables, "block_tables", _I32, 2), block_tables.shape[1],
+        _arg(context_lens, "context_lens", _I32, 1), S, H, Hkv, d, bs, NB, int(max_context_len), float(scale),
+        int(partition_size), _arg(device_error_out, "device_error_out", (torch.int32, torch.uint32)),
+        _stream(stream))
     _check(st, "pa_paged_attention_static")
     return out
 
@@ -208,22 +247,31 @@ def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, k_scale=
     """Write key/value[T,Hkv,d] into the caches at slot_mapping[T] (int64)."""
     T, Hkv, d = key.shape
     NB, bs = key_cache.shape[0], key_cache.shape[1]
-    st = lib.pa_reshape_and_cache(_ptr(key), _ptr(value), dtype_code(key.dtype), _ptr(key_cache),
-                                  _ptr(value_cache), cache_code(key_cache, k_scale), _ptr(k_scale), _ptr(v_scale),
-                                  _ptr(slot_mapping), T, Hkv, d, bs, NB, _stream(stream))
+    _same(key, value, "key/value")
+    _same(key_cache, value_cache, "key_cache/value_cache")
+    st = lib.pa_reshape_and_cache(_arg(key, "key"), _arg(value, "value"), dtype_code(key.dtype),
+                                  _arg(key_cache, "key_cache"), _arg(value_cache, "value_cache"),
+                                  cache_code(key_cache, k_scale), _arg(k_scale, "k_scale", _F32, (1, 2)),
+                                  _arg(v_scale, "v_scale", _F32, (1, 2)),
+                                  _arg(slot_mapping, "slot_mapping", _I64, 1), T, Hkv, d, bs, NB, _stream(stream))
     _check(st, "pa_reshape_and_cache")
 
 
 def copy_blocks(key_cache, value_cache, block_mapping, stream=None):
     """Copy whole blocks block_mapping[N,2] (src, dst) (int64, device) in both caches."""
     NB, bs, Hkv, d = key_cache.shape
-    st = lib.pa_copy_blocks(_ptr(key_cache), _ptr(value_cache), dtype_code(key_cache.dtype), _ptr(block_mapping),
+    _same(key_cache, value_cache, "key_cache/value_cache")
+    st = lib.pa_copy_blocks(_arg(key_cache, "key_cache"), _arg(value_cache, "value_cache"),
+                            dtype_code(key_cache.dtype), _arg(block_mapping, "block_mapping", _I64, 2),
                             block_mapping.shape[0], Hkv, d, bs, NB, _stream(stream))
     _check(st, "pa_copy_blocks")
 
 
 def pointer_array(tensors, device="cuda"):
-    """A device int64 array holding the data pointers of `tensors` (for the *_layers calls)."""
+    """A device int64 array holding the data pointers of `tensors` (for the *_layers calls); each tensor
+    must be a contiguous CUDA tensor."""
+    for i, t in enumerate(tensors):
+        _arg(t, f"layer {i} tensor")
     return torch.tensor([t.data_ptr() for t in tensors], dtype=torch.int64, device=device)
 
 
@@ -239,7 +287,8 @@ def reshape_and_cache_layers(keys, values, key_caches, value_caches, slot_mappin
     st = lib.pa_reshape_and_cache_layers(*[_ptr(a) for a in arrays[:2]], dtype_code(keys[0].dtype),
                                          *[_ptr(a) for a in arrays[2:]],
                                          cache_code(key_caches[0], k_scales[0] if k_scales is not None else None), _ptr(ks),
-                                         _ptr(vs), _ptr(slot_mapping), T, L, Hkv, d, bs, NB, _stream(stream))
+                                         _ptr(vs), _arg(slot_mapping, "slot_mapping", _I64, 1), T, L, Hkv, d, bs, NB,
+                                         _stream(stream))
     _check(st, "pa_reshape_and_cache_layers")
     return arrays  # keep the pointer arrays alive until the stream has used them
 
@@ -249,7 +298,8 @@ def copy_blocks_layers(key_caches, value_caches, block_mapping, stream=None):
     NB, bs, Hkv, d = key_caches[0].shape
     kp, vp = pointer_array(key_caches), pointer_array(value_caches)
     st = lib.pa_copy_blocks_layers(_ptr(kp), _ptr(vp), len(key_caches), dtype_code(key_caches[0].dtype),
-                                   _ptr(block_mapping), block_mapping.shape[0], Hkv, d, bs, NB, _stream(stream))
+                                   _arg(block_mapping, "block_mapping", _I64, 2), block_mapping.shape[0], Hkv, d, bs,
+                                   NB, _stream(stream))
     _check(st, "pa_copy_blocks_layers")
     return kp, vp
 
@@ -258,9 +308,13 @@ def swap_blocks(dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, 
     """Copy whole blocks src_pool[m[i,0]] -> dst_pool[m[i,1]]; pools on the device or in pinned host memory."""
     NBs, bs, Hkv, d = src_key_cache.shape
     NBd = dst_key_cache.shape[0]
-    st = lib.pa_swap_blocks(_ptr(dst_key_cache), _ptr(dst_value_cache), _ptr(src_key_cache), _ptr(src_value_cache),
-                            dtype_code(src_key_cache.dtype), _ptr(block_mapping), block_mapping.shape[0], Hkv, d, bs,
-                            NBs, NBd, _stream(stream))
+    # Pools and mapping may be device or pinned host memory; the library refuses pageable memory.
+    st = lib.pa_swap_blocks(_arg(dst_key_cache, "dst_key_cache", cuda=False),
+                            _arg(dst_value_cache, "dst_value_cache", cuda=False),
+                            _arg(src_key_cache, "src_key_cache", cuda=False),
+                            _arg(src_value_cache, "src_value_cache", cuda=False), dtype_code(src_key_cache.dtype),
+                            _arg(block_mapping, "block_mapping", _I64, 2, cuda=False), block_mapping.shape[0], Hkv,
+                            d, bs, NBs, NBd, _stream(stream))
     _check(st, "pa_swap_blocks")
 
 

@@ -137,3 +137,41 @@ def test_layer_ops_reject_bad_arguments(P):
     assert cb(16, 16, 4, P.PA_BF16, None, 3, 2, 64, 16, 4, None) == 1
     assert cb(16, 16, 4, P.PA_BF16, 16, 3, 1, 4, 1, 4, None) == 2          # an 8-byte block: not 16-byte vectors
     assert cb(16, 16, 4, P.PA_BF16, 16, 0, 2, 64, 16, 4, None) == 0        # no pairs
+
+
+def test_binding_rejects_tensors_the_library_would_misread(P):
+    """The binding checks what a pointer cannot carry (layout, element type, rank, device) and raises
+    before any library call."""
+    import torch
+    bt = torch.zeros((4, 8), dtype=torch.int32)
+    assert P._arg(bt, "block_tables", P._I32, 2, cuda=False) is not None
+    assert P._arg(None, "k_scale") is None
+    with pytest.raises(ValueError, match="contiguous"):
+        P._arg(bt.t(), "block_tables", P._I32, 2, cuda=False)
+    with pytest.raises(ValueError, match="dtype"):
+        P._arg(bt.to(torch.int64), "block_tables", P._I32, 2, cuda=False)
+    with pytest.raises(ValueError, match="dimensions"):
+        P._arg(bt.view(-1), "block_tables", P._I32, 2, cuda=False)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        P._arg(bt, "block_tables", P._I32, 2)
+    with pytest.raises(TypeError):
+        P._arg(bt.numpy(), "block_tables", P._I32, 2, cuda=False)
+    q = torch.zeros((2, 8, 64), dtype=torch.bfloat16)
+    kc = torch.zeros((4, 16, 2, 64), dtype=torch.bfloat16)
+    cl = torch.zeros(2, dtype=torch.int32)
+    ws = torch.zeros(1024, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="out/query"):
+        P.paged_attention(torch.zeros((2, 8, 32), dtype=torch.bfloat16), q, kc, kc, bt[:2], cl, 0.1, 64, ws)
+    with pytest.raises(ValueError, match="key_cache/value_cache"):
+        P.paged_attention(q.clone(), q, kc, kc.half(), bt[:2], cl, 0.1, 64, ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):       # host tensors never reach a kernel
+        P.paged_attention(q.clone(), q, kc, kc, bt[:2], cl, 0.1, 64, ws)
+    x = torch.zeros((3, 2, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="key/value"):
+        P.reshape_and_cache(x, x[:2], kc, kc, torch.zeros(3, dtype=torch.int64))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        P.reshape_and_cache(x, x, kc, kc, torch.zeros(3, dtype=torch.int64))
+    with pytest.raises(ValueError, match="contiguous"):   # swap pools may be host memory, but dense
+        P.swap_blocks(kc.transpose(1, 2), kc, kc, kc, torch.zeros((1, 2), dtype=torch.int64))
+    with pytest.raises(ValueError, match="dtype"):
+        P.swap_blocks(kc, kc, kc, kc, torch.zeros((1, 2), dtype=torch.int32))
