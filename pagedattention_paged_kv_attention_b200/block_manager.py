@@ -9,6 +9,7 @@ from __future__ import annotations
 import ctypes
 
 import numpy as np
+import torch
 
 from .pagedattn import PA_ERR_OUT_OF_BLOCKS, PagedAttnError, _check, lib
 
@@ -25,12 +26,21 @@ def _call(status, where):
     _check(status, where)
 
 
-def _addr(a):
-    if a is None:
-        return None
-    if isinstance(a, np.ndarray):
-        return a.ctypes.data
-    return a.data_ptr()
+_TORCH_DTYPE = {np.int64: torch.int64, np.int32: torch.int32}
+
+
+def _host_out(a, dtype, count, name):
+    """Address of a caller-supplied output buffer, which the manager writes through a raw host
+    pointer: it must be a numpy array or a CPU (e.g. pinned) torch tensor of `dtype`, dense, with room
+    for `count` elements."""
+    if isinstance(a, torch.Tensor):
+        if a.dtype == _TORCH_DTYPE[dtype] and a.is_cpu and a.is_contiguous() and a.numel() >= count:
+            return a.data_ptr()
+    elif isinstance(a, np.ndarray):
+        if a.dtype == dtype and a.flags.c_contiguous and a.size >= count:
+            return a.ctypes.data
+    raise ValueError(f"plan_decode: `{name}` must be a dense host array of {np.dtype(dtype)} with at least "
+                     f"{count} elements")
 
 
 class BlockManager:
@@ -94,8 +104,10 @@ class BlockManager:
                    np.empty(n, np.int32))
         slots, cow, tables, lens = out
         k = ctypes.c_int()
-        _call(lib.pa_bm_plan_decode(self._h, ids.ctypes.data, n, _addr(slots), _addr(cow), ctypes.byref(k),
-                                    _addr(tables), max_blocks, pad, _addr(lens)), "pa_bm_plan_decode")
+        _call(lib.pa_bm_plan_decode(self._h, ids.ctypes.data, n, _host_out(slots, np.int64, n, "slot_mapping"),
+                                    _host_out(cow, np.int64, 2 * n, "cow"), ctypes.byref(k),
+                                    _host_out(tables, np.int32, n * max_blocks, "tables"), max_blocks, pad,
+                                    _host_out(lens, np.int32, n, "lens")), "pa_bm_plan_decode")
         return slots, cow[:k.value], tables, lens
 
     def free_sequence(self, seq_id: int):

@@ -136,6 +136,31 @@ def test_plan_decode_checks_width_before_changing_anything(BM):
     assert s.tolist() == [4 * 1 + 0] and t.tolist() == [[0, 1]] and l.tolist() == [5] and len(p) == 0
 
 
+def test_plan_decode_output_buffers_are_checked(BM):
+    """The manager writes the plan through raw host pointers: caller buffers that are too small, of the
+    wrong dtype, strided or on a device are refused before the call, and nothing changes."""
+    import torch
+    bm = BM.BlockManager(16, 4)
+    bm.add_sequence(0, 3)
+    bm.add_sequence(1, 5)
+    good = (torch.empty(2, dtype=torch.int64), torch.empty((2, 2), dtype=torch.int64),
+            torch.empty((2, 3), dtype=torch.int32), torch.empty(2, dtype=torch.int32))
+    bad = [
+        (torch.empty(1, dtype=torch.int64),) + good[1:],                                  # slots too small
+        good[:2] + (torch.empty((2, 3), dtype=torch.int64),) + good[3:],                  # tables int64
+        good[:2] + (torch.empty((3, 2), dtype=torch.int32).t(),) + good[3:],             # strided
+        good[:3] + (np.empty(2, np.int64),),                                              # lens int64
+        good[:1] + (torch.empty((2, 2), dtype=torch.int64, device="meta"),) + good[2:],  # not host memory
+    ]
+    for out in bad:
+        with pytest.raises(ValueError):
+            bm.plan_decode([0, 1], 3, 0, out)
+        assert bm.sequence_info(0) == (3, 1, False) and bm.sequence_info(1) == (5, 2, False)
+    s, p, t, l = bm.plan_decode([0, 1], 3, -1, good)
+    assert s.tolist() == [3, 4 * 2 + 1] and l.tolist() == [4, 6] and t.tolist() == [[0, -1, -1], [1, 2, -1]]
+    assert len(p) == 0
+
+
 def test_out_of_blocks_is_all_or_nothing(BM):
     bm = BM.BlockManager(3, 2)
     bm.add_sequence(0, 2)
