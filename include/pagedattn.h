@@ -35,7 +35,7 @@
  * t % block_size ([T] sec. 2.1; [V] "PagedAttention的破局思路").
  *
  * Supported set (decode attention): head_size in {64, 128}; block_size in {8, 16, 32, 64};
- * num_heads % num_kv_heads == 0; num_blocks < 2^27; query/output dtype PA_F16 or PA_BF16; cache dtype
+ * num_heads % num_kv_heads == 0; num_seqs <= 65535; num_blocks < 2^27; query/output dtype PA_F16 or PA_BF16; cache dtype
  * equal to the query dtype, or PA_FP8_E4M3 / PA_FP8_E4M3_BLOCK with head_size 128. Anything else returns
  * PA_ERR_UNSUPPORTED.
  */
@@ -206,15 +206,20 @@ PA_API pa_status pa_paged_prefill(void* out, const void* query, pa_dtype q_dtype
  * sequence grows). For token i with slot = slot_mapping[i] in [0, num_blocks*block_size):
  *     key_cache[slot / block_size][slot % block_size][h][:] = key[i][h][:]   (same for value)
  * slot < 0 marks padding and is skipped; slots past the pool are skipped too. For an FP8 cache each
- * element stores the E4M3 code of (float)x / k_scale[h] (IEEE division, round to nearest even,
- * magnitudes beyond 448 saturate, any NaN becomes the canonical NaN code 0x7F).
+ * element stores the E4M3 code of (float)x / scale (IEEE division, round to nearest even, magnitudes
+ * beyond 448 saturate, any NaN becomes the canonical NaN code 0x7F), where scale is k_scale[h]
+ * (PA_FP8_E4M3) or k_scale[slot / block_size][h] (PA_FP8_E4M3_BLOCK); v_scale likewise for values.
  *
  *  key, value     [num_tokens][num_kv_heads][head_size], in_dtype (PA_F16 or PA_BF16); read only.
  *  key_cache,
- *  value_cache    as above, kv_dtype = in_dtype or PA_FP8_E4M3; written at the given slots only.
+ *  value_cache    as above, kv_dtype = in_dtype, PA_FP8_E4M3 or PA_FP8_E4M3_BLOCK; written at the
+ *                 given slots only.
  *  k_scale,
- *  v_scale        [num_kv_heads] fp32, required for PA_FP8_E4M3.
+ *  v_scale        fp32, required for the FP8 formats: [num_kv_heads] for PA_FP8_E4M3,
+ *                 [num_blocks][num_kv_heads] for PA_FP8_E4M3_BLOCK (read only; the caller chooses each
+ *                 block's scale before writing into it).
  *  slot_mapping   [num_tokens] int64.
+ * Supported: head_size a multiple of 8 and num_kv_heads * head_size <= 2^24 (else PA_ERR_UNSUPPORTED).
  * Two tokens mapped to the same slot race (the result is one of them). num_tokens == 0 is a no-op
  * (pointers may then be null).
  */

@@ -104,6 +104,9 @@ bool encode_cache_map(CUtensorMap* map, const void* cache, int elem_bytes, int h
 
 bool supported_block_size(int bs) { return bs == 8 || bs == 16 || bs == 32 || bs == 64; }
 
+// Elements of one token's [num_kv_heads][head_size] row that the cache-write kernels index with int.
+constexpr int64_t kMaxRowElems = int64_t(1) << 24;
+
 }  // namespace
 
 extern "C" {
@@ -231,8 +234,7 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dtype in_d
   if (fp8 && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4))) return PA_ERR_INVALID_ARGUMENT;
   if (!fp8 && kv_dtype != in_dtype) return PA_ERR_UNSUPPORTED;
   const int sstride = scale_block_stride(kv_dtype, num_kv_heads);
-  if (head_size % 8 != 0) return PA_ERR_UNSUPPORTED;
-  if (num_tokens == 0) return PA_OK;
+  if (head_size % 8 != 0 || static_cast<int64_t>(num_kv_heads) * head_size > kMaxRowElems) return PA_ERR_UNSUPPORTED;
   const int row = num_kv_heads * head_size;
   const int threads = static_cast<int>(std::min<size_t>(256, round_up(static_cast<size_t>(ceil_div(row, 8)), 32)));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -290,8 +292,8 @@ pa_status pa_reshape_and_cache_layers(const void* const* keys, const void* const
   if (fp8 && (!k_scales || !v_scales || !aligned(k_scales, 8) || !aligned(v_scales, 8))) return PA_ERR_INVALID_ARGUMENT;
   if (!fp8 && kv_dtype != in_dtype) return PA_ERR_UNSUPPORTED;
   const int sstride = scale_block_stride(kv_dtype, num_kv_heads);
-  if (head_size % 8 != 0 || num_layers > 65535) return PA_ERR_UNSUPPORTED;
-  if (num_tokens == 0 || num_layers == 0) return PA_OK;
+  if (head_size % 8 != 0 || num_layers > 65535 || static_cast<int64_t>(num_kv_heads) * head_size > kMaxRowElems)
+    return PA_ERR_UNSUPPORTED;
   const int row = num_kv_heads * head_size;
   const int threads = static_cast<int>(std::min<size_t>(256, round_up(static_cast<size_t>(ceil_div(row, 8)), 32)));
   const dim3 grid(static_cast<unsigned>(num_tokens), static_cast<unsigned>(num_layers));

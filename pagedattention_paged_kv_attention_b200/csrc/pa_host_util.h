@@ -16,7 +16,8 @@ namespace pa_host {
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+// ceil(a / b) for a >= 0, b > 0, without forming a + b - 1 (which overflows near INT_MAX).
+inline int ceil_div(int a, int b) { return a / b + (a % b != 0); }
 inline bool is_16bit(pa_dtype t) { return t == PA_F16 || t == PA_BF16; }
 inline bool is_fp8(pa_dtype t) { return t == PA_FP8_E4M3 || t == PA_FP8_E4M3_BLOCK; }
 inline bool is_dtype(pa_dtype t) { return t == PA_F16 || t == PA_BF16 || is_fp8(t); }

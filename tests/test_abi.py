@@ -175,3 +175,22 @@ def test_binding_rejects_tensors_the_library_would_misread(P):
         P.swap_blocks(kc.transpose(1, 2), kc, kc, kc, torch.zeros((1, 2), dtype=torch.int64))
     with pytest.raises(ValueError, match="dtype"):
         P.swap_blocks(kc, kc, kc, kc, torch.zeros((1, 2), dtype=torch.int32))
+
+
+def test_sizes_near_int_max_do_not_wrap(P):
+    """Partition counts are computed without int overflow: the workspace for a maximum context length
+    of 2^31 - 1 is the layout's size for ceil((2^31 - 1) / ps) partitions."""
+    r256 = lambda x: -(-x // 256) * 256
+    for L, ps in ((2**31 - 1, 64), (2**31 - 64, 64), (2**31 - 1, 4096), (1025, 64)):
+        rows = 8 * -(-L // ps)
+        assert P.workspace_size(1, 8, 8, 128, L, ps) == 256 + 2 * r256(rows * 4) + r256(rows * 128 * 4), (L, ps)
+
+
+def test_cache_writes_reject_rows_beyond_int_indexing(P):
+    """Every call here is refused during validation, before any CUDA call (the pointers are dummies)."""
+    L = P.lib
+    args = lambda hkv, d: (16, 16, P.PA_BF16, 16, 16, P.PA_BF16, None, None, 16, 3, hkv, d, 16, 4, None)
+    assert L.pa_reshape_and_cache(*args((1 << 16) + 1, 256)) == P.PA_ERR_UNSUPPORTED  # 2^24 + 256 elements
+    assert L.pa_reshape_and_cache(*args(1 << 24, 1 << 10)) == P.PA_ERR_UNSUPPORTED  # product overflows int
+    assert L.pa_reshape_and_cache_layers(16, 16, P.PA_BF16, 16, 16, P.PA_BF16, None, None, 16, 3, 2, 1 << 24,
+                                         1 << 10, 16, 4, None) == P.PA_ERR_UNSUPPORTED
