@@ -403,7 +403,9 @@ int or_swap_blocks(void* dst_key_cache, void* dst_value_cache, const void* src_k
  * values. The chunk is the last n_s of those tokens (reading: a chunk continues the sequence), so
  * query j of the chunk sits at position p = L_s - n_s + j and attends to t = 0 .. p:
  *   z_t = scale * sum_i q[row][h][i] * k_t[i],  out[row][h][:] = sum_t exp(z_t - m) v_t / sum_t exp(z_t - m)
- * with m = max_t z_t, k_t and v_t found through block_tables[s] as in decode.
+ * with m = max_t z_t, k_t and v_t found through block_tables[s] as in decode, and dequantised as in
+ * decode for the FP8 formats (code x the kv head's scale, or x the scale of the token's physical
+ * block and kv head).
  * --------------------------------------------------------------------------------------------- */
 typedef struct {
   double* out;                 /* [T][H][d] */
@@ -431,13 +433,12 @@ static int prefill_one(const or_prefill_job* a, int s, int row, int h, double* z
   const int p = a->context_lens[s] - n + j; /* position of this query token */
   const size_t q_base = ((size_t)row * a->num_heads + h) * d;
   double* o = a->out + q_base;
-  const double ks = (a->kv_dtype == OR_E4M3) ? (double)a->k_scale[kvh] : 1.0;
-  const double vs = (a->kv_dtype == OR_E4M3) ? (double)a->v_scale[kvh] : 1.0;
   for (int i = 0; i < d; ++i) o[i] = 0.0;
   for (int t = 0; t <= p; ++t) {
     int blk = a->block_tables[(size_t)s * a->max_blocks_per_seq + t / a->block_size];
     if (blk < 0 || blk >= a->num_blocks) return OR_BAD_BLOCK;
     size_t k_base = (((size_t)blk * a->block_size + t % a->block_size) * a->num_kv_heads + kvh) * d;
+    const double ks = kv_scale(a->k_scale, a->kv_dtype, blk, a->num_kv_heads, kvh);
     double dot = 0.0;
     for (int i = 0; i < d; ++i)
       dot += element(a->query, a->q_dtype, q_base + i) * (element(a->key_cache, a->kv_dtype, k_base + i) * ks);
@@ -451,6 +452,7 @@ static int prefill_one(const or_prefill_job* a, int s, int row, int h, double* z
   for (int t = 0; t <= p; ++t) {
     int blk = a->block_tables[(size_t)s * a->max_blocks_per_seq + t / a->block_size];
     size_t v_base = (((size_t)blk * a->block_size + t % a->block_size) * a->num_kv_heads + kvh) * d;
+    const double vs = kv_scale(a->v_scale, a->kv_dtype, blk, a->num_kv_heads, kvh);
     double w = exp(z[t] - m) / denom;
     for (int i = 0; i < d; ++i) o[i] += w * (element(a->value_cache, a->kv_dtype, v_base + i) * vs);
   }
@@ -492,8 +494,9 @@ int or_paged_prefill(double* out, const void* query, int q_dtype, const void* ke
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads) return OR_BAD_ARG;
   if (head_size <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq < 0) return OR_BAD_ARG;
   if (q_dtype != OR_F16 && q_dtype != OR_BF16) return OR_BAD_ARG;
-  if (kv_dtype != OR_F16 && kv_dtype != OR_BF16 && kv_dtype != OR_E4M3) return OR_BAD_ARG;
-  if (kv_dtype == OR_E4M3 && (!k_scale || !v_scale)) return OR_BAD_ARG;
+  if (kv_dtype != OR_F16 && kv_dtype != OR_BF16 && kv_dtype != OR_E4M3 && kv_dtype != OR_E4M3_BLOCK)
+    return OR_BAD_ARG;
+  if ((kv_dtype == OR_E4M3 || kv_dtype == OR_E4M3_BLOCK) && (!k_scale || !v_scale)) return OR_BAD_ARG;
   if (q_start[0] != 0) return OR_BAD_ARG;
   for (int s = 0; s < num_seqs; ++s) {
     int n = q_start[s + 1] - q_start[s];

@@ -84,3 +84,16 @@ def random_paged_case(rng: np.random.Generator, lens, num_heads, num_kv_heads, h
     inputs = dict(query_bits=bits16(q), q_dtype=dtype, key_cache=kc, value_cache=vc, kv_dtype=dtype,
                   block_tables=tables, context_lens=np.array(lens, np.int32))
     return inputs, q.to(torch.float64), Ks, Vs
+
+
+def logical_fp8(codes, scales, tables, s, L, bs):
+    """This test-side gather and decode of an FP8 cache: [L, Hkv, d] float64 for sequence s, each code
+    decoded by torch's float8_e4m3fn and multiplied by its scale -- scales [Hkv] (per kv head) or
+    [num_blocks, Hkv] (per physical block and kv head)."""
+    rows = []
+    for t in range(L):
+        blk = tables[s, t // bs]
+        c = torch.from_numpy(codes[blk, t % bs].copy()).view(torch.float8_e4m3fn).to(torch.float64)
+        sc = scales[blk] if scales.ndim == 2 else scales
+        rows.append(c * torch.from_numpy(sc.astype(np.float64))[:, None])
+    return torch.stack(rows)

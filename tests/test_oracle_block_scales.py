@@ -18,7 +18,7 @@ import torch
 import torch.nn.functional as F
 
 import oracle
-from helpers import bits16, random_paged_case
+from helpers import bits16, logical_fp8, random_paged_case
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "pa_oracle.c")
 
@@ -33,16 +33,6 @@ def fp8_case(rng, lens, H, Hkv, d, bs):
     vc = oracle.quantize_e4m3_blocks(vb, "bf16", vs)
     inputs = dict(inputs, key_cache=kc, value_cache=vc, kv_dtype="fp8_e4m3_block", k_scale=ks, v_scale=vs)
     return inputs, q
-
-
-def logical_fp8(codes, scales, tables, s, L, bs):
-    """This test's own gather and decode: [L, Hkv, d] float64."""
-    rows = []
-    for t in range(L):
-        blk = tables[s, t // bs]
-        c = torch.from_numpy(codes[blk, t % bs].copy()).view(torch.float8_e4m3fn).to(torch.float64)
-        rows.append(c * torch.from_numpy(scales[blk].astype(np.float64))[:, None])
-    return torch.stack(rows)
 
 
 @pytest.mark.parametrize("H,Hkv,d,bs,lens", [(8, 2, 32, 8, [9, 40, 1]), (4, 4, 16, 16, [33, 16, 70])])

@@ -9,8 +9,12 @@
 * Block placement does not matter (a permuted pool and table give the same output).
 * Negative control: attention without the causal rule differs, and so does a mask aligned to the
   start of the context.
+* FP8 caches (per kv head and per (block, kv head) scales): equal to the same SDPA on K/V that this
+  test decodes itself (torch's float8 decode times the scale of the token's physical block), and
+  one-token chunks equal the decode oracle bit for bit.
 * Planted mistakes in a copy of the C source (off-by-one in the causal bound, the chunk placed at the
-  start of the context, the row index of the query) fail these pins.
+  start of the context, the row index of the query, a per-block scale read at the logical block, the
+  value scale taken from the keys') fail these pins.
 """
 import os
 import shutil
@@ -23,7 +27,7 @@ import torch
 import torch.nn.functional as F
 
 import oracle
-from helpers import bits16, random_paged_case
+from helpers import bits16, logical_fp8, random_paged_case
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "pa_oracle.c")
 
@@ -133,12 +137,65 @@ def test_negative_controls():
     assert np.max(np.abs(out[:16] - o[0].permute(1, 0, 2).numpy())) > 1e-3
 
 
+FP8_FORMATS = ["fp8_e4m3", "fp8_e4m3_block"]
+
+
+def fp8_chunk_case(rng, lens, qlens, H, Hkv, d, bs, fmt):
+    """Query chunks over an FP8 cache quantised by the oracle's encoder (itself pinned against torch's
+    float8 cast), with random scales per kv head or per (block, kv head)."""
+    inputs, q, _, _ = chunk_case(rng, lens, qlens, H, Hkv, d, bs)
+    NB = inputs["key_cache"].shape[0]
+    shape = (NB, Hkv) if fmt == "fp8_e4m3_block" else (Hkv,)
+    ks = rng.uniform(0.002, 0.02, shape).astype(np.float32)
+    vs = rng.uniform(0.002, 0.02, shape).astype(np.float32)
+    quant = oracle.quantize_e4m3_blocks if fmt == "fp8_e4m3_block" else oracle.quantize_e4m3
+    kc = quant(inputs["key_cache"], "bf16", ks)
+    vc = quant(inputs["value_cache"], "bf16", vs)
+    return dict(inputs, key_cache=kc, value_cache=vc, kv_dtype=fmt, k_scale=ks, v_scale=vs), q
+
+
+def fp8_sdpa_reference(inputs, q, lens, bs, scale, H, Hkv):
+    t = inputs["block_tables"]
+    Ks = [logical_fp8(inputs["key_cache"], inputs["k_scale"], t, s, L, bs) for s, L in enumerate(lens)]
+    Vs = [logical_fp8(inputs["value_cache"], inputs["v_scale"], t, s, L, bs) for s, L in enumerate(lens)]
+    return sdpa_causal_end_aligned(q, Ks, Vs, inputs["q_start"], scale, H, Hkv)
+
+
+@pytest.mark.parametrize("case", CASES[:3])
+@pytest.mark.parametrize("fmt", FP8_FORMATS)
+def test_fp8_caches_match_sdpa_on_self_decoded_kv(case, fmt):
+    bs, H, Hkv, d, lens, qlens = case
+    rng = np.random.default_rng(zlib.crc32(repr((case, fmt)).encode()))
+    inputs, q = fp8_chunk_case(rng, lens, qlens, H, Hkv, d, bs, fmt)
+    out = oracle.paged_prefill(scale=0.2, **inputs)
+    np.testing.assert_allclose(out, fp8_sdpa_reference(inputs, q, lens, bs, 0.2, H, Hkv), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("fmt", FP8_FORMATS)
+def test_fp8_one_token_chunks_equal_decode(fmt):
+    rng = np.random.default_rng(11)
+    inputs, _ = fp8_chunk_case(rng, [1, 9, 31, 64], [1] * 4, 8, 2, 32, 8, fmt)
+    pre = oracle.paged_prefill(scale=0.3, **inputs)
+    dec = oracle.paged_attention(scale=0.3, **{k: v for k, v in inputs.items() if k != "q_start"})
+    assert np.array_equal(pre, dec)
+
+
 MUTANTS = [
     ("causal_off_by_one", "for (int t = 0; t <= p; ++t) {\n    int blk = a->block_tables[(size_t)s * a->max_blocks_per_seq + t / a->block_size];\n    if (blk",
      "for (int t = 0; t < p; ++t) {\n    int blk = a->block_tables[(size_t)s * a->max_blocks_per_seq + t / a->block_size];\n    if (blk"),
     ("chunk_at_start", "const int p = a->context_lens[s] - n + j;", "const int p = j;"),
     ("query_row", "const size_t q_base = ((size_t)row * a->num_heads + h) * d;\n  double* o",
      "const size_t q_base = ((size_t)j * a->num_heads + h) * d;\n  double* o"),
+    ("block_scale_logical_index",
+     "t % a->block_size) * a->num_kv_heads + kvh) * d;\n"
+     "    const double ks = kv_scale(a->k_scale, a->kv_dtype, blk, a->num_kv_heads, kvh);",
+     "t % a->block_size) * a->num_kv_heads + kvh) * d;\n"
+     "    const double ks = kv_scale(a->k_scale, a->kv_dtype, t / a->block_size, a->num_kv_heads, kvh);"),
+    ("value_scale_from_keys",
+     "t % a->block_size) * a->num_kv_heads + kvh) * d;\n"
+     "    const double vs = kv_scale(a->v_scale, a->kv_dtype, blk, a->num_kv_heads, kvh);",
+     "t % a->block_size) * a->num_kv_heads + kvh) * d;\n"
+     "    const double vs = kv_scale(a->k_scale, a->kv_dtype, blk, a->num_kv_heads, kvh);"),
 ]
 
 
@@ -161,6 +218,14 @@ def test_planted_mistakes_fail_the_pins(tmp_path, name, old, new):
                 out = oracle.paged_prefill(scale=0.2, **inputs)
                 if not np.allclose(out, sdpa_causal_end_aligned(q, Ks, Vs, inputs["q_start"], 0.2, H, Hkv),
                                    rtol=0, atol=1e-12):
+                    failures += 1
+            except Exception:
+                failures += 1
+            rng = np.random.default_rng(zlib.crc32(repr((case, "fp8_e4m3_block")).encode()))
+            inputs, q = fp8_chunk_case(rng, lens, qlens, H, Hkv, d, bs, "fp8_e4m3_block")
+            try:
+                out = oracle.paged_prefill(scale=0.2, **inputs)
+                if not np.allclose(out, fp8_sdpa_reference(inputs, q, lens, bs, 0.2, H, Hkv), rtol=0, atol=1e-12):
                     failures += 1
             except Exception:
                 failures += 1

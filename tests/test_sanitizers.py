@@ -3,7 +3,7 @@
 The C oracle and the native block manager (plain C++, no CUDA) are rebuilt with
 -fsanitize=address,undefined in a temporary directory and driven from a child Python process with the
 ASan runtime preloaded: every oracle operation on small ragged cases (decode attention in all cache
-formats, prefill, reshape_and_cache, copy_blocks, swap_blocks, the codecs), and a seeded block-manager
+formats, prefill over 16-bit and per-block FP8 caches, reshape_and_cache, copy_blocks, swap_blocks, the codecs), and a seeded block-manager
 session checked call by call against the manager's oracle. Any out-of-bounds access, use after free or
 undefined behaviour aborts the child.
 """
@@ -41,6 +41,12 @@ CHILD = textwrap.dedent(r'''
         qp = bits16(torch.randn(20, 4, 16).to(torch.bfloat16))
         oracle.paged_prefill(qp, "bf16", inputs["key_cache"], inputs["value_cache"], "bf16", inputs["block_tables"],
                              inputs["context_lens"], np.array([0, 10, 20], np.int32), 0.3)
+        NBp = inputs["key_cache"].shape[0]
+        bsc = np.full((NBp, 2), 0.01, np.float32)
+        oracle.paged_prefill(qp, "bf16", oracle.quantize_e4m3_blocks(inputs["key_cache"], "bf16", bsc),
+                             oracle.quantize_e4m3_blocks(inputs["value_cache"], "bf16", bsc), "fp8_e4m3_block",
+                             inputs["block_tables"], inputs["context_lens"], np.array([0, 10, 20], np.int32), 0.3,
+                             k_scale=bsc, v_scale=bsc)
         kc = inputs["key_cache"].copy(); vc = inputs["value_cache"].copy()
         NB = kc.shape[0]
         x = bits16(torch.randn(5, 2, 16).to(torch.bfloat16))
