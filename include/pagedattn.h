@@ -17,11 +17,16 @@
  *
  * Conventions for every entry point
  *  - Ownership: the caller allocates every buffer (the block pool is preallocated, [T] sec. 3.2). The
- *    library allocates nothing, keeps no per-call state and never frees caller memory.
+ *    library calls no allocator, keeps no per-call state and never frees caller memory; its one fixed
+ *    device array (PA_STATIC_WORKSPACE_BYTES) serves pa_paged_attention_static only.
  *  - Pointers are DEVICE pointers unless a parameter says "host". Every device pointer must be 16-byte
  *    aligned. Tensors are dense, row-major, in the layouts given below.
  *  - Asynchrony: each call validates its arguments on the host, enqueues its kernels on `stream` and
- *    returns without synchronising ([T] sec. 3.2). A NULL stream is the legacy default stream.
+ *    returns without synchronising ([T] sec. 3.2). A NULL stream is the legacy default stream. The
+ *    kernels of pa_copy_blocks, pa_reshape_and_cache and pa_paged_attention are launched with
+ *    programmatic stream serialisation: one may be scheduled while the previous kernel in the stream
+ *    finishes, but it waits for that kernel's completion and memory before its first global access,
+ *    so every memory effect keeps stream order.
  *  - Errors: invalid arguments are reported before anything is enqueued (nothing runs, no CUDA call is
  *    made). Launch failures return PA_ERR_CUDA. The library never aborts, never throws across the ABI
  *    and its kernels never trap; contract violations that only the device can see (a block id
