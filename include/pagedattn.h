@@ -23,7 +23,7 @@
  *    aligned. Tensors are dense, row-major, in the layouts given below.
  *  - Asynchrony: each call validates its arguments on the host, enqueues its kernels on `stream` and
  *    returns without synchronising ([T] sec. 3.2). A NULL stream is the legacy default stream. The
- *    kernels of pa_copy_blocks, pa_reshape_and_cache and pa_paged_attention are launched with
+ *    kernels of pa_copy_blocks, pa_reshape_and_cache and pa_paged_attention(_static) are launched with
  *    programmatic stream serialisation: one may be scheduled while the previous kernel in the stream
  *    finishes, but it waits for that kernel's completion and memory before its first global access,
  *    so every memory effect keeps stream order.
