@@ -28,7 +28,9 @@
  * are a stack that starts as 0, 1, 2, ... from the top; a released block goes back on top. Within
  * one call, sequences are served in the order given and a released table is walked front to back.
  *
- * Every call either completes or returns an error and leaves the manager unchanged. Sequence ids are
+ * Every call either completes or returns an error and leaves the manager unchanged; that includes a
+ * failed host allocation, which returns PA_ERR_HOST_MEMORY (no C++ exception crosses the ABI). A call
+ * performs its allocations before its first change. Sequence ids are
  * any int64 >= 0 chosen by the caller; PA_BM_NO_SEQUENCE (-1) means "none". All arrays are HOST
  * memory owned by the caller (pinned memory works and lets the outputs go straight to the device).
  * A manager may be used from several threads: calls are serialised by a lock inside it.

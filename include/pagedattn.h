@@ -69,7 +69,8 @@ typedef enum pa_status {
   PA_ERR_UNSUPPORTED = 2,               /* valid but outside the supported set above */
   PA_ERR_WORKSPACE_TOO_SMALL = 3,       /* workspace_bytes < pa_paged_attention_workspace_size(...) */
   PA_ERR_CUDA = 4,                      /* a CUDA runtime/driver call or a launch failed */
-  PA_ERR_OUT_OF_BLOCKS = 5              /* block manager: the pool has too few free blocks (no change) */
+  PA_ERR_OUT_OF_BLOCKS = 5,             /* block manager: the pool has too few free blocks (no change) */
+  PA_ERR_HOST_MEMORY = 6                /* block manager: a host allocation failed (no change) */
 } pa_status;
 
 typedef enum pa_dtype {

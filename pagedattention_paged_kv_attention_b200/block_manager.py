@@ -48,6 +48,7 @@ class BlockManager:
     blocks for swapping."""
 
     def __init__(self, num_blocks: int, block_size: int, num_host_blocks: int = 0):
+        self._h = None                    # set before the call, so a failed create still closes cleanly
         h = ctypes.c_void_p()
         _call(lib.pa_bm_create(num_blocks, block_size, num_host_blocks, ctypes.byref(h)), "pa_bm_create")
         self._h = h

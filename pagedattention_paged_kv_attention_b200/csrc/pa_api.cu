@@ -119,6 +119,7 @@ const char* pa_status_string(pa_status status) {
     case PA_ERR_WORKSPACE_TOO_SMALL: return "PA_ERR_WORKSPACE_TOO_SMALL: workspace smaller than pa_paged_attention_workspace_size()";
     case PA_ERR_CUDA: return "PA_ERR_CUDA: a CUDA call or kernel launch failed";
     case PA_ERR_OUT_OF_BLOCKS: return "PA_ERR_OUT_OF_BLOCKS: too few free blocks in the pool (state unchanged)";
+    case PA_ERR_HOST_MEMORY: return "PA_ERR_HOST_MEMORY: a host memory allocation failed (state unchanged)";
   }
   return "unknown pa_status";
 }

@@ -14,7 +14,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIBRARY_PATH = os.path.join(_HERE, "libpagedattn.so")
 
-PA_OK, PA_ERR_INVALID_ARGUMENT, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL, PA_ERR_CUDA, PA_ERR_OUT_OF_BLOCKS = range(6)
+(PA_OK, PA_ERR_INVALID_ARGUMENT, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL, PA_ERR_CUDA, PA_ERR_OUT_OF_BLOCKS,
+ PA_ERR_HOST_MEMORY) = range(7)
 PA_F16, PA_BF16, PA_FP8_E4M3, PA_FP8_E4M3_BLOCK = 0, 1, 2, 3
 PA_DEVERR_BLOCK_ID, PA_DEVERR_CONTEXT_LEN, PA_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 WORKSPACE_HEADER_BYTES = 256
