@@ -164,46 +164,19 @@ def reduce_sum(x, world, device):
 
 
 def run_reference(args, cfg, world, rank):
-    """The CPU oracle timed on the machine's host cores (rank 0 only)."""
+    """The CPU oracle timed on the machine's host cores (rank 0 only): --warmup untimed passes, then
+    --steps timed passes over the same deterministic sample as the GPU arm's cpu_baseline leg."""
     if rank != 0:
         return
-    import oracle
-    import dataclasses
-    cfg = dataclasses.replace(cfg, num_blocks=None)  # the sample's pool: 1.2x its blocks (placement only)
-    # pick a sample of sequences so that one step takes about 1 s
-    n, dt = 1, 0.0
-    while True:
-        w = W.make_workload(cfg, seed=cfg.seed, num_seqs=n, prefilled=True)
-        inp = oracle_inputs(cfg, w)
-        t0 = time.perf_counter()
-        oracle.paged_attention(**inp)
-        dt = time.perf_counter() - t0
-        if dt >= 0.5 or n >= cfg.num_seqs:
-            break
-        n = min(cfg.num_seqs, max(n * 2, int(n * 1.0 / max(dt, 1e-3))))
-    kv = W.ideal_bytes(w.context_lens.numpy(), cfg.num_kv_heads, cfg.head_size,
-                       1 if cfg.kv_dtype.startswith("fp8") else 2, cfg.block_size,
-                       cfg.num_heads, 2)["kv"]
-    for _ in range(args.warmup):
-        oracle.paged_attention(**inp)
-    times = []
-    for _ in range(args.steps):
-        t0 = time.perf_counter()
-        oracle.paged_attention(**inp)
-        times.append(time.perf_counter() - t0)
-    t = float(np.mean(times))
-    value = kv / t / 1e9
-    sample = (f"{n} of {cfg.num_seqs} sequences of the workload ({int(w.context_lens.sum())} context tokens), "
-              f"fp64 oracle, one step = one pass over the sample")
-    cores = oracle.default_threads()
-    line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "impl": "reference", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg.description, "name": cfg.name, "num_seqs_sampled": n},
-            "tokens_per_s": round(n / t, 3),
-            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                             "sample": sample},
-            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    rec = oracle_decode_timing(cfg, passes=args.steps, warmup=args.warmup)
+    lens = decode_lengths(cfg, cfg.seed)
+    line = {"metric": METRIC, "value": rec["value"], "unit": "GB/s", "impl": "reference", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(rec["pass_s"]["median"] * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": decode_config(cfg, lens, world),
+            "tokens_per_s": rec["tokens_per_s"],
+            "cpu_baseline": rec,
+            "e2e": {"value": rec["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
@@ -213,9 +186,10 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--op", default="decode", choices=["decode", "prefill", "swap", "layers", "plan"],
+    ap.add_argument("--op", default="decode", choices=["decode", "prefill", "swap", "layers", "plan", "trace"],
                     help="decode: the decode step (default); prefill: the causal prefill step; swap: swap_blocks "
-                         "host<->device; layers: multi-layer cache ops; plan: the block manager's decode plan")
+                         "host<->device; layers: multi-layer cache ops; plan: the block manager's decode plan; "
+                         "trace: per-CTA and per-item timing of the decode kernel (trace build)")
     ap.add_argument("--workload", default=None, choices=list(W.CONFIGS) + list(W.PREFILL_CONFIGS),
                     help="default: 7b (decode ops), prefill_7b (--op prefill)")
     ap.add_argument("--partition-size", type=int, default=None,
@@ -225,7 +199,9 @@ def main():
                     help="smaller batch of the same workload (profiling cases); default: the workload's")
     ap.add_argument("--pool-blocks", type=int, default=None,
                     help="override the pool size in blocks (profiling cases that must stay small)")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=8.0)
+    ap.add_argument("--no-extra-configs", action="store_true",
+                    help="time only --workload (by default the 7B line also carries a 70B-GQA sub-record)")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     if args.workload is None:
@@ -240,13 +216,11 @@ def main():
     if args.pool_blocks is not None:
         import dataclasses
         cfg = dataclasses.replace(cfg, num_blocks=args.pool_blocks)
-    if args.partition_size is None:
-        args.partition_size = cfg.partition_size
     world, rank, local = dist_setup(args)
 
-    if args.op in ("swap", "layers", "plan"):
+    if args.op in ("swap", "layers", "plan", "trace"):
         if rank == 0:
-            {"swap": run_swap, "layers": run_layers, "plan": run_plan}[args.op](args, cfg)
+            {"swap": run_swap, "layers": run_layers, "plan": run_plan, "trace": run_trace}[args.op](args, cfg)
         if world > 1:
             torch.distributed.destroy_process_group()
         return
@@ -260,6 +234,75 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    peaks = measured_peaks()
+    peak = peaks["hbm_gbs"] if peaks else 6650.0
+    rec = measure_decode(args, cfg, P, dev, rank, world, peak, peaks is not None, checks=True)
+    extra = {}
+    if (args.workload == "7b" and not args.no_extra_configs and args.num_seqs is None and args.pool_blocks is None
+            and args.partition_size is None):
+        # The second configuration the bandwidth target names, in the same run and process.
+        extra["70b_gqa"] = measure_decode(args, W.CONFIGS["70b_gqa"], P, dev, rank, world, peak, peaks is not None,
+                                          checks=False)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": rec["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f16",
+            "data": "synthetic",
+            "config": decode_config(cfg, decode_lengths(cfg, cfg.seed)[:args.num_seqs or cfg.num_seqs], world),
+        }
+        line.update({k: v for k, v in rec.items() if k not in ("value", "ms_per_step")})
+        if extra:
+            line["configs"] = {name: {k: v for k, v in r.items() if k not in ("gpu_launches",)}
+                               for name, r in extra.items()}
+            for name, r in extra.items():
+                line["configs"][name]["config"] = decode_config(W.CONFIGS[name], decode_lengths(W.CONFIGS[name],
+                                                                W.CONFIGS[name].seed), world)
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_decode_timing(cfg, seconds=args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def timed_launches(fn, reps=10, warmup=3):
+    """Median CUDA-event time (ms) of one call of fn on the current stream."""
+    for _ in range(warmup):
+        fn()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    torch.cuda.synchronize()
+    for a, b in evs:
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return float(np.median([a.elapsed_time(b) for a, b in evs]))
+
+
+def read_ceilings(P, dev, key_cache, value_cache, block_tables, context_lens, kv_bytes):
+    """Read-only ceilings measured in this process (include/pa_probe.h): a sequential stream over 2 GiB
+    (HBM), the same 16-byte loads over the batch's own K/V rows through its block table (no compute),
+    and a 32 MiB buffer read 64 times over (L2)."""
+    sink = torch.zeros(1, dtype=torch.int64, device=dev)
+    big = torch.empty(2 << 30, dtype=torch.uint8, device=dev)
+    t_stream = timed_launches(lambda: P.probe_stream_read(big, 1, sink))
+    del big
+    small = torch.empty(32 << 20, dtype=torch.uint8, device=dev)
+    t_l2 = timed_launches(lambda: P.probe_stream_read(small, 64, sink))
+    del small
+    t_paged = timed_launches(lambda: P.probe_paged_read(key_cache, value_cache, block_tables, context_lens, sink))
+    return {"hbm_read_stream_gbs": round((2 << 30) / (t_stream * 1e-3) / 1e9, 1),
+            "paged_read_gbs": round(kv_bytes / (t_paged * 1e-3) / 1e9, 1),
+            "l2_read_gbs": round(64 * (32 << 20) / (t_l2 * 1e-3) / 1e9, 1),
+            "method": "pa_probe_stream_read over 2 GiB once (HBM) and over 32 MiB 64 times (L2); "
+                      "pa_probe_paged_read over this batch's valid K/V rows; median of 10 event-timed launches"}
+
+
+def measure_decode(args, cfg, P, dev, rank, world, peak, peak_measured, checks):
+    """One workload's decode step timed on the device (K steps after W warm-ups, back to back), through
+    the public API end to end, and with its roofline; with checks, also the read ceilings and an L2-flush
+    check of the attention call."""
     w = W.make_workload(cfg, seed=cfg.seed + 1000 * rank, device=dev, num_seqs=args.num_seqs)
     S, H, d = w.query.shape
     kv_bytes = 1 if cfg.kv_dtype.startswith("fp8") else 2
@@ -275,12 +318,14 @@ def main():
         P.reshape_and_cache(key_cache.view(NB * bs, Hkv, d), value_cache.view(NB * bs, Hkv, d), kq, vq, slots, ks, vs)
         key_cache, value_cache = kq, vq
         del slots
+        w.key_values = w.value_values = None
     lens = w.context_lens.cpu().numpy()
     mcl = int(lens.max())
     ideal = W.ideal_bytes(lens, cfg.num_kv_heads, d, kv_bytes, cfg.block_size, H, 2)
-    ps = P.partition_size(S, H, cfg.num_kv_heads, mcl, args.partition_size)
+    part_req = args.partition_size if args.partition_size is not None else cfg.partition_size
+    ps = P.partition_size(S, H, cfg.num_kv_heads, mcl, part_req)
     parts = max(1, -(-mcl // ps))
-    ws = P.make_workspace(S, H, cfg.num_kv_heads, d, mcl, args.partition_size, device=dev)
+    ws = P.make_workspace(S, H, cfg.num_kv_heads, d, mcl, part_req, device=dev)
     out = torch.empty_like(w.query)
     stream = torch.cuda.current_stream(dev)
 
@@ -291,14 +336,14 @@ def main():
         if ev is not None:
             ev[0].record(stream)
         P.paged_attention(o, q, key_cache, value_cache, tables, clens, cfg.softmax_scale, mcl, ws, ks, vs,
-                          partition_size=args.partition_size)
+                          partition_size=part_req)
         if ev is not None:
             ev[1].record(stream)
 
     inputs = (w.query, w.new_key, w.new_value, w.slot_mapping, w.block_tables, w.context_lens)
     launches_per_step = 2 + (1 if parts > 1 else 0) + (1 if w.cow_mapping.shape[0] else 0)
 
-    # ---- device-resident timing ----
+    # ---- device-resident timing: K steps back to back (the K/V read per step is larger than L2) ----
     for _ in range(args.warmup):
         step(*inputs, out)
     kernel_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -381,44 +426,52 @@ def main():
     e2e_ms = reduce_max(e0.elapsed_time(e1) / args.steps, world, dev)
     e2e_value = total_kv / (e2e_ms * 1e-3) / 1e9
 
+    achieved = ideal["total"] / (attn_ms * 1e-3) / 1e9
+    rec = {
+        "value": round(value, 2), "ms_per_step": round(max_step_ms, 4),
+        "plan": {"partition_size": ps, "partitions": parts, "num_seqs": S},
+        "tokens_per_s": round(total_seqs / (max_step_ms * 1e-3), 1),
+        "pct_of_measured_hbm_peak": round(100 * value / peak, 2),
+        "pct_of_8tbs": round(100 * value / 8000.0, 2),
+        "roofline": {"kernel": "paged_attention (pa_paged_attention call: main kernel%s)" %
+                     (" + split-K reduce" if parts > 1 else ""),
+                     "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_source": "measured" if peak_measured else "fallback",
+                     "algorithmic_bytes_per_launch": ideal["total"], "avg_launch_ms": round(attn_ms, 4),
+                     "traffic": recorded_traffic(cfg.name)},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
+                "copies": "one packed pinned upload per step (overlapping the previous step's kernels) "
+                          "and the output read back on its own stream, all inside the timed region"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    del dev_packed, views, outs, host_out, host_packed
     if rank == 0:
-        peaks = measured_peaks()
-        peak = peaks["hbm_gbs"] if peaks else 6650.0
-        achieved = ideal["total"] / (attn_ms * 1e-3) / 1e9
-        workload = cfg.name
-        line = {
-            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(max_step_ms, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f16",
-            "data": "synthetic",
-            "config": {"workload": cfg.description, "name": cfg.name, "num_seqs": S, "num_heads": H,
-                       "num_kv_heads": cfg.num_kv_heads, "head_size": d, "block_size": cfg.block_size,
-                       "kv_dtype": cfg.kv_dtype, "context_tokens": int(lens.sum()), "max_context_len": mcl,
-                       "partition_size": ps, "partitions": parts, "seed": cfg.seed,
-                       "l2": "inputs larger than L2: %.2f GB of K/V read per step vs 126 MB L2" % (ideal["kv"] / 1e9),
-                       "parallelism": f"dp{world} (independent sequence batches)"},
-            "tokens_per_s": round(total_seqs / (max_step_ms * 1e-3), 1),
-            "pct_of_measured_hbm_peak": round(100 * value / peak, 2),
-            "pct_of_8tbs": round(100 * value / 8000.0, 2),
-            "roofline": {"kernel": "paged_attention (pa_paged_attention call: main kernel%s)" %
-                         (" + split-K reduce" if parts > 1 else ""),
-                         "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "peak_source": "measured" if peaks else "fallback",
-                         "algorithmic_bytes_per_launch": ideal["total"], "avg_launch_ms": round(attn_ms, 4),
-                         "traffic": recorded_traffic(workload)},
-            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
-                    "copies": "one packed pinned upload per step (overlapping the previous step's kernels) "
-                              "and the output read back on its own stream, all inside the timed region"},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks.summary(),
-        }
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_seconds)
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
+        # Read ceilings in this process, and the attention call's fraction of each.
+        ceil = read_ceilings(P, dev, key_cache, value_cache, w.block_tables, w.context_lens, ideal["kv"])
+        rec["ceilings"] = ceil
+        rec["roofline"]["frac_of_read_stream"] = round(achieved / ceil["hbm_read_stream_gbs"], 4)
+        rec["roofline"]["frac_of_paged_read"] = round(achieved / ceil["paged_read_gbs"], 4)
+        if checks:
+            # L2 flush check: the same attention call with L2 flushed (a write of twice the L2 size)
+            # before each step, per-step event timing; against the back-to-back figure above.
+            l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+            flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for i in range(args.steps):
+                flush.fill_(i & 0xFF)
+                step(*inputs, out, evs[i])
+            torch.cuda.synchronize()
+            flushed_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+            rec["l2_flush_check"] = {"flush_bytes": 2 * l2, "attn_ms_flushed": round(flushed_ms, 4),
+                                     "attn_ms_back_to_back": round(attn_ms, 4),
+                                     "back_to_back_over_flushed": round(flushed_ms / attn_ms, 4)}
+            del flush
+    del key_cache, value_cache, w
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_prefill(args, cfg, world, rank):
@@ -602,6 +655,79 @@ def run_prefill_reference(args, cfg, world, rank):
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.default_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+TRACE_CTA_BASE, TRACE_MAX_CTAS = 8, 1024   # word offsets of the trace build's records (pa_attention.cuh)
+
+
+def run_trace(args, cfg):
+    """Where the decode kernel's time goes at the end of a launch. Builds the PA_TRACE variant of the
+    library (same kernels; they also stamp %globaltimer into the workspace), runs the workload's decode
+    step, and summarises one launch: per-CTA start/end, per-item start/finish, the split-K reduce's
+    span; idle SM time after each CTA's last item, and in the last 10% of the launch."""
+    from pagedattention_paged_kv_attention_b200 import build as B
+    lib = B.build(defines=["PA_TRACE"], output=os.path.join(os.path.dirname(B.LIBRARY), "libpagedattn_trace.so"))
+    os.environ["PA_LIBRARY_PATH"] = lib
+    from pagedattention_paged_kv_attention_b200 import pagedattn as P
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = W.make_workload(cfg, seed=cfg.seed, device=dev, num_seqs=args.num_seqs)
+    assert not cfg.kv_dtype.startswith("fp8"), "trace op: 16-bit caches"
+    S, H, d = w.query.shape
+    lens = w.context_lens.cpu().numpy()
+    mcl = int(lens.max())
+    part_req = args.partition_size if args.partition_size is not None else cfg.partition_size
+    ps = P.partition_size(S, H, cfg.num_kv_heads, mcl, part_req)
+    parts = max(1, -(-mcl // ps))
+    ws = P.make_workspace(S, H, cfg.num_kv_heads, d, mcl, part_req, device=dev)
+    nbytes = ws.numel() * ws.element_size()
+    g_tile = 1
+    while g_tile < H // cfg.num_kv_heads and g_tile < 8:
+        g_tile *= 2
+    items = parts * S * (-(-cfg.num_kv_heads // 8)) * (-(-(H // cfg.num_kv_heads) // g_tile))
+    trace_words = 8 + 4 * TRACE_MAX_CTAS + 4 * items
+    trace = ws.view(torch.uint8)[nbytes - ((trace_words * 8 + 255) // 256 * 256):].view(torch.int64)
+    out = torch.empty_like(w.query)
+    summaries = []
+    for rep in range(args.warmup + args.steps):
+        trace.zero_()
+        P.reshape_and_cache(w.new_key, w.new_value, w.key_values, w.value_values, w.slot_mapping)
+        P.paged_attention(out, w.query, w.key_values, w.value_values, w.block_tables, w.context_lens,
+                          cfg.softmax_scale, mcl, ws, partition_size=part_req)
+        torch.cuda.synchronize()
+        if rep < args.warmup:
+            continue
+        t = trace.cpu().numpy().view(np.uint64).astype(np.float64)
+        cta = t[TRACE_CTA_BASE:TRACE_CTA_BASE + 4 * TRACE_MAX_CTAS].reshape(-1, 4)
+        cta = cta[cta[:, 0] > 0]
+        it = t[TRACE_CTA_BASE + 4 * TRACE_MAX_CTAS:].reshape(-1, 4)[:items]
+        it = it[it[:, 0] > 0]
+        t0, t_end = cta[:, 0].min(), cta[:, 1].max()
+        span = t_end - t0
+        ends = cta[:, 1]
+        win = t_end - 0.1 * span
+        busy_last10 = np.clip(ends - win, 0, None).sum() / (len(cta) * 0.1 * span)
+        red_start = (2 ** 64 - 1) - t[0] if parts > 1 and t[0] > 0 else None
+        summaries.append({
+            "span_us": span / 1e3, "ctas": int(len(cta)), "items": int(len(it)),
+            "cta_start_spread_us": (cta[:, 0].max() - t0) / 1e3,
+            "cta_end_before_last_us": {q: float(np.percentile(t_end - ends, q)) / 1e3 for q in (10, 50, 90, 100)},
+            "idle_after_last_item_frac": float((t_end - ends).sum() / (len(cta) * span)),
+            "idle_in_last_10pct_frac": float(1 - busy_last10),
+            "last_item_start_before_end_us": float((t_end - it[:, 0].max()) / 1e3),
+            "item_us": {q: float(np.percentile(it[:, 1] - it[:, 0], q)) / 1e3 for q in (10, 50, 90, 100)},
+            "item_tokens": {q: float(np.percentile(it[:, 3], q)) for q in (10, 50, 90, 100)},
+            "reduce_start_after_main_end_us": None if red_start is None else float((red_start - t_end) / 1e3),
+            "reduce_span_us": None if red_start is None else float((t[1] - red_start) / 1e3),
+        })
+    med = lambda key: float(np.median([x[key] for x in summaries]))
+    line = {"metric": "decode kernel timeline (trace build)", "impl": "ours", "unit": "us", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "value": round(med("span_us"), 2),
+            "config": {"workload": cfg.description, "name": cfg.name, "num_seqs": S, "partition_size": ps,
+                       "partitions": parts, "items": items},
+            "median": {k: round(med(k), 4) for k in ("span_us", "idle_after_last_item_frac",
+                                                     "idle_in_last_10pct_frac", "last_item_start_before_end_us")},
+            "launches": summaries}
     print(json.dumps(line), flush=True)
 
 
@@ -801,35 +927,112 @@ def oracle_inputs(cfg, w):
                 scale=cfg.softmax_scale, k_scale=ks, v_scale=vs)
 
 
-def cpu_baseline(cfg, seconds):
-    """The oracle (as it stands) on a bounded sample of the same workload, on the host cores."""
+def host_cores():
+    """Host CPU facts behind the oracle figures: logical CPUs, the CPUs this process may run on, and the
+    cgroup CPU quota when one is set."""
+    info = {"cpu_count": os.cpu_count()}
+    try:
+        info["affinity"] = len(os.sched_getaffinity(0))
+    except AttributeError:
+        info["affinity"] = os.cpu_count()
+    try:
+        quota, period = open("/sys/fs/cgroup/cpu.max").read().split()[:2]
+        info["cgroup_quota_cpus"] = None if quota == "max" else round(int(quota) / int(period), 2)
+    except (OSError, ValueError):
+        info["cgroup_quota_cpus"] = None
+    return info
+
+
+def oracle_threads():
+    """Threads for the all-core oracle figure: the CPUs this process may use (and no more than the
+    cgroup quota allows)."""
+    h = host_cores()
+    n = h["affinity"] or 1
+    if h["cgroup_quota_cpus"]:
+        n = min(n, max(1, int(h["cgroup_quota_cpus"])))
+    return n
+
+
+ORACLE_ALL_CORE_GFLOP = 2.0    # work of one all-core oracle pass (about a second on 16 cores)
+ORACLE_ONE_CORE_GFLOP = 0.15   # work of one single-thread pass
+
+
+def decode_lengths(cfg, seed):
+    """The batch's context lengths, as make_workload draws them (no values are generated)."""
+    return W._lengths(cfg, np.random.default_rng(W.sub_seeds(seed)[0]), cfg.num_seqs)
+
+
+def decode_config(cfg, lens, world):
+    """The workload's description in the JSON line; both arms print the same one."""
+    kv = W.ideal_bytes(lens, cfg.num_kv_heads, cfg.head_size, 1 if cfg.kv_dtype.startswith("fp8") else 2,
+                       cfg.block_size, cfg.num_heads, 2)["kv"]
+    return {"workload": cfg.description, "name": cfg.name, "num_seqs": len(lens), "num_heads": cfg.num_heads,
+            "num_kv_heads": cfg.num_kv_heads, "head_size": cfg.head_size, "block_size": cfg.block_size,
+            "kv_dtype": cfg.kv_dtype, "context_tokens": int(np.sum(lens)), "max_context_len": int(np.max(lens)),
+            "seed": cfg.seed,
+            "l2": "inputs larger than L2: %.2f GB of K/V read per step vs 126 MB L2" % (kv / 1e9),
+            "parallelism": f"dp{world} (independent sequence batches)"}
+
+
+def first_sequences(cfg, lens, gflop):
+    """How many leading sequences of the batch fit in `gflop` of attention work (at least one)."""
+    work = np.cumsum(np.asarray(lens, dtype=np.float64) * cfg.num_heads * 4 * cfg.head_size)
+    return int(max(1, min(len(lens), np.searchsorted(work, gflop * 1e9, side="right"))))
+
+
+def time_passes(fn, passes, warmup):
+    for _ in range(warmup):
+        fn()
+    times = []
+    for _ in range(passes):
+        t0 = time.perf_counter()
+        fn()
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+def oracle_decode_timing(cfg, passes=None, warmup=1, seconds=8.0):
+    """The oracle, as it stands, on a deterministic sample of the decode workload: the first sequences
+    of the batch (seed cfg.seed) that fit in ORACLE_ALL_CORE_GFLOP, on all usable host cores; and the
+    first ones that fit in ORACLE_ONE_CORE_GFLOP on one thread. Each figure is the K/V bytes of its
+    sample over the median pass time. passes=None fills about `seconds` with passes (at least 3)."""
     import dataclasses
     import oracle
-    cfg = dataclasses.replace(cfg, num_blocks=None)  # the sample's pool: 1.2x its blocks (placement only)
-    n = 1
-    while True:
-        w = W.make_workload(cfg, seed=cfg.seed, num_seqs=n, prefilled=True)
+    threads = oracle_threads()
+    lens = decode_lengths(cfg, cfg.seed)
+    cfg_s = dataclasses.replace(cfg, num_blocks=None)   # the sample's pool: 1.2x its blocks (placement only)
+    kv_elem = 1 if cfg.kv_dtype.startswith("fp8") else 2
+
+    def case(n, nthreads):
+        w = W.make_workload(cfg_s, seed=cfg.seed, num_seqs=n, prefilled=True)
         inp = oracle_inputs(cfg, w)
+        kv = W.ideal_bytes(w.context_lens.numpy(), cfg.num_kv_heads, cfg.head_size, kv_elem, cfg.block_size,
+                           cfg.num_heads, 2)["kv"]
+        return (lambda: oracle.paged_attention(**inp, num_threads=nthreads)), kv, int(w.context_lens.sum())
+
+    n_all = first_sequences(cfg, lens, ORACLE_ALL_CORE_GFLOP)
+    fn, kv, tokens = case(n_all, threads)
+    if passes is None:
         t0 = time.perf_counter()
-        oracle.paged_attention(**inp)
-        dt = time.perf_counter() - t0
-        if dt >= seconds / 3 or n >= cfg.num_seqs:
-            break
-        n = min(cfg.num_seqs, max(n * 2, int(n * seconds / 3 / max(dt, 1e-3))))
-    reps, total = 0, 0.0
-    while total < seconds * 2 / 3 or reps == 0:
-        t0 = time.perf_counter()
-        oracle.paged_attention(**inp)
-        total += time.perf_counter() - t0
-        reps += 1
-    t = total / reps
-    kv = W.ideal_bytes(w.context_lens.numpy(), cfg.num_kv_heads, cfg.head_size,
-                       1 if cfg.kv_dtype.startswith("fp8") else 2, cfg.block_size,
-                       cfg.num_heads, 2)["kv"]
-    return {"value": round(kv / t / 1e9, 4), "unit": "GB/s", "cores": oracle.default_threads(), "kind": "oracle",
-            "sample": f"{n} of {cfg.num_seqs} sequences ({int(w.context_lens.sum())} context tokens), "
-                      f"{reps} timed passes of {t:.2f} s, fp64",
-            "tokens_per_s": round(n / t, 3)}
+        fn()
+        passes = max(3, int(seconds / max(time.perf_counter() - t0, 1e-3)))
+        warmup = max(0, warmup - 1)
+    times = time_passes(fn, passes, warmup)
+    t = float(np.median(times))
+    n_one = first_sequences(cfg, lens, ORACLE_ONE_CORE_GFLOP)
+    fn1, kv1, tokens1 = case(n_one, 1)
+    times1 = time_passes(fn1, 3, 1)
+    t1 = float(np.median(times1))
+    stats = lambda ts: {"median": round(float(np.median(ts)), 4), "min": round(min(ts), 4),
+                        "max": round(max(ts), 4), "passes": len(ts)}
+    return {"value": round(kv / t / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {n_all} of {cfg.num_seqs} sequences ({tokens} context tokens, {kv} K/V bytes), "
+                      f"fp64, {threads} threads, median of {len(times)} passes",
+            "tokens_per_s": round(n_all / t, 3), "pass_s": stats(times), "host": host_cores(),
+            "single_thread": {"value": round(kv1 / t1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                              "sample": f"first {n_one} sequences ({tokens1} context tokens, {kv1} K/V bytes), "
+                                        f"fp64, 1 thread, median of 3 passes",
+                              "pass_s": stats(times1)}}
 
 
 if __name__ == "__main__":

@@ -127,8 +127,10 @@ PA_API size_t pa_paged_attention_workspace_size(int num_seqs, int num_heads, int
  *  value_cache    [num_blocks][block_size][num_kv_heads][head_size], kv_dtype; read only.
  *  k_scale,
  *  v_scale        [num_kv_heads] fp32 dequantisation scales; required for PA_FP8_E4M3, else ignored.
- *  block_tables   [num_seqs][max_blocks_per_seq] int32 physical block ids; entries past
- *                 ceil(context_lens[s]/block_size) are never read.
+ *  block_tables   [num_seqs][max_blocks_per_seq] int32 physical block ids; only the first
+ *                 min(ceil(context_lens[s]/block_size), max_blocks_per_seq) entries of row s are
+ *                 read, so the rest may hold anything (the kernel prefetches ids a window at a time,
+ *                 clamped to that count).
  *  context_lens   [num_seqs] int32.
  *  max_context_len host int, >= every context_lens[s]; sizes the launch (partitions).
  *  scale          the softmax scale (1/sqrt(head_size) in the pages' formula).
@@ -158,7 +160,12 @@ PA_API pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dty
  *    exits; a call whose pa_paged_attention_workspace_size(...) exceeds it returns
  *    PA_ERR_WORKSPACE_TOO_SMALL without enqueuing anything;
  *  - set-up: the first call on each device looks up the array's device address on that device (it
- *    must be the current device); make that first call before any stream capture;
+ *    must be the current device); make that first call before any stream capture. The address is
+ *    kept per device together with the context it was found in, and looked up again when another
+ *    context is current; after cudaDeviceReset the module is loaded anew and the array may move, so
+ *    do not keep using this entry point across a device reset;
+ *  - checks: every argument check of pa_paged_attention (except those on the workspace) runs first,
+ *    with the same results; only then is the request's size compared with the array;
  *  - sharing: every call on a device uses the same array, which keeps the last call's contents; calls
  *    that overlap on the GPU (different streams without ordering) race and give undefined results;
  *  - errors: the device error word lives in the array; when device_error_out (a DEVICE pointer to

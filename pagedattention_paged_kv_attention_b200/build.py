@@ -1,6 +1,9 @@
 """Build libpagedattn.so in-tree with nvcc for sm_100a (static CUDA runtime, no torch extension).
 
-    python -m pagedattention_paged_kv_attention_b200.build [--force] [-D NAME=VALUE ...]
+    python -m pagedattention_paged_kv_attention_b200.build [--force] [-D NAME=VALUE ...] [--output PATH]
+
+-D PA_TRACE --output libpagedattn_trace.so builds the timing-trace variant of the decode kernels (their
+work is unchanged; they also write %globaltimer records into the workspace) under another name.
 
 Each translation unit (.cu, and the host-only .cpp) is compiled in parallel, then linked into one shared library next to this
 file. The library exports only the C ABI declared in include/*.h.
@@ -18,7 +21,7 @@ LIBRARY = os.path.join(HERE, "libpagedattn.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 SOURCES = ["pa_api.cu", "pa_attention_bf16.cu", "pa_attention_f16.cu", "pa_static_workspace.cu",
-           "pa_prefill.cu", "pa_block_manager.cpp"]
+           "pa_prefill.cu", "pa_probe.cu", "pa_block_manager.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
@@ -39,7 +42,7 @@ def build(force=False, defines=(), output=None, verbose=False):
     output = output or LIBRARY
     if not force and not _stale(output, defines):
         return output
-    build_dir = os.path.join(HERE, "_build")
+    build_dir = os.path.join(HERE, "_build", "-".join(sorted(defines)) or "default")
     os.makedirs(build_dir, exist_ok=True)
     dflags = [f"-D{d}" for d in defines]
 
@@ -70,4 +73,5 @@ def build(force=False, defines=(), output=None, verbose=False):
 if __name__ == "__main__":
     args = sys.argv[1:]
     defines = [args[i + 1] for i, a in enumerate(args) if a == "-D"]
-    print(build(force="--force" in args, defines=defines, verbose="-v" in args))
+    output = next((os.path.abspath(args[i + 1]) for i, a in enumerate(args) if a == "--output"), None)
+    print(build(force="--force" in args, defines=defines, output=output, verbose="-v" in args))

@@ -63,10 +63,10 @@ int plan_partition(int num_seqs, int num_heads, int num_kv_heads, int max_contex
 }
 
 struct WorkspaceLayout {
-  size_t part_m, part_l, part_o, total;
+  size_t part_m, part_l, part_o, trace, total;
 };
 
-WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_size, int partitions) {
+WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int num_kv_heads, int head_size, int partitions) {
   WorkspaceLayout w{};
   w.total = PA_WORKSPACE_HEADER_BYTES;
   if (partitions > 1) {
@@ -76,6 +76,16 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_size, int
     w.part_o = w.part_l + round_up(rows * 4, 256);
     w.total = w.part_o + round_up(rows * head_size * 4, 256);
   }
+#ifdef PA_TRACE
+  // Timing records of the trace build (pa::kTraceItemBase words, then 4 per work item) at the end.
+  int g_tile, subgroups;
+  group_tiling(num_heads / num_kv_heads, &g_tile, &subgroups);
+  const size_t items = static_cast<size_t>(partitions) * num_seqs * ceil_div(num_kv_heads, pa::kHeadBlock) * subgroups;
+  w.trace = w.total;
+  w.total += round_up((pa::kTraceItemBase + 4 * items) * 8, 256);
+#else
+  (void)num_kv_heads;
+#endif
   return w;
 }
 
@@ -107,7 +117,72 @@ bool supported_block_size(int bs) { return bs == 8 || bs == 16 || bs == 32 || bs
 // Elements of one token's [num_kv_heads][head_size] row that the cache-write kernels index with int.
 constexpr int64_t kMaxRowElems = int64_t(1) << 24;
 
+// The plan of a valid paged-attention call (sizes only; no pointer is dereferenced).
+struct AttnPlan {
+  bool empty;
+  int ps, partitions, g_tile, subgroups, head_blocks;
+  unsigned long long items;
+  WorkspaceLayout ws;
+};
+
+pa_status check_attention(const void* out, const void* query, pa_dtype q_dtype, const void* key_cache,
+                          const void* value_cache, pa_dtype kv_dtype, const float* k_scale, const float* v_scale,
+                          const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                          int num_seqs, int num_heads, int num_kv_heads, int head_size, int block_size,
+                          int num_blocks, int max_context_len, float scale, int partition_size, AttnPlan* plan) {
+  *plan = AttnPlan{};
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
+      head_size <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 ||
+      partition_size < 0 || !std::isfinite(scale))
+    return PA_ERR_INVALID_ARGUMENT;
+  if (!is_dtype(q_dtype) || !is_dtype(kv_dtype) || !is_16bit(q_dtype)) return PA_ERR_INVALID_ARGUMENT;
+  if (num_seqs == 0) {
+    plan->empty = true;
+    return PA_OK;
+  }
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens) return PA_ERR_INVALID_ARGUMENT;
+  if (!aligned(out, 16) || !aligned(query, 16) || !aligned(key_cache, 16) || !aligned(value_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return PA_ERR_INVALID_ARGUMENT;
+  const bool fp8 = is_fp8(kv_dtype);
+  if (fp8 && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4))) return PA_ERR_INVALID_ARGUMENT;
+  if (!fp8 && kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;
+  if (head_size != 64 && head_size != 128) return PA_ERR_UNSUPPORTED;
+  if (fp8 && head_size != 128) return PA_ERR_UNSUPPORTED;
+  if (!supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
+  if (num_blocks >= (1 << 27)) return PA_ERR_UNSUPPORTED;  // block ids ride in 28 bits of a stage message
+  plan->ps = plan_partition(num_seqs, num_heads, num_kv_heads, max_context_len, partition_size);
+  if (plan->ps <= 0) return PA_ERR_INVALID_ARGUMENT;
+  plan->partitions = std::max(1, ceil_div(max_context_len, plan->ps));
+  group_tiling(num_heads / num_kv_heads, &plan->g_tile, &plan->subgroups);
+  plan->head_blocks = ceil_div(num_kv_heads, pa::kHeadBlock);
+  plan->items = static_cast<unsigned long long>(plan->partitions) * num_seqs * plan->head_blocks * plan->subgroups;
+  if (num_seqs > 65535 || plan->items > 0x7fffffffULL) return PA_ERR_UNSUPPORTED;
+  plan->ws = workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, plan->partitions);
+  return PA_OK;
+}
+
 }  // namespace
+
+namespace pa_host {
+
+pa_status paged_attention_check(const void* out, const void* query, pa_dtype q_dtype, const void* key_cache,
+                                const void* value_cache, pa_dtype kv_dtype, const float* k_scale,
+                                const float* v_scale, const int32_t* block_tables, int max_blocks_per_seq,
+                                const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                                int head_size, int block_size, int num_blocks, int max_context_len, float scale,
+                                int partition_size, size_t* workspace_bytes, bool* empty) {
+  AttnPlan plan;
+  const pa_status st = check_attention(out, query, q_dtype, key_cache, value_cache, kv_dtype, k_scale, v_scale,
+                                       block_tables, max_blocks_per_seq, context_lens, num_seqs, num_heads,
+                                       num_kv_heads, head_size, block_size, num_blocks, max_context_len, scale,
+                                       partition_size, &plan);
+  *workspace_bytes = plan.ws.total;
+  *empty = plan.empty;
+  return st;
+}
+
+}  // namespace pa_host
 
 extern "C" {
 
@@ -135,7 +210,7 @@ size_t pa_paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv
   const int ps = plan_partition(num_seqs, num_heads, num_kv_heads, max_context_len, partition_size);
   if (ps <= 0) return 0;
   const int partitions = std::max(1, ceil_div(max_context_len, ps));
-  return workspace_layout(num_seqs, num_heads, head_size, partitions).total;
+  return workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, partitions).total;
 }
 
 pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dtype, const void* key_cache,
@@ -146,35 +221,20 @@ pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dtype, con
                              int partition_size, void* workspace, size_t workspace_bytes,
                              pa_stream_t stream) {
   // ---- validation: no CUDA call before every check has passed ----
-  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
-      head_size <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 ||
-      partition_size < 0 || !std::isfinite(scale))
-    return PA_ERR_INVALID_ARGUMENT;
-  if (!is_dtype(q_dtype) || !is_dtype(kv_dtype) || !is_16bit(q_dtype)) return PA_ERR_INVALID_ARGUMENT;
-  if (num_seqs == 0) return PA_OK;  // empty batch: nothing is read or written
-  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens || !workspace)
-    return PA_ERR_INVALID_ARGUMENT;
-  if (!aligned(out, 16) || !aligned(query, 16) || !aligned(key_cache, 16) || !aligned(value_cache, 16) ||
-      !aligned(workspace, 16) || !aligned(block_tables, 4) || !aligned(context_lens, 4))
-    return PA_ERR_INVALID_ARGUMENT;
+  AttnPlan plan;
+  const pa_status checked = check_attention(out, query, q_dtype, key_cache, value_cache, kv_dtype, k_scale, v_scale,
+                                            block_tables, max_blocks_per_seq, context_lens, num_seqs, num_heads,
+                                            num_kv_heads, head_size, block_size, num_blocks, max_context_len, scale,
+                                            partition_size, &plan);
+  if (checked != PA_OK) return checked;
+  if (plan.empty) return PA_OK;  // empty batch: nothing is read or written
+  if (!workspace || !aligned(workspace, 16)) return PA_ERR_INVALID_ARGUMENT;
+  if (workspace_bytes < plan.ws.total) return PA_ERR_WORKSPACE_TOO_SMALL;
+  const int ps = plan.ps, partitions = plan.partitions, g_tile = plan.g_tile, subgroups = plan.subgroups;
+  const int head_blocks = plan.head_blocks;
+  const unsigned long long items = plan.items;
   const bool fp8 = is_fp8(kv_dtype);
-  if (fp8 && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4))) return PA_ERR_INVALID_ARGUMENT;
-  if (!fp8 && kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;
-  if (head_size != 64 && head_size != 128) return PA_ERR_UNSUPPORTED;
-  if (fp8 && head_size != 128) return PA_ERR_UNSUPPORTED;
-  if (!supported_block_size(block_size)) return PA_ERR_UNSUPPORTED;
-  if (num_blocks >= (1 << 27)) return PA_ERR_UNSUPPORTED;  // block ids ride in 28 bits of a stage message
-  const int ps = plan_partition(num_seqs, num_heads, num_kv_heads, max_context_len, partition_size);
-  if (ps <= 0) return PA_ERR_INVALID_ARGUMENT;
-  const int partitions = std::max(1, ceil_div(max_context_len, ps));
-  int g_tile, subgroups;
-  group_tiling(num_heads / num_kv_heads, &g_tile, &subgroups);
-  const int head_blocks = ceil_div(num_kv_heads, pa::kHeadBlock);
-  const unsigned long long items =
-      static_cast<unsigned long long>(partitions) * num_seqs * head_blocks * subgroups;
-  if (num_seqs > 65535 || items > 0x7fffffffULL) return PA_ERR_UNSUPPORTED;
-  const WorkspaceLayout ws = workspace_layout(num_seqs, num_heads, head_size, partitions);
-  if (workspace_bytes < ws.total) return PA_ERR_WORKSPACE_TOO_SMALL;
+  const WorkspaceLayout& ws = plan.ws;
 
   // ---- launch ----
   CUtensorMap tk, tv;
@@ -212,6 +272,9 @@ pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dtype, con
   a.num_items = static_cast<unsigned int>(items);
   a.scale_log2 = scale * pa::kLog2e;
   a.scale_block_stride = scale_block_stride(kv_dtype, num_kv_heads);
+#ifdef PA_TRACE
+  a.trace = reinterpret_cast<unsigned long long*>(wsb + ws.trace);
+#endif
   const int grid = static_cast<int>(std::min<unsigned long long>(static_cast<unsigned long long>(sms), items));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = q_dtype == PA_BF16 ? pa::launch_attention_bf16(tk, tv, a, fp8, head_size, g_tile, grid, st)
@@ -301,22 +364,19 @@ pa_status pa_reshape_and_cache_layers(const void* const* keys, const void* const
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const float* const* ks = fp8 ? k_scales : nullptr;
   const float* const* vs = fp8 ? v_scales : nullptr;
-  if (in_dtype == PA_BF16) {
-    if (fp8)
-      pa::reshape_and_cache_layers_kernel<__nv_bfloat16, __nv_fp8_e4m3><<<grid, threads, 0, st>>>(
-          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks, sstride);
-    else
-      pa::reshape_and_cache_layers_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, threads, 0, st>>>(
-          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks, sstride);
-  } else {
-    if (fp8)
-      pa::reshape_and_cache_layers_kernel<__half, __nv_fp8_e4m3><<<grid, threads, 0, st>>>(
-          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks, sstride);
-    else
-      pa::reshape_and_cache_layers_kernel<__half, __half><<<grid, threads, 0, st>>>(
-          keys, values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size, block_size, num_blocks, sstride);
-  }
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const auto launch = [&](auto in_tag, auto cache_tag) {
+    using IT = decltype(in_tag);
+    using KVT = decltype(cache_tag);
+    return pa_host::launch_plain(pa::reshape_and_cache_layers_kernel<IT, KVT>, grid, dim3(threads), 0, st, keys,
+                                 values, key_caches, value_caches, ks, vs, slot_mapping, num_kv_heads, head_size,
+                                 block_size, num_blocks, sstride);
+  };
+  cudaError_t e;
+  if (in_dtype == PA_BF16)
+    e = fp8 ? launch(__nv_bfloat16{}, __nv_fp8_e4m3{}) : launch(__nv_bfloat16{}, __nv_bfloat16{});
+  else
+    e = fp8 ? launch(__half{}, __nv_fp8_e4m3{}) : launch(__half{}, __half{});
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_copy_blocks_layers(void* const* key_caches, void* const* value_caches, int num_layers, pa_dtype kv_dtype,
@@ -331,10 +391,11 @@ pa_status pa_copy_blocks_layers(void* const* key_caches, void* const* value_cach
   const int64_t block_bytes = static_cast<int64_t>(block_size) * num_kv_heads * head_size * elem_bytes(kv_dtype);
   if (block_bytes % 16 != 0 || num_layers > 65535) return PA_ERR_UNSUPPORTED;
   if (num_pairs == 0 || num_layers == 0) return PA_OK;
-  pa::copy_blocks_layers_kernel<<<dim3(static_cast<unsigned>(num_pairs), 2, static_cast<unsigned>(num_layers)), 256, 0,
-                                  reinterpret_cast<cudaStream_t>(stream)>>>(key_caches, value_caches, block_mapping,
-                                                                            block_bytes, num_blocks);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const cudaError_t e = pa_host::launch_plain(
+      pa::copy_blocks_layers_kernel, dim3(static_cast<unsigned>(num_pairs), 2, static_cast<unsigned>(num_layers)),
+      dim3(256), 0, reinterpret_cast<cudaStream_t>(stream), key_caches, value_caches, block_mapping, block_bytes,
+      num_blocks);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 namespace {
@@ -375,10 +436,12 @@ pa_status pa_swap_blocks(void* dst_key_cache, void* dst_value_cache, const void*
   void* sv = device_reachable(src_value_cache);
   void* bm = device_reachable(block_mapping);
   if (!dk || !dv || !sk || !sv || !bm) return PA_ERR_INVALID_ARGUMENT;
-  pa::swap_blocks_kernel<<<dim3(static_cast<unsigned>(num_pairs), 2), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint8_t*>(dk), static_cast<uint8_t*>(dv), static_cast<const uint8_t*>(sk),
-      static_cast<const uint8_t*>(sv), static_cast<const int64_t*>(bm), block_bytes, src_num_blocks, dst_num_blocks);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const cudaError_t e = pa_host::launch_plain(
+      pa::swap_blocks_kernel, dim3(static_cast<unsigned>(num_pairs), 2), dim3(256), 0,
+      reinterpret_cast<cudaStream_t>(stream), static_cast<uint8_t*>(dk), static_cast<uint8_t*>(dv),
+      static_cast<const uint8_t*>(sk), static_cast<const uint8_t*>(sv), static_cast<const int64_t*>(bm), block_bytes,
+      src_num_blocks, dst_num_blocks);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_copy_blocks_check(const int64_t* host_block_mapping, int num_pairs, int num_blocks) {
@@ -398,8 +461,9 @@ pa_status pa_copy_blocks_check(const int64_t* host_block_mapping, int num_pairs,
 pa_status pa_selftest_wait_timeout(unsigned int* device_error_word, unsigned long long limit_ns, pa_stream_t stream) {
   if (!device_error_word || !aligned(device_error_word, 4) || limit_ns == 0 || limit_ns > 10000000000ull)
     return PA_ERR_INVALID_ARGUMENT;
-  pa::selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(device_error_word, limit_ns);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const cudaError_t e = pa_host::launch_plain(pa::selftest_wait_kernel, dim3(1), dim3(32), 0,
+                                              reinterpret_cast<cudaStream_t>(stream), device_error_word, limit_ns);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_get_device_error(const void* workspace, unsigned int* err_out, pa_stream_t stream) {

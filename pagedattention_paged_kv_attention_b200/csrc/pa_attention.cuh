@@ -96,7 +96,15 @@ struct AttnArgs {
   unsigned int num_items;       // num_partitions * num_seqs * head_blocks * subgroups
   float scale_log2;             // softmax scale * log2(e)
   int scale_block_stride;       // FP8 scales: 0 = per kv head, num_kv_heads = per (block, kv head)
+  unsigned long long* trace;    // timing records, written only by builds with PA_TRACE defined (else null)
 };
+
+// Timing records of a PA_TRACE build (%globaltimer, ns), in 64-bit words: [0] ~(first start of a
+// split-K reduce CTA), [1] last end of one; CTA c at kTraceCtaBase + 4c: start, end, items, SM id;
+// item i at kTraceItemBase + 4i: producer start, consumer finish, CTA, tokens.
+constexpr int kTraceMaxCtas = 1024;
+constexpr int kTraceCtaBase = 8;
+constexpr int kTraceItemBase = kTraceCtaBase + 4 * kTraceMaxCtas;
 
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
@@ -291,6 +299,14 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
   // tokens in the cache, a reset workspace) must be visible.
   grid_dependency_wait();
   grid_dependents_launch();
+#ifdef PA_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < kTraceMaxCtas) {
+    unsigned int smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    args.trace[kTraceCtaBase + 4 * blockIdx.x] = global_timer_ns();
+    args.trace[kTraceCtaBase + 4 * blockIdx.x + 3] = smid;
+  }
+#endif
   __syncthreads();
 
   if (warp == 0) {
@@ -311,6 +327,8 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     // Items flow through a two-deep software pipeline: while item i streams, the loads describing item
     // i+1 (its context length and a window of its block ids, one id per lane per 32 boxes) are in
     // flight, and the work counter has already been asked for item i+2. All state is in registers.
+    // Only the table entries the context needs (the first ceil(L / block_size), at most the table's
+    // width) are ever read; the rest of the window holds 0 and is never used.
     unsigned int cur_idx = 0, nxt_idx = 0;
     int cur_L = 0, nxt_L = 0;
     int cur_ids[kIdWindow], nxt_ids[kIdWindow];
@@ -319,10 +337,11 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     if ((IDX) < args.num_items) {                                                                      \
       const ItemCoord pc_ = decode_item((IDX), args);                                                  \
       LV = __ldg(args.context_lens + pc_.s);                                                           \
+      const int need_ = LV <= 0 ? 0 : cmin(args.max_blocks_per_seq, LV / bs + (LV % bs != 0));         \
       const int32_t* row_ = args.block_tables + static_cast<size_t>(pc_.s) * args.max_blocks_per_seq;  \
       _Pragma("unroll") for (int j_ = 0; j_ < kIdWindow; ++j_) {                                       \
         const int entry_ = ((pc_.part * boxes_per_part + j_ * 32 + lane) * kBoxTokens) / bs;           \
-        IDS[j_] = entry_ < args.max_blocks_per_seq ? __ldg(row_ + entry_) : 0;                         \
+        IDS[j_] = entry_ < need_ ? __ldg(row_ + entry_) : 0;                                           \
       }                                                                                                \
     }                                                                                                  \
   } while (0)
@@ -375,7 +394,14 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             inf.h_sub = h_sub;
             inf.heads = heads;
             inf.write_final = n_parts <= 1;
-            inf.pad0 = inf.pad1 = 0;
+            inf.pad0 = static_cast<int>(cur_idx);
+            inf.pad1 = 0;
+#ifdef PA_TRACE
+            unsigned long long* rec = args.trace + kTraceItemBase + 4ull * cur_idx;
+            rec[0] = global_timer_ns();
+            rec[2] = blockIdx.x;
+            rec[3] = static_cast<unsigned long long>(tok_end - tok_begin);
+#endif
             infos[qb] = inf;
             mbar_arrive_expect_tx(&qfull[qb], row_bytes * kv_here);
           }
@@ -796,6 +822,10 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
 
+#ifdef PA_TRACE
+      if ((m.flags & kMsgLast) && cw == 0 && lane == 0)
+        args.trace[kTraceItemBase + 4ull * static_cast<unsigned int>(inf.pad0) + 1] = global_timer_ns();
+#endif
       if constexpr (S::kMma) {
        if ((m.flags & kMsgLast) && active) {
         // ---- end of the item (tensor-core path): row g = lane/4 is query head g ----
@@ -887,6 +917,9 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
 
   // The last CTA to finish resets the work counter for the next launch on this workspace.
   __syncthreads();
+#ifdef PA_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < kTraceMaxCtas) args.trace[kTraceCtaBase + 4 * blockIdx.x + 1] = global_timer_ns();
+#endif
   if (threadIdx.x == 0) {
     __threadfence();
     const unsigned int done = atomicAdd(args.header + kWsDone, 1u);
@@ -908,6 +941,15 @@ paged_attention_reduce(const AttnArgs args) {
   constexpr int kPer = D / 32;  // elements per lane: 4 for d = 128, 2 for d = 64
   grid_dependency_wait();
   grid_dependents_launch();
+#ifdef PA_TRACE
+  if (threadIdx.x == 0) atomicMax(args.trace, ~global_timer_ns());
+  struct TraceEnd {
+    unsigned long long* t;
+    __device__ ~TraceEnd() {  // thread 0's exit stands for its CTA's
+      if (threadIdx.x == 0) atomicMax(t + 1, global_timer_ns());
+    }
+  } trace_end{args.trace};
+#endif
   const int lane = threadIdx.x & 31;
   const long row = static_cast<long>(blockIdx.x) * kReduceWarps + (threadIdx.x >> 5);
   if (row >= static_cast<long>(args.num_seqs) * args.num_heads) return;

@@ -58,4 +58,30 @@ cudaError_t launch_overlapped(void (*kernel)(Params...), dim3 grid, dim3 block, 
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Ordinary launch (full stream serialisation) whose status is the launch's own: unlike <<<>>> followed
+// by cudaGetLastError, it neither reports nor clears an earlier error left by the caller's code.
+template <typename... Params, typename... Args>
+cudaError_t launch_plain(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                         Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Every argument check of pa_paged_attention except those on the workspace, with no CUDA call. On
+// PA_OK, *workspace_bytes is the workspace the call needs and *empty tells whether the call has
+// nothing to do (num_seqs == 0). Defined in pa_api.cu; pa_paged_attention_static runs it before
+// comparing that size with its fixed array.
+pa_status paged_attention_check(const void* out, const void* query, pa_dtype q_dtype, const void* key_cache,
+                                const void* value_cache, pa_dtype kv_dtype, const float* k_scale,
+                                const float* v_scale, const int32_t* block_tables, int max_blocks_per_seq,
+                                const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                                int head_size, int block_size, int num_blocks, int max_context_len, float scale,
+                                int partition_size, size_t* workspace_bytes, bool* empty);
+
 }  // namespace pa_host

@@ -60,8 +60,7 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
   const int smem = static_cast<int>(pa::pf::Layout<D>::kBytes);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kernel<<<grid, pa::pf::kThreads, smem, st>>>(tq, tk, tv, a);
-  return cudaGetLastError();
+  return pa_host::launch_plain(kernel, grid, dim3(pa::pf::kThreads), static_cast<size_t>(smem), st, tq, tk, tv, a);
 }
 
 }  // namespace

@@ -12,7 +12,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIBRARY_PATH = os.path.join(_HERE, "libpagedattn.so")
+# PA_LIBRARY_PATH selects another in-tree build of the same library (e.g. the timing-trace variant).
+LIBRARY_PATH = os.environ.get("PA_LIBRARY_PATH") or os.path.join(_HERE, "libpagedattn.so")
 
 (PA_OK, PA_ERR_INVALID_ARGUMENT, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE_TOO_SMALL, PA_ERR_CUDA, PA_ERR_OUT_OF_BLOCKS,
  PA_ERR_HOST_MEMORY) = range(7)
@@ -30,6 +31,8 @@ EXPORTS = (
     "pa_bm_create", "pa_bm_destroy", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_append_slots",
     "pa_bm_block_tables", "pa_bm_plan_decode", "pa_bm_free_sequence", "pa_bm_swap_out", "pa_bm_swap_in",
     "pa_bm_num_free_blocks", "pa_bm_sequence_info", "pa_bm_ref_count",
+    # include/pa_probe.h
+    "pa_probe_stream_read", "pa_probe_paged_read",
 )
 
 if not os.path.exists(LIBRARY_PATH):
@@ -50,6 +53,10 @@ lib.pa_paged_attention.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _p, _
 lib.pa_paged_attention_static.restype = _i
 lib.pa_paged_attention_static.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i,
                                           _f, _i, _p, _p]
+lib.pa_probe_stream_read.restype = _i
+lib.pa_probe_stream_read.argtypes = [_p, _sz, _i, _p, _p]
+lib.pa_probe_paged_read.restype = _i
+lib.pa_probe_paged_read.argtypes = [_p, _p, _i, _p, _i, _p, _i, _i, _i, _i, _i, _p, _p]
 lib.pa_paged_prefill.restype = _i
 lib.pa_paged_prefill.argtypes = [_p, _p, _i, _p, _p, _i, _p, _i, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _sz,
                                  _p]
@@ -339,3 +346,30 @@ def selftest_wait_timeout(device_error_word, limit_ns, stream=None):
 
 def clear_device_error(workspace, stream=None):
     _check(lib.pa_clear_device_error(_ptr(workspace), _stream(stream)), "pa_clear_device_error")
+
+
+def probe_stream_read(buf, repeat=1, sink=None, stream=None):
+    """Read-bandwidth probe (include/pa_probe.h): reads every byte of the device tensor `buf`,
+    `repeat` times over, with 16-byte loads and no compute. `sink`: optional one-element int64 device
+    tensor the probe may write."""
+    if sink is None:
+        sink = torch.zeros(1, dtype=torch.int64, device=buf.device)
+    nbytes = buf.numel() * buf.element_size()
+    _check(lib.pa_probe_stream_read(_arg(buf, "buf"), nbytes, int(repeat), _arg(sink, "sink", _I64),
+                                    _stream(stream)), "pa_probe_stream_read")
+    return sink
+
+
+def probe_paged_read(key_cache, value_cache, block_tables, context_lens, sink=None, stream=None):
+    """Reads exactly the K/V rows of the batch's valid tokens through the block table, with plain loads
+    and no compute (include/pa_probe.h)."""
+    if sink is None:
+        sink = torch.zeros(1, dtype=torch.int64, device=key_cache.device)
+    NB, bs, Hkv, d = key_cache.shape
+    _same(key_cache, value_cache, "key_cache/value_cache")
+    S, max_blocks = block_tables.shape
+    _check(lib.pa_probe_paged_read(_arg(key_cache, "key_cache", dim=4), _arg(value_cache, "value_cache", dim=4),
+                                   dtype_code(key_cache.dtype), _arg(block_tables, "block_tables", _I32, 2),
+                                   max_blocks, _arg(context_lens, "context_lens", _I32, 1), S, Hkv, d, bs, NB,
+                                   _arg(sink, "sink", _I64), _stream(stream)), "pa_probe_paged_read")
+    return sink

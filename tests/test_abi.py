@@ -88,6 +88,35 @@ def test_attention_rejects_bad_arguments_without_cuda(P, over, status):
     assert call_attention(P, **over) == status
 
 
+def call_static(P, **over):
+    args = dict(out=16, query=16, q_dtype=P.PA_BF16, key_cache=16, value_cache=16, kv_dtype=P.PA_BF16, k_scale=None,
+                v_scale=None, block_tables=16, max_blocks_per_seq=4, context_lens=16, num_seqs=2, num_heads=8,
+                num_kv_heads=2, head_size=128, block_size=16, num_blocks=10, max_context_len=64, scale=0.1,
+                partition_size=0, device_error_out=None, stream=None)
+    args.update(over)
+    return P.lib.pa_paged_attention_static(*args.values())
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(out=None), 1), (dict(out=8), 1), (dict(num_heads=6, num_kv_heads=4), 1), (dict(q_dtype=7), 1),
+    (dict(kv_dtype=2), 1), (dict(head_size=96), 2), (dict(block_size=4), 2), (dict(kv_dtype=0), 2),
+    (dict(device_error_out=18), 1), (dict(num_seqs=0), 0),
+])
+def test_static_entry_checks_arguments_like_the_workspace_entry(P, over, status):
+    assert call_static(P, **over) == status
+
+
+@pytest.mark.parametrize("bad", [dict(q_dtype=7), dict(kv_dtype=2), dict(head_size=96), dict(out=None)])
+def test_static_entry_reports_a_bad_argument_before_an_oversize_request(P, bad):
+    """A request too large for the fixed array that is also invalid for another reason reports the
+    other reason: the argument checks come before the size comparison."""
+    big = dict(num_seqs=2048, num_heads=64, num_kv_heads=8, max_blocks_per_seq=2048, max_context_len=32768,
+               partition_size=64)
+    assert call_static(P, **big) == P.PA_ERR_WORKSPACE_TOO_SMALL
+    assert call_static(P, **big, **bad) == call_attention(P, **{k: v for k, v in big.items()}, **bad)
+    assert call_static(P, **big, **bad) in (P.PA_ERR_INVALID_ARGUMENT, P.PA_ERR_UNSUPPORTED)
+
+
 def test_reshape_and_copy_reject_bad_arguments(P):
     L = P.lib
     ok = dict(key=16, value=16, in_dtype=P.PA_BF16, key_cache=16, value_cache=16, kv_dtype=P.PA_BF16,

@@ -6,6 +6,7 @@
 * sequences that share prefix blocks give bitwise the same output as private copies of the blocks;
 * a block id outside the pool and a context longer than its table set the device error word and
   NaN the affected rows without faulting; every other row stays correct;
+* block-table entries past ceil(L / block_size) may hold anything (decode and prefill);
 * empty batches and zero-length contexts.
 """
 import numpy as np
@@ -141,3 +142,49 @@ def test_copy_blocks_touches_only_destinations(P):
     bad = w.cow_mapping.clone()
     bad[1, 1] = bad[0, 0]                      # a destination that is also a source
     assert not P.copy_blocks_check(bad, w.num_blocks)
+
+
+def poisoned_past_context(tables, lens, block_size, num_blocks, extra=160):
+    """The block tables widened by `extra` columns, with every entry past ceil(L / block_size) of each
+    row replaced by ids outside the pool (negative, past the pool, INT32_MAX)."""
+    S, mb = tables.shape
+    wide = torch.empty((S, mb + extra), dtype=torch.int32)
+    wide[:, :mb] = tables
+    bad = torch.tensor([-1, num_blocks, 2 ** 31 - 1, -(2 ** 31)], dtype=torch.int32)
+    for s in range(S):
+        need = -(-int(lens[s]) // block_size)
+        wide[s, need:] = bad.repeat((mb + extra - need) // 4 + 1)[:mb + extra - need]
+    return wide
+
+
+@pytest.mark.parametrize("name", ["7b", "70b_gqa", "long_splitk"])
+def test_table_entries_past_the_context_are_not_used(P, name):
+    """Only the first ceil(L / block_size) entries of a table row are read: poisoning the rest with
+    ids outside the pool changes no output bit and sets no error bit."""
+    cfg = W.CONFIGS[name]
+    w = W.make_workload(cfg, num_seqs=10, prefilled=True)
+    wide = poisoned_past_context(w.block_tables, w.context_lens, cfg.block_size, w.num_blocks)
+    ref, ws_ref = run(P, w, write_new=False, copy=False, partition_size=cfg.partition_size)
+    out, ws = run(P, w, write_new=False, copy=False, partition_size=cfg.partition_size, block_tables=wide)
+    assert P.get_device_error(ws) == 0 and P.get_device_error(ws_ref) == 0
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+
+
+def test_prefill_table_entries_past_the_context_are_not_used(P):
+    cfg = W.PREFILL_CONFIGS["prefill_tiny"]
+    w = W.make_prefill_workload(cfg)
+    dev = torch.device("cuda")
+    kc, vc = w.key_values.to(dev), w.value_values.to(dev)
+    P.reshape_and_cache(w.new_key.to(dev), w.new_value.to(dev), kc, vc, w.slot_mapping.to(dev))
+    q = w.query.to(dev)
+    outs = []
+    for tables in (w.block_tables, poisoned_past_context(w.block_tables, w.context_lens, cfg.block_size,
+                                                         w.num_blocks)):
+        out = torch.full_like(q, float("nan"))
+        ws = torch.zeros(64, dtype=torch.int32, device=dev)
+        P.paged_prefill(out, q, kc, vc, tables.to(dev), w.context_lens.to(dev), w.q_start.to(dev),
+                        cfg.softmax_scale, w.max_q_len, ws)
+        torch.cuda.synchronize()
+        assert P.get_device_error(ws) == 0
+        outs.append(out)
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
