@@ -53,7 +53,7 @@ constexpr int kHeadBlock = 8;            // kv heads per work item (one consumer
 constexpr int kConsumerWarps = kHeadBlock;
 constexpr int kBoxTokens = 8;            // tokens per TMA box (block_size >= 8); one swizzle atom
 constexpr int kMaxStages = 8;            // ring depth cap (the depth itself is per variant, see Layout)
-constexpr int kSmemBudget = 200 * 1024;  // shared memory the layout may use (of 227 KB per CTA)
+constexpr int kSmemBudget = 204 * 1024;  // shared memory the layout may use (of 227 KB per CTA)
 constexpr int kQueryBuffers = 2;
 constexpr int kIdWindow = 4;             // block ids prefetched per item: 32 * kIdWindow stages
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
@@ -163,7 +163,10 @@ struct ItemInfo {
 template <typename QT, int D, int G, int EB>
 struct Layout {
   using S = Shape<D, G, EB>;
-  static constexpr int kQueryOne = kHeadBlock * G * D * int(sizeof(QT));       // [8 kv heads][G][D]
+  // Query rows [8 kv heads][G][kQRow]: each row padded by 32 bytes, so that the fragment loads of the
+  // G rows at an item's start fall in different banks (rows 256 bytes apart would share them).
+  static constexpr int kQRow = D + 32 / int(sizeof(QT));
+  static constexpr int kQueryOne = kHeadBlock * G * kQRow * int(sizeof(QT));
   static constexpr int kSmall = kConsumerWarps * S::kTS * G * 4 + kConsumerWarps * G * 4 + 1024;
   // Ring depth: as many stages as the budget leaves after the query buffers and small tables.
   static constexpr int kStages = cmin(kMaxStages, (kSmemBudget - kQueryBuffers * kQueryOne - kSmall) / S::kStageBytes);
@@ -406,11 +409,13 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
             mbar_arrive_expect_tx(&qfull[qb], row_bytes * kv_here);
           }
           __syncwarp();
-          if (lane < kv_here) {
+          // One bulk copy per query row (row r = kv * heads + g), into its padded slot.
+          for (int r = lane; r < kv_here * heads; r += 32) {
+            const int kv = r / heads, g = r - kv * heads;
             const QT* qsrc = static_cast<const QT*>(args.query) +
-                             (static_cast<size_t>(c.s) * args.num_heads + (kvh0 + lane) * args.group + h_sub) * D;
-            bulk_copy_g2s(smem + Lay::kQuery + qb * Lay::kQueryOne + lane * G * D * sizeof(QT), qsrc, row_bytes,
-                          &qfull[qb]);
+                             (static_cast<size_t>(c.s) * args.num_heads + (kvh0 + kv) * args.group + h_sub + g) * D;
+            bulk_copy_g2s(smem + Lay::kQuery + qb * Lay::kQueryOne + (kv * G + g) * Lay::kQRow * sizeof(QT), qsrc,
+                          static_cast<uint32_t>(D * sizeof(QT)), &qfull[qb]);
           }
 
           const int32_t* row = args.block_tables + static_cast<size_t>(c.s) * args.max_blocks_per_seq;
@@ -535,21 +540,27 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           if (active && !BS) qscale *= args.k_scale[inf.kvh0 + cw];
         }
         zitem = qscale;
-        const QT* qs = reinterpret_cast<const QT*>(smem + Lay::kQuery + qb * Lay::kQueryOne) + cw * G * D;
+        const QT* qs = reinterpret_cast<const QT*>(smem + Lay::kQuery + qb * Lay::kQueryOne) + cw * G * Lay::kQRow;
         if constexpr (S::kMma) {
           const int g = lane >> 2, t4 = lane & 3;
           const bool row_ok = active && g < inf.heads;
 #pragma unroll
           for (int ks = 0; ks < S::kKSteps; ++ks) {
             if constexpr (EB == 2) {
-              qa[ks][0] = row_ok ? *reinterpret_cast<const uint32_t*>(qs + g * D + ks * 16 + 2 * t4) : 0u;
-              qa[ks][1] = row_ok ? *reinterpret_cast<const uint32_t*>(qs + g * D + ks * 16 + 8 + 2 * t4) : 0u;
+              qa[ks][0] = row_ok ? *reinterpret_cast<const uint32_t*>(qs + g * Lay::kQRow + ks * 16 + 2 * t4) : 0u;
+              qa[ks][1] = row_ok ? *reinterpret_cast<const uint32_t*>(qs + g * Lay::kQRow + ks * 16 + 8 + 2 * t4) : 0u;
             } else {
               // FP8 K fragments come from ldmatrix over byte rows (see the stage code): step ks holds
               // d = 16*ks + 4*t4 + {0,1} in b0 and + {2,3} in b1, so the query uses the same order.
-              const QT* qrow = qs + g * D + ks * 16 + 4 * t4;
-              qa[ks][0] = row_ok ? pack2<__half>(to_f32(qrow[0]), to_f32(qrow[1])) : 0u;
-              qa[ks][1] = row_ok ? pack2<__half>(to_f32(qrow[2]), to_f32(qrow[3])) : 0u;
+              // One 8-byte load per lane (the four values of this step), conflict-free with the padded rows.
+              if (row_ok) {
+                const uint2 raw = *reinterpret_cast<const uint2*>(qs + g * Lay::kQRow + ks * 16 + 4 * t4);
+                const QT* qrow = reinterpret_cast<const QT*>(&raw);
+                qa[ks][0] = pack2<__half>(to_f32(qrow[0]), to_f32(qrow[1]));
+                qa[ks][1] = pack2<__half>(to_f32(qrow[2]), to_f32(qrow[3]));
+              } else {
+                qa[ks][0] = qa[ks][1] = 0u;
+              }
             }
           }
 #pragma unroll
@@ -561,7 +572,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           for (int jj = 0; jj < S::kNPL; ++jj) {
             const int pc = qk_piece<S, EB>(jj, ds, tslot);
             if (active && g < inf.heads) {
-              const uint4 raw = *reinterpret_cast<const uint4*>(qs + g * D + pc * 8);
+              const uint4 raw = *reinterpret_cast<const uint4*>(qs + g * Lay::kQRow + pc * 8);
               const QT* e = reinterpret_cast<const QT*>(&raw);
 #pragma unroll
               for (int k = 0; k < 4; ++k)

@@ -223,3 +223,23 @@ def test_cache_writes_reject_rows_beyond_int_indexing(P):
     assert L.pa_reshape_and_cache(*args(1 << 24, 1 << 10)) == P.PA_ERR_UNSUPPORTED  # product overflows int
     assert L.pa_reshape_and_cache_layers(16, 16, P.PA_BF16, 16, 16, P.PA_BF16, None, None, 16, 3, 2, 1 << 24,
                                          1 << 10, 16, 4, None) == P.PA_ERR_UNSUPPORTED
+
+
+def test_probes_reject_bad_arguments(P):
+    L = P.lib
+    assert L.pa_probe_stream_read(None, 1024, 1, 16, None) == P.PA_ERR_INVALID_ARGUMENT
+    assert L.pa_probe_stream_read(16, 1000, 1, 16, None) == P.PA_ERR_INVALID_ARGUMENT      # not a multiple of 16
+    assert L.pa_probe_stream_read(24, 1024, 1, 16, None) == P.PA_ERR_INVALID_ARGUMENT      # misaligned
+    assert L.pa_probe_stream_read(16, 1024, 0, 16, None) == P.PA_ERR_INVALID_ARGUMENT      # repeat < 1
+    assert L.pa_probe_stream_read(16, 1024, 1, None, None) == P.PA_ERR_INVALID_ARGUMENT    # no sink
+    ok = dict(kc=16, vc=16, dt=P.PA_BF16, bt=16, mb=4, cl=16, S=2, Hkv=8, d=128, bs=16, NB=10, sink=16)
+
+    def paged(**over):
+        a = dict(ok, **over)
+        return L.pa_probe_paged_read(a["kc"], a["vc"], a["dt"], a["bt"], a["mb"], a["cl"], a["S"], a["Hkv"], a["d"],
+                                     a["bs"], a["NB"], a["sink"], None)
+    assert paged(S=0) == P.PA_OK
+    assert paged(kc=None) == P.PA_ERR_INVALID_ARGUMENT
+    assert paged(bt=18) == P.PA_ERR_INVALID_ARGUMENT
+    assert paged(dt=9) == P.PA_ERR_INVALID_ARGUMENT
+    assert paged(Hkv=1, d=4) == P.PA_ERR_UNSUPPORTED            # token row of 8 bytes: not 16-byte vectors

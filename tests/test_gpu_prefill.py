@@ -8,9 +8,10 @@ takes the same two steps on the same seeded inputs.
   within one KV tile and across several, whole prompts and chunks (including one-token and empty
   chunks): every output element is compared. Rows with short prefixes reach |out| of a few units, so
   each element is bounded by the stated tolerance plus half an ulp of the output dtype there.
-* The full-size workloads in the benchmark's launch configuration: the step runs whole; sampled rows
-  are recomputed by the oracle one by one (a row at position p equals a one-token chunk of the
-  context truncated to p + 1).
+* The full-size workloads in the benchmark's launch configuration: the step runs whole; every row of
+  whole sequences (the shortest prompt; for the chunked workload two adjacent sequences) is compared
+  with the oracle, and sampled rows of the rest are recomputed one by one (a row at position p equals
+  a one-token chunk of the context truncated to p + 1).
 * Contract violations (a chunk longer than its context, a block id outside the pool) set the device
   error word without faulting.
 """
@@ -137,6 +138,36 @@ def test_prefill_full_size_sampled_rows(P, name):
     ref = sampled_rows_reference(w, kc, vc, rows)
     err = np.max(np.abs(got[rows] - ref))
     assert err <= TOLERANCE[cfg.dtype], f"{name}: max-abs error {err} on {len(rows)} sampled rows"
+
+
+def whole_sequences(name, lens, q_start):
+    """Sequences whose every row is checked at full size: for the chunked workload the two adjacent
+    sequences with the smallest total context (so a sequence boundary in the query rows lies between
+    them), for the prompt workloads the shortest prompt. The oracle is fp64 and slow; these keep the
+    test to tens of seconds while covering every query tile and every diagonal tile of each sequence."""
+    if name == "chunked_prefill":
+        pair = int(np.argmin(lens[:-1] + lens[1:]))
+        return [pair, pair + 1]
+    return [int(np.argmin(lens))]
+
+
+@pytest.mark.parametrize("name", ["prefill_7b", "prefill_70b_gqa", "chunked_prefill"])
+def test_prefill_full_size_every_row_of_whole_sequences(P, name):
+    cfg = W.PREFILL_CONFIGS[name]
+    w = W.make_prefill_workload(cfg)
+    out, ws, _, _ = gpu_prefill_step(P, w)
+    torch.cuda.synchronize()
+    assert P.get_device_error(ws) == 0
+    got = out.double().cpu().numpy()
+    kc, vc = oracle_pools(w)
+    lens, q_start = w.context_lens.numpy(), w.q_start.numpy()
+    seqs = whole_sequences(name, lens, q_start)
+    rows = np.concatenate([np.arange(q_start[s], q_start[s + 1]) for s in seqs])
+    sub_start = np.concatenate([[0], np.cumsum([q_start[s + 1] - q_start[s] for s in seqs])]).astype(np.int32)
+    ref = oracle.paged_prefill(bits16(w.query)[rows], cfg.dtype, kc, vc, cfg.dtype, w.block_tables.numpy()[seqs],
+                               lens[seqs], sub_start, cfg.softmax_scale)
+    err = np.max(np.abs(got[rows] - ref))
+    assert err <= TOLERANCE[cfg.dtype], f"{name}: max-abs error {err} over every row of sequences {seqs}"
 
 
 def test_contract_violations_are_flagged(P):
