@@ -31,6 +31,7 @@ import workloads as W  # noqa: E402
 METRIC = "paged decode attention: achieved KV-read HBM GB/s & % of peak; tokens/s"
 KERNEL_SOURCES = ("pa_attention.cuh", "pa_device.cuh", "pa_launch.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "paged_attention_main_7b_traffic.json")
+MERGE_COUNTERS = 16384   # PA_MERGE_COUNTERS (include/pagedattn.h)
 THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
                  0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                  0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
@@ -341,7 +342,9 @@ def measure_decode(args, cfg, P, dev, rank, world, peak, peak_measured, checks):
             ev[1].record(stream)
 
     inputs = (w.query, w.new_key, w.new_value, w.slot_mapping, w.block_tables, w.context_lens)
-    launches_per_step = 2 + (1 if parts > 1 else 0) + (1 if w.cow_mapping.shape[0] else 0)
+    units = S * (-(-cfg.num_kv_heads // 8)) * (-(-(H // cfg.num_kv_heads) // min(8, 1 << (H // cfg.num_kv_heads - 1).bit_length())))
+    merge_kernel = parts > 1 and units > MERGE_COUNTERS    # else the attention kernel merges the partitions
+    launches_per_step = 2 + (1 if merge_kernel else 0) + (1 if w.cow_mapping.shape[0] else 0)
 
     # ---- device-resident timing: K steps back to back (the K/V read per step is larger than L2) ----
     for _ in range(args.warmup):
@@ -434,7 +437,7 @@ def measure_decode(args, cfg, P, dev, rank, world, peak, peak_measured, checks):
         "pct_of_measured_hbm_peak": round(100 * value / peak, 2),
         "pct_of_8tbs": round(100 * value / 8000.0, 2),
         "roofline": {"kernel": "paged_attention (pa_paged_attention call: main kernel%s)" %
-                     (" + split-K reduce" if parts > 1 else ""),
+                     (" + split-K reduce" if merge_kernel else (", split-K merged in-kernel" if parts > 1 else "")),
                      "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": "measured" if peak_measured else "fallback",
                      "algorithmic_bytes_per_launch": ideal["total"], "avg_launch_ms": round(attn_ms, 4),

@@ -162,7 +162,7 @@ def test_table_entries_past_the_context_are_not_used(P, name):
     """Only the first ceil(L / block_size) entries of a table row are read: poisoning the rest with
     ids outside the pool changes no output bit and sets no error bit."""
     cfg = W.CONFIGS[name]
-    w = W.make_workload(cfg, num_seqs=10, prefilled=True)
+    w = W.make_workload(cfg, num_seqs=min(10, cfg.num_seqs), prefilled=True)
     wide = poisoned_past_context(w.block_tables, w.context_lens, cfg.block_size, w.num_blocks)
     ref, ws_ref = run(P, w, write_new=False, copy=False, partition_size=cfg.partition_size)
     out, ws = run(P, w, write_new=False, copy=False, partition_size=cfg.partition_size, block_tables=wide)
