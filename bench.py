@@ -31,7 +31,6 @@ import workloads as W  # noqa: E402
 METRIC = "paged decode attention: achieved KV-read HBM GB/s & % of peak; tokens/s"
 KERNEL_SOURCES = ("pa_attention.cuh", "pa_device.cuh", "pa_launch.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "paged_attention_main_7b_traffic.json")
-MERGE_COUNTERS = 16384   # PA_MERGE_COUNTERS (include/pagedattn.h)
 THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
                  0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                  0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
@@ -201,6 +200,7 @@ def main():
     ap.add_argument("--pool-blocks", type=int, default=None,
                     help="override the pool size in blocks (profiling cases that must stay small)")
     ap.add_argument("--cpu-seconds", type=float, default=8.0)
+    ap.add_argument("--trace-out", default=None, help="trace op: also save the raw records of the last launch (.npz)")
     ap.add_argument("--no-extra-configs", action="store_true",
                     help="time only --workload (by default the 7B line also carries a 70B-GQA sub-record)")
     args = ap.parse_args()
@@ -342,9 +342,7 @@ def measure_decode(args, cfg, P, dev, rank, world, peak, peak_measured, checks):
             ev[1].record(stream)
 
     inputs = (w.query, w.new_key, w.new_value, w.slot_mapping, w.block_tables, w.context_lens)
-    units = S * (-(-cfg.num_kv_heads // 8)) * (-(-(H // cfg.num_kv_heads) // min(8, 1 << (H // cfg.num_kv_heads - 1).bit_length())))
-    merge_kernel = parts > 1 and units > MERGE_COUNTERS    # else the attention kernel merges the partitions
-    launches_per_step = 2 + (1 if merge_kernel else 0) + (1 if w.cow_mapping.shape[0] else 0)
+    launches_per_step = 2 + (1 if parts > 1 else 0) + (1 if w.cow_mapping.shape[0] else 0)
 
     # ---- device-resident timing: K steps back to back (the K/V read per step is larger than L2) ----
     for _ in range(args.warmup):
@@ -437,7 +435,7 @@ def measure_decode(args, cfg, P, dev, rank, world, peak, peak_measured, checks):
         "pct_of_measured_hbm_peak": round(100 * value / peak, 2),
         "pct_of_8tbs": round(100 * value / 8000.0, 2),
         "roofline": {"kernel": "paged_attention (pa_paged_attention call: main kernel%s)" %
-                     (" + split-K reduce" if merge_kernel else (", split-K merged in-kernel" if parts > 1 else "")),
+                     (" + split-K reduce" if parts > 1 else ""),
                      "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": "measured" if peak_measured else "fallback",
                      "algorithmic_bytes_per_launch": ideal["total"], "avg_launch_ms": round(attn_ms, 4),
@@ -707,6 +705,8 @@ def run_trace(args, cfg):
         it = it[it[:, 0] > 0]
         t0, t_end = cta[:, 0].min(), cta[:, 1].max()
         span = t_end - t0
+        if args.trace_out:
+            np.savez(args.trace_out, cta=cta, items=it, lens=lens, partition_size=ps, header=t[:8])
         ends = cta[:, 1]
         win = t_end - 0.1 * span
         busy_last10 = np.clip(ends - win, 0, None).sum() / (len(cta) * 0.1 * span)

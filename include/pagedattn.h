@@ -95,12 +95,6 @@ typedef enum pa_dtype {
 /* Bytes of the workspace header that holds the device error word (the workspace's first bytes). */
 #define PA_WORKSPACE_HEADER_BYTES 256
 
-/* Split-K completion counters (8 bytes each) that follow the header when a context is split into
- * P > 1 partitions. Calls with at most this many (sequence, 8-kv-head block, query-head subgroup)
- * units merge the partitions inside the attention kernel; larger calls merge them with a second
- * kernel. */
-#define PA_MERGE_COUNTERS 16384
-
 /*
  * Tokens per context partition that pa_paged_attention will use for these sizes.
  * partition_size > 0 requests that size (it must be a multiple of 64); 0 lets the library choose from
@@ -113,8 +107,7 @@ PA_API int pa_paged_attention_partition_size(int num_seqs, int num_heads, int nu
 /*
  * Workspace bytes pa_paged_attention needs for these sizes (same partition_size rule as above):
  * PA_WORKSPACE_HEADER_BYTES for the error word plus, when the context is split into P > 1
- * partitions, PA_MERGE_COUNTERS * 8 bytes of completion counters and fp32 partial results
- * num_seqs*num_heads*P*(head_size + 2)*4 bytes (each array rounded up to 256 bytes).
+ * partitions, fp32 partial results num_seqs*num_heads*P*(head_size + 2)*4 bytes.
  * Returns 0 if the arguments are invalid. Host only; makes no CUDA call.
  */
 PA_API size_t pa_paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_size,
@@ -142,12 +135,9 @@ PA_API size_t pa_paged_attention_workspace_size(int num_seqs, int num_heads, int
  *  max_context_len host int, >= every context_lens[s]; sizes the launch (partitions).
  *  scale          the softmax scale (1/sqrt(head_size) in the pages' formula).
  *  partition_size 0 = library's choice, else a multiple of 64 (tokens per split-K partition).
- *  workspace      device scratch of workspace_bytes >= pa_paged_attention_workspace_size(...). The
- *                 caller zeroes it once, whole, before its first use (cudaMemset); the kernels leave
- *                 their counters ready for the next call, so one workspace serves calls of any sizes
- *                 it is large enough for. Its first PA_WORKSPACE_HEADER_BYTES hold the error word,
- *                 which the kernels only OR into (clear it with pa_clear_device_error). After a call
- *                 that recorded PA_DEVERR_TIMEOUT, zero the workspace again.
+ *  workspace      device scratch of workspace_bytes >= pa_paged_attention_workspace_size(...); its
+ *                 first PA_WORKSPACE_HEADER_BYTES hold the error word, which the caller zeroes once
+ *                 (e.g. with cudaMemset or pa_clear_device_error) and the kernels only OR into.
  * Calls that share a workspace must be ordered on one stream. num_seqs == 0 is a no-op (pointers
  * may then be NULL).
  */
@@ -321,8 +311,7 @@ PA_API pa_status pa_copy_blocks_check(const int64_t* host_block_mapping, int num
 PA_API pa_status pa_get_device_error(const void* workspace, unsigned int* err_out, pa_stream_t stream);
 
 /* Zero the device error word of a workspace (enqueued on `stream`, asynchronous). Only that word: the
- * rest of the header belongs to the kernels, so never zero the header alone -- zero the whole
- * workspace, or nothing. */
+ * rest of the header holds the kernels' own counters, which they leave at zero after every call. */
 PA_API pa_status pa_clear_device_error(void* workspace, pa_stream_t stream);
 
 /*

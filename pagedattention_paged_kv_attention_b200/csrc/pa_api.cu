@@ -63,19 +63,15 @@ int plan_partition(int num_seqs, int num_heads, int num_kv_heads, int max_contex
 }
 
 struct WorkspaceLayout {
-  size_t counters, part_m, part_l, part_o, trace, total;
+  size_t part_m, part_l, part_o, trace, total;
 };
 
-// Split contexts (P > 1): the split-K completion counters sit at a fixed offset right after the header
-// (PA_MERGE_COUNTERS of 8 bytes, whatever the sizes, so that no later call's partials ever overlap an
-// earlier call's counters), then the fp32 partials.
 WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int num_kv_heads, int head_size, int partitions) {
   WorkspaceLayout w{};
   w.total = PA_WORKSPACE_HEADER_BYTES;
   if (partitions > 1) {
     const size_t rows = static_cast<size_t>(num_seqs) * num_heads * partitions;
-    w.counters = w.total;
-    w.part_m = w.counters + static_cast<size_t>(PA_MERGE_COUNTERS) * 8;
+    w.part_m = w.total;
     w.part_l = w.part_m + round_up(rows * 4, 256);
     w.part_o = w.part_l + round_up(rows * 4, 256);
     w.total = w.part_o + round_up(rows * head_size * 4, 256);
@@ -125,9 +121,7 @@ constexpr int64_t kMaxRowElems = int64_t(1) << 24;
 struct AttnPlan {
   bool empty;
   int ps, partitions, g_tile, subgroups, head_blocks;
-  unsigned long long items;  // attention work items
-  unsigned long long units;  // split-K merge units (sequence, head block, query-head subgroup)
-  bool merge_in_kernel;      // partitions merged by the attention kernel itself (else by the reduce kernel)
+  unsigned long long items;
   WorkspaceLayout ws;
 };
 
@@ -163,9 +157,7 @@ pa_status check_attention(const void* out, const void* query, pa_dtype q_dtype, 
   group_tiling(num_heads / num_kv_heads, &plan->g_tile, &plan->subgroups);
   plan->head_blocks = ceil_div(num_kv_heads, pa::kHeadBlock);
   plan->items = static_cast<unsigned long long>(plan->partitions) * num_seqs * plan->head_blocks * plan->subgroups;
-  plan->units = static_cast<unsigned long long>(num_seqs) * plan->head_blocks * plan->subgroups;
-  plan->merge_in_kernel = plan->partitions > 1 && plan->units <= PA_MERGE_COUNTERS;
-  if (num_seqs > 65535 || plan->items + plan->units > 0x7fffffffULL) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > 65535 || plan->items > 0x7fffffffULL) return PA_ERR_UNSUPPORTED;
   plan->ws = workspace_layout(num_seqs, num_heads, num_kv_heads, head_size, plan->partitions);
   return PA_OK;
 }
@@ -278,14 +270,12 @@ pa_status pa_paged_attention(void* out, const void* query, pa_dtype q_dtype, con
   a.partition_size = ps;
   a.num_partitions = partitions;
   a.num_items = static_cast<unsigned int>(items);
-  a.unit_done = plan.merge_in_kernel ? reinterpret_cast<unsigned long long*>(wsb + ws.counters) : nullptr;
-  a.num_tickets = static_cast<unsigned int>(items + (plan.merge_in_kernel ? plan.units : 0));
   a.scale_log2 = scale * pa::kLog2e;
   a.scale_block_stride = scale_block_stride(kv_dtype, num_kv_heads);
 #ifdef PA_TRACE
   a.trace = reinterpret_cast<unsigned long long*>(wsb + ws.trace);
 #endif
-  const int grid = static_cast<int>(std::min<unsigned long long>(static_cast<unsigned long long>(sms), a.num_tickets));
+  const int grid = static_cast<int>(std::min<unsigned long long>(static_cast<unsigned long long>(sms), items));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = q_dtype == PA_BF16 ? pa::launch_attention_bf16(tk, tv, a, fp8, head_size, g_tile, grid, st)
                                      : pa::launch_attention_f16(tk, tv, a, fp8, head_size, g_tile, grid, st);
@@ -490,7 +480,7 @@ pa_status pa_get_device_error(const void* workspace, unsigned int* err_out, pa_s
 pa_status pa_clear_device_error(void* workspace, pa_stream_t stream) {
   if (!workspace || !aligned(workspace, 16)) return PA_ERR_INVALID_ARGUMENT;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // The error word only: the header's other words are the kernels' own (work counter, launch count).
+  // The error word only: the header's other words are the kernels' own (work and finished-CTA counters).
   return cudaMemsetAsync(workspace, 0, sizeof(unsigned int), st) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

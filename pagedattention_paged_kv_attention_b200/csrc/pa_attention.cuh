@@ -60,15 +60,10 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kPartitionQuantum = 64;    // partition sizes are multiples of this
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Workspace header words: error bits, work counter, finished-CTA counter, launch count (the tag of the
-// split-K merge counters).
+// Workspace header words: error bits, work counter, finished-CTA counter.
 constexpr int kWsError = 0;
 constexpr int kWsWork = 1;
 constexpr int kWsDone = 2;
-constexpr int kWsLaunch = 3;
-// Stage-message item values: the end of work, and a split-K merge (no data in the slot).
-constexpr int kItemEnd = -1;
-constexpr int kItemMerge = -2;
 
 // Stage message flags.
 constexpr int kMsgFirst = 1;
@@ -98,10 +93,7 @@ struct AttnArgs {
   int num_blocks;
   int partition_size;           // tokens per partition, multiple of kPartitionQuantum
   int num_partitions;
-  unsigned int num_items;       // attention items: num_partitions * num_seqs * head_blocks * subgroups
-  unsigned int num_tickets;     // num_items, plus one merge ticket per unit when unit_done is set
-  unsigned long long* unit_done;  // split-K completion counters, one per unit (sequence, head block,
-                                  // subgroup); null: the partitions are merged by the reduce kernel
+  unsigned int num_items;       // num_partitions * num_seqs * head_blocks * subgroups
   float scale_log2;             // softmax scale * log2(e)
   int scale_block_stride;       // FP8 scales: 0 = per kv head, num_kv_heads = per (block, kv head)
   unsigned long long* trace;    // timing records, written only by builds with PA_TRACE defined (else null)
@@ -268,58 +260,6 @@ __device__ __forceinline__ bool context_len_invalid(int L, const AttnArgs& a) {
   return L < 0 || L > a.max_blocks_per_seq * a.block_size || L > a.num_partitions * a.partition_size;
 }
 
-// Merge unit of an attention item: (sequence, head block, query-head subgroup).
-__device__ __forceinline__ unsigned int merge_unit(int s, int hb, int sub, const AttnArgs& a) {
-  return (static_cast<unsigned int>(s) * a.head_blocks + hb) * a.subgroups + sub;
-}
-
-// Launch tag of the merge counters (never zero).
-__device__ __forceinline__ unsigned int launch_tag(const AttnArgs& a) {
-  return (__ldcg(a.header + kWsLaunch) & 0x7fffffffu) | 0x80000000u;
-}
-
-// Log-sum-exp merge of one output row's partitions: out = sum_p w_p o_p / sum_p w_p with
-// w_p = l_p 2^(m_p - max m). One warp; lanes hold D/32 consecutive elements. The partials were written
-// by other CTAs of this launch, so they are read through L2 (__ldcg), never a stale L1 line.
-template <typename QT, int D>
-__device__ __forceinline__ void merge_partitions(const AttnArgs& a, size_t row, int n_parts, int lane) {
-  constexpr int kPer = D / 32;
-  const size_t base = row * a.num_partitions;
-  float M = -INFINITY;
-  for (int p = lane; p < n_parts; p += 32) M = fmaxf(M, __ldcg(a.part_m + base + p));
-#pragma unroll
-  for (int b = 16; b > 0; b >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, b));
-  float wsum = 0.f;
-  float acc[kPer];
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-  const float* po = a.part_o + base * D + lane * kPer;
-  for (int p0 = 0; p0 < n_parts; p0 += 32) {
-    const int p = p0 + lane;
-    const float w_lane = p < n_parts ? __ldcg(a.part_l + base + p) * fast_exp2(__ldcg(a.part_m + base + p) - M) : 0.f;
-    const int cnt = min(32, n_parts - p0);
-#pragma unroll 8
-    for (int i = 0; i < cnt; ++i) {
-      const float w = __shfl_sync(0xffffffffu, w_lane, i);
-      wsum += w;
-      if constexpr (kPer == 4) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(po + static_cast<size_t>(p0 + i) * D));
-        acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
-      } else {
-        const float2 v = __ldcg(reinterpret_cast<const float2*>(po + static_cast<size_t>(p0 + i) * D));
-        acc[0] += w * v.x; acc[1] += w * v.y;
-      }
-    }
-  }
-  const float r = 1.0f / wsum;
-  QT* out = static_cast<QT*>(a.out) + row * D + lane * kPer;
-  if constexpr (kPer == 4) {
-    *reinterpret_cast<uint2*>(out) = pack4<QT>(acc[0] * r, acc[1] * r, acc[2] * r, acc[3] * r);
-  } else {
-    *reinterpret_cast<uint32_t*>(out) = pack2<QT>(acc[0] * r, acc[1] * r);
-  }
-}
-
 // BS: FP8 cache with per-(block, kv head) scales (args.scale_block_stride != 0); a separate
 // instantiation so that the per-head FP8 path carries none of its work.
 template <typename QT, typename KVT, int D, int G, bool BS>
@@ -397,9 +337,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     int cur_ids[kIdWindow], nxt_ids[kIdWindow];
 #define PA_PREPARE(IDX, LV, IDS)                                                                       \
   do {                                                                                                 \
-    if ((IDX) >= args.num_items && (IDX) < args.num_tickets) {                                         \
-      LV = __ldg(args.context_lens + ((IDX) - args.num_items) / (args.head_blocks * args.subgroups));   \
-    } else if ((IDX) < args.num_items) {                                                               \
+    if ((IDX) < args.num_items) {                                                                      \
       const ItemCoord pc_ = decode_item((IDX), args);                                                  \
       LV = __ldg(args.context_lens + pc_.s);                                                           \
       const int need_ = LV <= 0 ? 0 : cmin(args.max_blocks_per_seq, LV / bs + (LV % bs != 0));         \
@@ -416,37 +354,10 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     cur_idx = __shfl_sync(0xffffffffu, ticket, 0);
     PA_PREPARE(cur_idx, cur_L, cur_ids);
     if (lane == 0) ticket = atomicAdd(args.header + kWsWork, 1u);
-    while (!aborted && cur_idx < args.num_tickets) {
+    while (!aborted && cur_idx < args.num_items) {
       nxt_idx = __shfl_sync(0xffffffffu, ticket, 0);
       PA_PREPARE(nxt_idx, nxt_L, nxt_ids);
       if (lane == 0) ticket = atomicAdd(args.header + kWsWork, 1u);
-      if (cur_idx >= args.num_items) {
-        // Split-K merge ticket (they follow every attention ticket): one message, no data. Units whose
-        // sequence has one partition (or an empty or invalid context) were finished by its item.
-        const unsigned int u = cur_idx - args.num_items;
-        const int L = cur_L;
-        const int n_parts = (L <= 0 || context_len_invalid(L, args)) ? 1 : (L + args.partition_size - 1) / args.partition_size;
-        if (n_parts > 1) {
-          const int slot = issued % kStages;
-          bool ok2 = true;
-          if (lane == 0) ok2 = mbar_wait(&empty[slot], (static_cast<uint32_t>(issued / kStages) & 1u) ^ 1u, err);
-          if (!__shfl_sync(0xffffffffu, ok2, 0)) {
-            aborted = true;
-            break;
-          }
-          if (lane == 0) {
-            msgs[slot] = StageMsg{kItemMerge, n_parts, 0, static_cast<int>(u)};
-            mbar_arrive(&full[slot]);
-          }
-          __syncwarp();
-          ++issued;
-        }
-        cur_idx = nxt_idx;
-        cur_L = nxt_L;
-#pragma unroll
-        for (int j = 0; j < kIdWindow; ++j) cur_ids[j] = nxt_ids[j];
-        continue;
-      }
       const ItemCoord c = decode_item(cur_idx, args);
       const int L = cur_L;
       const bool bad_len = context_len_invalid(L, args);
@@ -580,7 +491,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
       bool ok = true;
       if (lane == 0) ok = mbar_wait(&empty[slot], (static_cast<uint32_t>(issued / kStages) & 1u) ^ 1u, err);
       if (__shfl_sync(0xffffffffu, ok, 0) && lane == 0) {
-        msgs[slot] = StageMsg{kItemEnd, 0, 0, 0};
+        msgs[slot] = StageMsg{-1, 0, 0, 0};
         mbar_arrive(&full[slot]);
       }
       ++issued;
@@ -611,41 +522,12 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     bool active = false;  // this warp's kv head exists in the current item
     float zitem = 0.f;    // per-head FP8: scale_log2 * k_scale of this warp's kv head for the item
     ItemInfo inf{};
-    const unsigned int tag = args.unit_done ? launch_tag(args) : 0u;
 
     for (int j = 0;; ++j) {
       const int slot = j % kStages;
       if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], static_cast<uint32_t>(j / kStages) & 1u, err))) break;
       const StageMsg m = msgs[slot];
-      if (m.item == kItemEnd) break;
-      if (m.item == kItemMerge) {
-        // Split-K merge of one unit: this warp merges the rows of its kv head once every partition of
-        // the unit has been written (n_parts items x the unit's kv heads completions).
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[slot]);
-        const unsigned int u = static_cast<unsigned int>(m.blk1);
-        const int per_seq = args.head_blocks * args.subgroups;
-        const int ms = static_cast<int>(u / per_seq);
-        const int mr = static_cast<int>(u % per_seq);
-        const int mkvh0 = (mr / args.subgroups) * kHeadBlock;
-        const int mh_sub = (mr % args.subgroups) * G;
-        const int mkv_here = cmin(kHeadBlock, args.num_kv_heads - mkvh0);
-        if (cw < mkv_here) {
-          const unsigned long long want =
-              (static_cast<unsigned long long>(tag) << 32) | static_cast<unsigned int>(m.ntok * mkv_here);
-          bool ok = true;
-          if (lane == 0) ok = wait_tagged_count(args.unit_done + u, want, err);
-          if (__shfl_sync(0xffffffffu, ok, 0)) {
-            (void)ld_acquire_u64(args.unit_done + u);  // every lane acquires (the count is final)
-            const int mheads = cmin(G, args.group - mh_sub);
-            for (int g = 0; g < mheads; ++g)
-              merge_partitions<QT, D>(args,
-                                      static_cast<size_t>(ms) * args.num_heads + (mkvh0 + cw) * args.group + mh_sub + g,
-                                      m.ntok, lane);
-          }
-        }
-        continue;
-      }
+      if (m.item < 0) break;
       if (m.flags & kMsgFirst) {
         // New item: load this head's query rows and reset the state.
         const int qb = m.item % kQueryBuffers;
@@ -1041,19 +923,10 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           }
         }
       }
-      // A partial result of a split context: count it on its unit once every lane's writes are visible
-      // (each lane fences, then the warp synchronises, then one lane counts).
-      if (args.unit_done && (m.flags & kMsgLast) && active && !inf.write_final) {
-        __threadfence();
-        __syncwarp();
-        if (lane == 0)
-          tagged_count(args.unit_done + merge_unit(inf.s, inf.kvh0 / kHeadBlock, inf.h_sub / G, args), tag, err);
-      }
     }
   }
 
-  // The last CTA to finish resets the work counter for the next launch on this workspace and advances
-  // the launch count (the next launch's counter tag).
+  // The last CTA to finish resets the work counter for the next launch on this workspace.
   __syncthreads();
 #ifdef PA_TRACE
   if (threadIdx.x == 0 && blockIdx.x < kTraceMaxCtas) args.trace[kTraceCtaBase + 4 * blockIdx.x + 1] = global_timer_ns();
@@ -1064,7 +937,6 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     if (done == gridDim.x - 1) {
       atomicExch(args.header + kWsWork, 0u);
       atomicExch(args.header + kWsDone, 0u);
-      atomicAdd(args.header + kWsLaunch, 1u);
     }
   }
 }

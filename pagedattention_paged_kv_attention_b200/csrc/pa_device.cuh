@@ -83,46 +83,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
 }
 
 // ------------------------------------------------------------------------------------------------
-// Completion counters shared by the CTAs of one launch (split-K merge). A counter's high word holds
-// the launch's tag and its low word a count; a counter whose tag is not this launch's (zero, or left
-// by an earlier launch) counts as zero, so counters never need resetting.
-// ------------------------------------------------------------------------------------------------
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Adds one completion to *c under `tag` (relaxed CAS; the caller fences its data writes first).
-__device__ __forceinline__ void tagged_count(unsigned long long* c, unsigned int tag, unsigned int* error_word) {
-  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(c);
-  for (int i = 0; i < (1 << 20); ++i) {
-    const unsigned long long want = static_cast<unsigned int>(cur >> 32) == tag
-                                        ? cur + 1ull
-                                        : ((static_cast<unsigned long long>(tag) << 32) | 1ull);
-    const unsigned long long prev = atomicCAS(c, cur, want);
-    if (prev == cur) return;
-    cur = prev;
-  }
-  atomicOr(error_word, PA_DEVERR_TIMEOUT);  // a CAS that never wins: give up instead of spinning
-}
-
-// Bounded wait until *c == want, with acquire ordering. false (and PA_DEVERR_TIMEOUT) after limit_ns.
-__device__ __forceinline__ bool wait_tagged_count(const unsigned long long* c, unsigned long long want,
-                                                  unsigned int* error_word, uint64_t limit_ns = kWaitLimitNs) {
-  if (ld_acquire_u64(c) == want) return true;
-  const uint64_t start = global_timer_ns();
-  for (uint32_t spin = 0;; ++spin) {
-    __nanosleep(128);
-    if (ld_acquire_u64(c) == want) return true;
-    if ((spin & 15u) == 15u && global_timer_ns() - start > limit_ns) {
-      atomicOr(error_word, PA_DEVERR_TIMEOUT);
-      return false;
-    }
-  }
-}
-
-// ------------------------------------------------------------------------------------------------
 // TMA: 4-D tiled load global -> shared, completion counted on an mbarrier (no multicast).
 // ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -22,7 +22,7 @@ cudaError_t launch_attention_one(const CUtensorMap& tk, const CUtensorMap& tv, c
   if (e != cudaSuccess) return e;
   e = pa_host::launch_overlapped(kernel, dim3(grid), dim3(kThreads), smem, stream, tk, tv, a);
   if (e != cudaSuccess) return e;
-  if (a.num_partitions > 1 && a.unit_done == nullptr) {  // merges not done by the main kernel
+  if (a.num_partitions > 1) {
     const long rows = static_cast<long>(a.num_heads) * a.num_seqs;
     e = pa_host::launch_overlapped(paged_attention_reduce<QT, D>,
                                    dim3(static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps)),

@@ -19,7 +19,6 @@ LIBRARY_PATH = os.environ.get("PA_LIBRARY_PATH") or os.path.join(_HERE, "libpage
  PA_ERR_HOST_MEMORY) = range(7)
 PA_F16, PA_BF16, PA_FP8_E4M3, PA_FP8_E4M3_BLOCK = 0, 1, 2, 3
 PA_DEVERR_BLOCK_ID, PA_DEVERR_CONTEXT_LEN, PA_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
-MERGE_COUNTERS = 16384   # PA_MERGE_COUNTERS: split-K units merged inside the attention kernel
 WORKSPACE_HEADER_BYTES = 256
 
 # Every symbol the public header declares (checked by the CPU test suite).

@@ -66,37 +66,6 @@ def test_split_k_partition_sizes(P, partition_size):
     assert P.get_device_error(ws) == 0
 
 
-def test_split_k_beyond_the_counter_capacity_uses_the_merge_kernel(P):
-    """A batch with more split-K units (sequence, 8-kv-head block, query-head subgroup) than the
-    workspace's PA_MERGE_COUNTERS is merged by the second kernel instead of inside the attention
-    kernel. The oracle checks a sample of its sequences; the same sequences run as a small batch (merged
-    in-kernel) must give bitwise the same rows, since both merges take the same arithmetic steps."""
-    S, Hkv, G = 5462, 8, 24                                   # 3 subgroups of 8 query heads: 16386 units
-    assert S * ((G + 7) // 8) > P.MERGE_COUNTERS
-    rng = np.random.default_rng(5462)
-    lens = rng.integers(65, 73, size=S)                       # two partitions of 64 tokens each
-    cfg = W.Config(name="units", description="many split-K units", num_seqs=S, num_heads=Hkv * G, num_kv_heads=Hkv,
-                   head_size=64, block_size=8, dtype="bf16", kv_dtype="bf16", seed=91, context_lens=tuple(lens))
-    w = W.make_workload(cfg, prefilled=True)
-    kc, vc = to_device_pool(bits16(w.key_values), cfg), to_device_pool(bits16(w.value_values), cfg)
-    out, ws = gpu_step(P, w, kc, vc, write_new=False, copy=False, partition_size=64)
-    torch.cuda.synchronize()
-    assert P.get_device_error(ws) == 0
-    sample = np.sort(rng.choice(S, size=24, replace=False))
-    ref = oracle.paged_attention(bits16(w.query)[sample], cfg.dtype, bits16(w.key_values), bits16(w.value_values),
-                                 cfg.kv_dtype, w.block_tables.numpy()[sample], w.context_lens.numpy()[sample],
-                                 cfg.softmax_scale)
-    assert max_abs_err(out[torch.from_numpy(sample).cuda()], ref) <= TOLERANCE["bf16"]
-    small = torch.empty_like(out[:24])
-    idx = torch.from_numpy(sample).cuda()
-    ws_small = P.make_workspace(24, cfg.num_heads, Hkv, 64, int(w.context_lens.max()), 64)
-    P.paged_attention(small, w.query.cuda()[idx].contiguous(), kc, vc, w.block_tables.cuda()[idx].contiguous(),
-                      w.context_lens.cuda()[idx].contiguous(), cfg.softmax_scale, int(w.context_lens.max()), ws_small,
-                      partition_size=64)
-    torch.cuda.synchronize()
-    assert torch.equal(small.view(torch.int16), out[idx].view(torch.int16))
-
-
 def small_case(kv_dtype, dtype, head_size, block_size, H, Hkv, lens, seed):
     cfg = W.Config(name="case", description="ragged parity case", num_seqs=len(lens), num_heads=H,
                    num_kv_heads=Hkv, head_size=head_size, block_size=block_size, dtype=dtype,
