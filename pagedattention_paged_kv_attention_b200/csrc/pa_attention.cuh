@@ -58,6 +58,10 @@ constexpr int kQueryBuffers = 2;
 constexpr int kIdWindow = 4;             // block ids prefetched per item: 32 * kIdWindow stages
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kPartitionQuantum = 64;    // partition sizes are multiples of this
+constexpr int kOrderMaxSeqs = 1024;      // batches up to this size take their items longest first
+constexpr int kOrderMaxRounds = 128;     // ... when the context splits into at most this many partitions
+constexpr int kRemBins = 128;            // partial partitions are ordered by size in this many bins
+constexpr int kClaimAhead = 4;           // the next item is claimed when this many stages remain to issue
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Workspace header words: error bits, work counter, finished-CTA counter.
@@ -159,6 +163,20 @@ struct ItemInfo {
   int s, part, kvh0, h_sub, heads, write_final, pad0, pad1;  // h_sub: first query-head offset in a group
 };
 
+// Work order of one launch, built by every CTA from the context lengths (the same table in each):
+// first the full partitions round by round (round r = partition r of every sequence that has more
+// than r full partitions, sequences with more full partitions first), then each sequence's last,
+// partial partition (or the single item of an empty or invalid context), largest first. Tickets map
+// one to one onto real items, and the smallest items come last.
+struct OrderTable {
+  uint16_t full[kOrderMaxSeqs];          // sequences by full-partition count, descending
+  uint16_t part[kOrderMaxSeqs];          // sequences with a partial item, by its size, descending
+  int round_start[kOrderMaxRounds + 1];  // round r's first index into `full`-ordered items
+  int nf_cursor[kOrderMaxRounds + 1];    // counting-sort cursors by full-partition count
+  int rem_cursor[kRemBins];              // counting-sort cursors by partial size
+  int ok, full_items, part_items, pad;
+};
+
 // Shared-memory layout (byte offsets from the 1024-aligned base).
 template <typename QT, int D, int G, int EB>
 struct Layout {
@@ -181,7 +199,8 @@ struct Layout {
   static constexpr int kBars = (kInfo + kQueryBuffers * int(sizeof(ItemInfo)) + 7) / 8 * 8;
   // full[kStages], empty[kStages], qfull[NQ], qempty[NQ]
   static constexpr int kNumBars = 2 * kStages + 2 * kQueryBuffers;
-  static constexpr int kEnd = kBars + kNumBars * 8;
+  static constexpr int kOrder = (kBars + kNumBars * 8 + 15) / 16 * 16;
+  static constexpr int kEnd = kOrder + int(sizeof(OrderTable));
   static constexpr int kAllocBytes = kEnd + 1024;  // alignment slack
   static_assert(kAllocBytes <= 227 * 1024, "shared memory layout too large");
 };
@@ -260,6 +279,133 @@ __device__ __forceinline__ bool context_len_invalid(int L, const AttnArgs& a) {
   return L < 0 || L > a.max_blocks_per_seq * a.block_size || L > a.num_partitions * a.partition_size;
 }
 
+// How a sequence enters the work order: its full partitions, whether it has one more item (a partial
+// last partition, or the single item of an empty or invalid context), and that item's size bin.
+struct SeqClass {
+  int nf, pr, bin;
+};
+__device__ __forceinline__ SeqClass classify_seq(int L, const AttnArgs& a) {
+  const bool valid = L > 0 && !context_len_invalid(L, a);
+  const int ps = a.partition_size;
+  SeqClass c;
+  c.nf = valid ? L / ps : 0;
+  const int rem = valid ? L % ps : 0;
+  c.pr = (!valid || rem != 0) ? 1 : 0;
+  c.bin = static_cast<int>((static_cast<long long>(rem) * kRemBins) / ps);
+  return c;
+}
+
+// Exclusive scan of v[0..n) (n <= 32 * 5) by one warp, in place; returns the total.
+__device__ __forceinline__ int warp_exclusive_scan(int* v, int n, int lane) {
+  constexpr int kPer = 5;
+  int local[kPer];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int idx = lane * kPer + i;
+    local[i] = idx < n ? v[idx] : 0;
+    sum += local[i];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  int run = incl - sum;
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int idx = lane * kPer + i;
+    if (idx < n) v[idx] = run;
+    run += local[i];
+  }
+  __syncwarp();
+  return total;
+}
+
+// Builds the work order (one warp). Counting sorts with ranks taken in sequence order (match_any),
+// so every CTA builds the same table. Leaves ok = 0 when the batch is too large for the table.
+__device__ __noinline__ static void build_order(OrderTable* ot, const AttnArgs& a, int lane) {
+  const int S = a.num_seqs, P = a.num_partitions;
+  if (S > kOrderMaxSeqs || P > kOrderMaxRounds) {
+    if (lane == 0) ot->ok = 0;
+    __syncwarp();
+    return;
+  }
+  // Histograms, highest count first: index P - nf and kRemBins - 1 - bin.
+  for (int i = lane; i <= P; i += 32) ot->nf_cursor[i] = 0;
+  for (int i = lane; i < kRemBins; i += 32) ot->rem_cursor[i] = 0;
+  __syncwarp();
+  for (int s = lane; s < S; s += 32) {
+    const SeqClass c = classify_seq(__ldg(a.context_lens + s), a);
+    atomicAdd(&ot->nf_cursor[P - c.nf], 1);
+    if (c.pr) atomicAdd(&ot->rem_cursor[kRemBins - 1 - c.bin], 1);
+  }
+  __syncwarp();
+  // Round r holds the sequences with more than r full partitions: nf_cursor (after the scan) at index
+  // P - r is how many sequences have more than r of them.
+  const int part_items = warp_exclusive_scan(ot->rem_cursor, kRemBins, lane);
+  warp_exclusive_scan(ot->nf_cursor, P + 1, lane);
+  for (int r = lane; r < P; r += 32) ot->round_start[r] = ot->nf_cursor[P - r];  // sequences in round r
+  __syncwarp();
+  const int full_items = warp_exclusive_scan(ot->round_start, P, lane);
+  if (lane == 0) {
+    ot->round_start[P] = full_items;
+    ot->full_items = full_items;
+    ot->part_items = part_items;
+    ot->ok = 1;
+  }
+  __syncwarp();
+  // Scatter in sequence order: lanes with the same key take consecutive places, by lane.
+  const unsigned lt = (1u << lane) - 1u;
+  for (int s0 = 0; s0 < S; s0 += 32) {
+    const int s = s0 + lane;
+    const bool in = s < S;
+    const SeqClass c = classify_seq(in ? __ldg(a.context_lens + s) : 0, a);
+    const int kf = in ? P - c.nf : -1;
+    const unsigned peers_f = __match_any_sync(0xffffffffu, kf);
+    const int base_f = in ? ot->nf_cursor[kf] : 0;
+    const int kr = (in && c.pr) ? kRemBins - 1 - c.bin : -1;
+    const unsigned peers_r = __match_any_sync(0xffffffffu, kr);
+    const int base_r = kr >= 0 ? ot->rem_cursor[kr] : 0;
+    __syncwarp();
+    if (in) {
+      ot->full[base_f + __popc(peers_f & lt)] = static_cast<uint16_t>(s);
+      if ((peers_f & lt) == 0) ot->nf_cursor[kf] = base_f + __popc(peers_f);
+    }
+    if (kr >= 0) {
+      ot->part[base_r + __popc(peers_r & lt)] = static_cast<uint16_t>(s);
+      if ((peers_r & lt) == 0) ot->rem_cursor[kr] = base_r + __popc(peers_r);
+    }
+    __syncwarp();
+  }
+}
+
+// Ticket -> item under the work order. part = -1 marks a sequence's last item, whose partition index
+// follows from its length (partial partition, or 0 for an empty or invalid context).
+__device__ __forceinline__ ItemCoord decode_ordered(unsigned int t, const AttnArgs& a, const OrderTable* ot) {
+  const unsigned int per = static_cast<unsigned int>(a.head_blocks) * a.subgroups;
+  const unsigned int q = t / per, r = t - q * per;
+  ItemCoord c;
+  c.hb = static_cast<int>(r / a.subgroups);
+  c.sub = static_cast<int>(r - static_cast<unsigned int>(c.hb) * a.subgroups);
+  if (q < static_cast<unsigned int>(ot->full_items)) {
+    int lo = 0, hi = a.num_partitions - 1;  // the last round whose start is <= q
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (static_cast<unsigned int>(ot->round_start[mid]) <= q) lo = mid; else hi = mid - 1;
+    }
+    c.part = lo;
+    c.s = ot->full[q - ot->round_start[lo]];
+  } else {
+    c.part = -1;
+    c.s = ot->part[q - ot->full_items];
+  }
+  return c;
+}
+
 // BS: FP8 cache with per-(block, kv head) scales (args.scale_block_stride != 0); a separate
 // instantiation so that the per-head FP8 path carries none of its work.
 template <typename QT, typename KVT, int D, int G, bool BS>
@@ -310,6 +456,8 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     args.trace[kTraceCtaBase + 4 * blockIdx.x + 3] = smid;
   }
 #endif
+  OrderTable* order = reinterpret_cast<OrderTable*>(smem + Lay::kOrder);
+  if (warp == 0) build_order(order, args, lane);
   __syncthreads();
 
   if (warp == 0) {
@@ -327,38 +475,52 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     int local = 0;   // CTA-local item sequence number
     int issued = 0;  // stages issued so far (ring position)
 
-    // Items flow through a two-deep software pipeline: while item i streams, the loads describing item
-    // i+1 (its context length and a window of its block ids, one id per lane per 32 boxes) are in
-    // flight, and the work counter has already been asked for item i+2. All state is in registers.
-    // Only the table entries the context needs (the first ceil(L / block_size), at most the table's
-    // width) are ever read; the rest of the window holds 0 and is never used.
+    // The next item is claimed late -- when kClaimAhead stages of the current one remain to be issued --
+    // so that a CTA holds at most a few stages of unstarted work while others may run dry; its context
+    // length and a window of its block ids (one id per lane per 32 boxes) are loaded while those stages
+    // issue. Only the table entries the context needs (the first ceil(L / block_size), at most the
+    // table's width) are ever read; the rest of the window holds 0 and is never used.
+    const bool ordered = order->ok != 0;
+    const unsigned int num_tickets = ordered
+        ? static_cast<unsigned int>(order->full_items + order->part_items) * args.head_blocks * args.subgroups
+        : args.num_items;
     unsigned int cur_idx = 0, nxt_idx = 0;
+    ItemCoord cur_c{}, nxt_c{};
     int cur_L = 0, nxt_L = 0;
     int cur_ids[kIdWindow], nxt_ids[kIdWindow];
-#define PA_PREPARE(IDX, LV, IDS)                                                                       \
+    bool have_next = false;
+#define PA_PREPARE(IDX, C, LV, IDS)                                                                    \
   do {                                                                                                 \
-    if ((IDX) < args.num_items) {                                                                      \
-      const ItemCoord pc_ = decode_item((IDX), args);                                                  \
-      LV = __ldg(args.context_lens + pc_.s);                                                           \
+    if ((IDX) < num_tickets) {                                                                         \
+      C = ordered ? decode_ordered((IDX), args, order) : decode_item((IDX), args);                     \
+      LV = __ldg(args.context_lens + C.s);                                                             \
+      if (C.part < 0) C.part = (LV > 0 && !context_len_invalid(LV, args)) ? (LV - 1) / args.partition_size : 0; \
       const int need_ = LV <= 0 ? 0 : cmin(args.max_blocks_per_seq, LV / bs + (LV % bs != 0));         \
-      const int32_t* row_ = args.block_tables + static_cast<size_t>(pc_.s) * args.max_blocks_per_seq;  \
+      const int32_t* row_ = args.block_tables + static_cast<size_t>(C.s) * args.max_blocks_per_seq;    \
       _Pragma("unroll") for (int j_ = 0; j_ < kIdWindow; ++j_) {                                       \
-        const int entry_ = ((pc_.part * boxes_per_part + j_ * 32 + lane) * kBoxTokens) / bs;           \
+        const int entry_ = ((C.part * boxes_per_part + j_ * 32 + lane) * kBoxTokens) / bs;             \
         IDS[j_] = entry_ < need_ ? __ldg(row_ + entry_) : 0;                                           \
       }                                                                                                \
     }                                                                                                  \
   } while (0)
+#define PA_CLAIM_NEXT()                                                                                \
+  do {                                                                                                 \
+    unsigned int t_ = 0;                                                                               \
+    if (lane == 0) t_ = atomicAdd(args.header + kWsWork, 1u);                                          \
+    nxt_idx = __shfl_sync(0xffffffffu, t_, 0);                                                         \
+    PA_PREPARE(nxt_idx, nxt_c, nxt_L, nxt_ids);                                                        \
+    have_next = true;                                                                                  \
+  } while (0)
 
-    unsigned int ticket = 0;
-    if (lane == 0) ticket = atomicAdd(args.header + kWsWork, 1u);
-    cur_idx = __shfl_sync(0xffffffffu, ticket, 0);
-    PA_PREPARE(cur_idx, cur_L, cur_ids);
-    if (lane == 0) ticket = atomicAdd(args.header + kWsWork, 1u);
-    while (!aborted && cur_idx < args.num_items) {
-      nxt_idx = __shfl_sync(0xffffffffu, ticket, 0);
-      PA_PREPARE(nxt_idx, nxt_L, nxt_ids);
-      if (lane == 0) ticket = atomicAdd(args.header + kWsWork, 1u);
-      const ItemCoord c = decode_item(cur_idx, args);
+    {
+      unsigned int t0 = 0;
+      if (lane == 0) t0 = atomicAdd(args.header + kWsWork, 1u);
+      cur_idx = __shfl_sync(0xffffffffu, t0, 0);
+      PA_PREPARE(cur_idx, cur_c, cur_L, cur_ids);
+    }
+    while (!aborted && cur_idx < num_tickets) {
+      have_next = false;
+      const ItemCoord c = cur_c;
       const int L = cur_L;
       const bool bad_len = context_len_invalid(L, args);
       const int n_parts = bad_len ? 1 : (L + args.partition_size - 1) / args.partition_size;
@@ -423,7 +585,9 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           const int op_box = lane / (2 * S::kChunks);
           const int op_kv = (lane / S::kChunks) & 1;
           const int op_ch = lane % S::kChunks;
+          const int claim_at = cmax(0, n_stages - kClaimAhead);
           for (int k = 0; k < n_stages; ++k) {
+            if (k == claim_at) PA_CLAIM_NEXT();
             const int t0 = tok_begin + k * S::kTS;
             const int ntok = cmin(S::kTS, tok_end - t0);
             const int nbox = (ntok + kBoxTokens - 1) / kBoxTokens;
@@ -479,11 +643,15 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           ++local;
         }
       }
+      if (aborted) break;
+      if (!have_next) PA_CLAIM_NEXT();  // items without stages (empty, invalid or past the context)
       cur_idx = nxt_idx;
+      cur_c = nxt_c;
       cur_L = nxt_L;
 #pragma unroll
       for (int j = 0; j < kIdWindow; ++j) cur_ids[j] = nxt_ids[j];
     }
+#undef PA_CLAIM_NEXT
 #undef PA_PREPARE
     // No work left: one terminating message.
     if (!aborted) {
