@@ -488,16 +488,27 @@ def run_prefill(args, cfg, world, rank):
     H, d = cfg.num_heads, cfg.head_size
     flops = 4.0 * d * H * w.causal_pairs()
     key_cache, value_cache = w.key_values, w.value_values
+    ks = vs = None
+    if cfg.cache_dtype.startswith("fp8"):
+        # The product's own quantiser fills the FP8 pools from the drawn values.
+        NB, bs, Hkv, _ = key_cache.shape
+        ks, vs = w.k_scale.to(dev), w.v_scale.to(dev)
+        kq = torch.empty((NB, bs, Hkv, d), dtype=torch.uint8, device=dev)
+        vq = torch.empty_like(kq)
+        slots = torch.arange(NB * bs, dtype=torch.int64, device=dev)
+        P.reshape_and_cache(key_cache.view(NB * bs, Hkv, d), value_cache.view(NB * bs, Hkv, d), kq, vq, slots, ks, vs)
+        key_cache, value_cache = kq, vq
+        del slots
     out = torch.empty_like(w.query)
     ws = torch.zeros(64, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
     mq = w.max_q_len
 
     def step(q, nk, nv, slots, tables, lens, qs, o, ev=None):
-        P.reshape_and_cache(nk, nv, key_cache, value_cache, slots)
+        P.reshape_and_cache(nk, nv, key_cache, value_cache, slots, ks, vs)
         if ev is not None:
             ev[0].record(stream)
-        P.paged_prefill(o, q, key_cache, value_cache, tables, lens, qs, cfg.softmax_scale, mq, ws)
+        P.paged_prefill(o, q, key_cache, value_cache, tables, lens, qs, cfg.softmax_scale, mq, ws, ks, vs)
         if ev is not None:
             ev[1].record(stream)
 
@@ -557,11 +568,12 @@ def run_prefill(args, cfg, world, rank):
     T = w.query.shape[0]
     line = {"metric": "paged prefill attention: causal TFLOP/s", "value": round(value, 2), "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": cfg.dtype if not cfg.cache_dtype.startswith("fp8") else "f16",
             "data": "synthetic",
             "config": {"workload": cfg.description, "name": cfg.name, "num_seqs": cfg.num_seqs, "query_tokens": T,
                        "causal_pairs_per_head": w.causal_pairs(), "num_heads": H, "num_kv_heads": cfg.num_kv_heads,
-                       "head_size": d, "block_size": cfg.block_size,
+                       "head_size": d, "block_size": cfg.block_size, "kv_dtype": cfg.cache_dtype,
                        "l2": f"inputs larger than L2: {(w.query.numel() * 2 * 2 + key_cache.numel() * 4) / 1e9:.2f} GB "
                              "of query, output and K/V per step vs 126 MB L2",
                        "parallelism": f"dp{world} (independent batches)"},
@@ -593,11 +605,17 @@ def _prefill_sample(cfg, rows_wanted):
     pos = lens[seq] - n + (rows - q_start[seq])
     kc, vc = bits16(w.key_values), bits16(w.value_values)
     import oracle
-    oracle.reshape_and_cache(bits16(w.new_key), bits16(w.new_value), cfg.dtype, kc, vc, cfg.dtype,
-                             w.slot_mapping.numpy())
+    kd = cfg.cache_dtype
+    ks = vs = None
+    if kd.startswith("fp8"):   # the oracle's own quantiser fills its FP8 pools
+        ks, vs = w.k_scale.numpy(), w.v_scale.numpy()
+        quant = oracle.quantize_e4m3 if kd == "fp8_e4m3" else oracle.quantize_e4m3_blocks
+        kc, vc = quant(kc, cfg.dtype, ks), quant(vc, cfg.dtype, vs)
+    oracle.reshape_and_cache(bits16(w.new_key), bits16(w.new_value), cfg.dtype, kc, vc, kd, w.slot_mapping.numpy(),
+                             ks, vs)
     inp = dict(query_bits=bits16(w.query)[rows], q_dtype=cfg.dtype, key_cache=kc, value_cache=vc,
-               kv_dtype=cfg.dtype, block_tables=w.block_tables.numpy()[seq], context_lens=(pos + 1).astype(np.int32),
-               q_start=np.arange(len(rows) + 1, dtype=np.int32), scale=cfg.softmax_scale)
+               kv_dtype=kd, block_tables=w.block_tables.numpy()[seq], context_lens=(pos + 1).astype(np.int32),
+               q_start=np.arange(len(rows) + 1, dtype=np.int32), scale=cfg.softmax_scale, k_scale=ks, v_scale=vs)
     flops = 4.0 * cfg.head_size * cfg.num_heads * float((pos + 1).sum())
     return inp, flops, len(rows)
 

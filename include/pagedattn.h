@@ -197,7 +197,15 @@ PA_API pa_status pa_paged_attention_static(void* out, const void* query, pa_dtyp
  *
  *  out, query     [num_q_tokens][num_heads][head_size], q_dtype (PA_F16 / PA_BF16); 16-byte aligned.
  *  key_cache,
- *  value_cache    [num_blocks][block_size][num_kv_heads][head_size], kv_dtype == q_dtype.
+ *  value_cache    [num_blocks][block_size][num_kv_heads][head_size]; kv_dtype == q_dtype, or E4M3
+ *                 (PA_FP8_E4M3 / PA_FP8_E4M3_BLOCK, head_size 128; the tutorial page, sec. 3.2, stores
+ *                 blocks in FP8) dequantised as code * scale as in pa_paged_attention.
+ *  k_scale,
+ *  v_scale        fp32 scales as in pa_paged_attention ([num_kv_heads], or [num_blocks][num_kv_heads] for
+ *                 PA_FP8_E4M3_BLOCK); required for the FP8 formats, else ignored. The FP8 path runs the
+ *                 tensor cores on f16: E4M3 values are exact in f16; a bf16 query is rounded to f16
+ *                 (magnitudes past 65504 overflow); per-block scales multiply the f16 values (one
+ *                 rounding of code * scale), per-kv-head scales are applied in fp32.
  *  block_tables   [num_seqs][max_blocks_per_seq] int32; context_lens [num_seqs] int32;
  *  q_start        [num_seqs + 1] int32, non-decreasing, q_start[0] = 0, q_start[num_seqs] = num_q_tokens.
  *  max_q_len      >= max_s n_s (sizes the grid; tiles past a sequence's chunk exit at once).
@@ -208,7 +216,8 @@ PA_API pa_status pa_paged_attention_static(void* out, const void* query, pa_dtyp
  * PA_DEVERR_CONTEXT_LEN and NaNs its rows; a block id outside the pool sets PA_DEVERR_BLOCK_ID.
  */
 PA_API pa_status pa_paged_prefill(void* out, const void* query, pa_dtype q_dtype, const void* key_cache,
-                                  const void* value_cache, pa_dtype kv_dtype, const int32_t* block_tables,
+                                  const void* value_cache, pa_dtype kv_dtype, const float* k_scale,
+                                  const float* v_scale, const int32_t* block_tables,
                                   int max_blocks_per_seq, const int32_t* context_lens, const int32_t* q_start,
                                   int num_seqs, int num_q_tokens, int num_heads, int num_kv_heads, int head_size,
                                   int block_size, int num_blocks, int max_q_len, float scale, void* workspace,

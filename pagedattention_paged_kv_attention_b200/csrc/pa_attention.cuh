@@ -53,8 +53,8 @@ constexpr int kHeadBlock = 8;            // kv heads per work item (one consumer
 constexpr int kConsumerWarps = kHeadBlock;
 constexpr int kBoxTokens = 8;            // tokens per TMA box (block_size >= 8); one swizzle atom
 constexpr int kMaxStages = 8;            // ring depth cap (the depth itself is per variant, see Layout)
-constexpr int kSmemBudget = 204 * 1024;  // shared memory the layout may use (of 227 KB per CTA)
-constexpr int kQueryBuffers = 2;
+constexpr int kSmemBudget = 216 * 1024;  // ring + query + small tables (the order table and slack come on top; 227 KB per CTA)
+constexpr int kQueryBuffers = 1;         // consumers copy the query into registers at an item's first stage
 constexpr int kIdWindow = 4;             // block ids prefetched per item: 32 * kIdWindow stages
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kPartitionQuantum = 64;    // partition sizes are multiples of this

@@ -37,26 +37,27 @@ bool encode_query_map(CUtensorMap* map, const void* query, int head_size, int nu
 }
 
 // Cache [NB][bs][Hkv][d] as {d, token, kv head, block}; box = one 128-byte chunk of the bs token rows
-// of one kv head of one block.
-bool encode_block_map(CUtensorMap* map, const void* cache, int head_size, int num_kv_heads, int block_size,
-                      int num_blocks) {
+// of one kv head of one block (64 columns of a 16-bit cache, 128 of an E4M3 one).
+bool encode_block_map(CUtensorMap* map, const void* cache, int elem_bytes, int head_size, int num_kv_heads,
+                      int block_size, int num_blocks) {
   auto encode = pa_host::tensor_map_encoder();
   if (!encode) return false;
-  const cuuint64_t e = 2;
+  const cuuint64_t e = static_cast<cuuint64_t>(elem_bytes);
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_size), static_cast<cuuint64_t>(block_size),
                         static_cast<cuuint64_t>(num_kv_heads), static_cast<cuuint64_t>(num_blocks)};
   cuuint64_t strides[3] = {num_kv_heads * head_size * e, head_size * e, block_size * num_kv_heads * head_size * e};
-  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(block_size), 1, 1};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(block_size), 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(cache), dims, strides, box, estr,
+  return encode(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
+                const_cast<void*>(cache), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, int D>
+template <typename T, int D, int KVB = 2, bool BS = false>
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const pa::pf::PrefillArgs& a, dim3 grid, cudaStream_t st) {
-  auto kernel = pa::pf::paged_prefill_kernel<T, D>;
+  auto kernel = pa::pf::paged_prefill_kernel<T, D, KVB, BS>;
   const int smem = static_cast<int>(pa::pf::Layout<D>::kBytes);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -66,7 +67,8 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
 }  // namespace
 
 extern "C" pa_status pa_paged_prefill(void* out, const void* query, pa_dtype q_dtype, const void* key_cache,
-                                      const void* value_cache, pa_dtype kv_dtype, const int32_t* block_tables,
+                                      const void* value_cache, pa_dtype kv_dtype, const float* k_scale,
+                                      const float* v_scale, const int32_t* block_tables,
                                       int max_blocks_per_seq, const int32_t* context_lens, const int32_t* q_start,
                                       int num_seqs, int num_q_tokens, int num_heads, int num_kv_heads,
                                       int head_size, int block_size, int num_blocks, int max_q_len, float scale,
@@ -84,7 +86,10 @@ extern "C" pa_status pa_paged_prefill(void* out, const void* query, pa_dtype q_d
     return PA_ERR_INVALID_ARGUMENT;
   if (workspace_bytes < PA_WORKSPACE_HEADER_BYTES) return PA_ERR_WORKSPACE_TOO_SMALL;
   const int group = num_heads / num_kv_heads;
-  if (kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;  // 16-bit caches only
+  const bool fp8 = pa_host::is_fp8(kv_dtype);
+  if (fp8 && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4))) return PA_ERR_INVALID_ARGUMENT;
+  if (!fp8 && kv_dtype != q_dtype) return PA_ERR_UNSUPPORTED;
+  if (fp8 && head_size != 128) return PA_ERR_UNSUPPORTED;
   if (head_size != 64 && head_size != 128) return PA_ERR_UNSUPPORTED;
   if (block_size != 8 && block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128)
     return PA_ERR_UNSUPPORTED;
@@ -95,11 +100,16 @@ extern "C" pa_status pa_paged_prefill(void* out, const void* query, pa_dtype q_d
 
   CUtensorMap tq, tk, tv;
   if (!encode_query_map(&tq, query, head_size, num_heads, num_q_tokens, group, tile_tokens) ||
-      !encode_block_map(&tk, key_cache, head_size, num_kv_heads, block_size, num_blocks) ||
-      !encode_block_map(&tv, value_cache, head_size, num_kv_heads, block_size, num_blocks))
+      !encode_block_map(&tk, key_cache, pa_host::elem_bytes(kv_dtype), head_size, num_kv_heads, block_size,
+                        num_blocks) ||
+      !encode_block_map(&tv, value_cache, pa_host::elem_bytes(kv_dtype), head_size, num_kv_heads, block_size,
+                        num_blocks))
     return PA_ERR_CUDA;
   pa::pf::PrefillArgs a{};
   a.out = out;
+  a.k_scale = fp8 ? k_scale : nullptr;
+  a.v_scale = fp8 ? v_scale : nullptr;
+  a.scale_block_stride = pa_host::scale_block_stride(kv_dtype, num_kv_heads);
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.q_start = q_start;
@@ -119,11 +129,21 @@ extern "C" pa_status pa_paged_prefill(void* out, const void* query, pa_dtype q_d
                   static_cast<unsigned>(num_seqs));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (q_dtype == PA_BF16)
-    e = head_size == 128 ? launch_prefill<__nv_bfloat16, 128>(tq, tk, tv, a, grid, st)
-                         : launch_prefill<__nv_bfloat16, 64>(tq, tk, tv, a, grid, st);
-  else
-    e = head_size == 128 ? launch_prefill<__half, 128>(tq, tk, tv, a, grid, st)
-                         : launch_prefill<__half, 64>(tq, tk, tv, a, grid, st);
+  const bool per_block = kv_dtype == PA_FP8_E4M3_BLOCK;
+  if (q_dtype == PA_BF16) {
+    if (fp8)
+      e = per_block ? launch_prefill<__nv_bfloat16, 128, 1, true>(tq, tk, tv, a, grid, st)
+                    : launch_prefill<__nv_bfloat16, 128, 1, false>(tq, tk, tv, a, grid, st);
+    else
+      e = head_size == 128 ? launch_prefill<__nv_bfloat16, 128>(tq, tk, tv, a, grid, st)
+                           : launch_prefill<__nv_bfloat16, 64>(tq, tk, tv, a, grid, st);
+  } else {
+    if (fp8)
+      e = per_block ? launch_prefill<__half, 128, 1, true>(tq, tk, tv, a, grid, st)
+                    : launch_prefill<__half, 128, 1, false>(tq, tk, tv, a, grid, st);
+    else
+      e = head_size == 128 ? launch_prefill<__half, 128>(tq, tk, tv, a, grid, st)
+                           : launch_prefill<__half, 64>(tq, tk, tv, a, grid, st);
+  }
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

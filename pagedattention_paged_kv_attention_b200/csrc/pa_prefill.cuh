@@ -21,6 +21,12 @@
 //                 a running max m that is raised only when a row's maximum exceeds it by more than 8
 //                 (then O and the sum are rescaled in place), and writes P (16-bit pairs) over S for the
 //                 PV MMA; at the end it normalises O and stores the row.
+// FP8-E4M3 caches (KVB = 1; tutorial page, sec. 3.2 "关键性能优化": blocks stored in FP8) take the same
+// path on f16 operands. TMA lands each E4M3 tile (128 keys x 128 one-byte columns) in the upper half of
+// its f16 operand slot; warps 2-3 widen it in place (every E4M3 value is exact in f16), each thread
+// owning whole rows, so a row is read before it is overwritten. A bf16 query is converted to f16 in
+// place once. Per-kv-head scales are exact fp32 factors on the softmax scale (K) and on the output (V);
+// per-block scales multiply the widened values (f16, one extra rounding of code x scale).
 // Every wait is bounded; a timed-out wait records PA_DEVERR_TIMEOUT and the CTA winds down (waiting,
 // bounded, for its own copies and MMAs) before it frees TMEM.
 #pragma once
@@ -46,6 +52,9 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8 betw
 
 struct PrefillArgs {
   void* out;                    // [T][H][d]
+  const float* k_scale;         // FP8: [Hkv] or [num_blocks][Hkv] (scale_block_stride = Hkv); else null
+  const float* v_scale;
+  int scale_block_stride;
   const int32_t* block_tables;  // [S][max_blocks_per_seq]
   const int32_t* context_lens;  // [S]
   const int32_t* q_start;       // [S + 1]
@@ -74,6 +83,7 @@ struct Layout {
 struct Bars {
   uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages], s_full[kTiles],
       p_full[kTiles], o_final[kTiles], mma_done;
+  uint64_t q_ready, k_load[kStages], v_load[kStages];  // FP8: query in f16, E4M3 tiles landed
   uint32_t tmem_base;
   int abort;
 };
@@ -116,11 +126,46 @@ __device__ __forceinline__ uint32_t pack_pair<__half>(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
-template <typename T, int D>
+// Widens row r of an E4M3 tile in place: the row's 128 codes (128-byte swizzled row r at `staged`) become
+// 128 f16 values in the two 128-byte-swizzled chunks of the f16 tile at `tile` (chunk stride
+// kKvTile * 128), multiplied by `scale` when it is not 1. The whole row is read before any write.
+__device__ __forceinline__ void widen_row(uint8_t* tile, const uint8_t* staged, int r, __half2 scale, bool scaled) {
+  uint4 q[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) q[u] = *reinterpret_cast<const uint4*>(staged + r * 128 + ((u ^ (r & 7)) << 4));
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+    uint32_t h[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      h[2 * k] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[k] & 0xffffu));
+      h[2 * k + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[k] >> 16));
+    }
+    if (scaled) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        __half2 x = *reinterpret_cast<__half2*>(&h[k]);
+        x = __hmul2(x, scale);
+        h[k] = *reinterpret_cast<uint32_t*>(&x);
+      }
+    }
+    // Values 16u .. 16u + 15 are f16 units 2u and 2u + 1 of the row: chunk u / 4, units 2(u % 4) + {0, 1}.
+    uint8_t* row = tile + (u >> 2) * (kKvTile * 128) + r * 128;
+    *reinterpret_cast<uint4*>(row + (((2 * (u & 3)) ^ (r & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4*>(row + (((2 * (u & 3) + 1) ^ (r & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+  }
+}
+
+// KVB: cache element bytes (2: a T cache; 1: E4M3). BS: E4M3 with per-(block, kv head) scales.
+template <typename T, int D, int KVB, bool BS>
 __global__ void __launch_bounds__(kThreads, 1)
 paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, const PrefillArgs a) {
   using L = Layout<D>;
+  constexpr bool kFp8 = KVB == 1;
+  using MT = typename std::conditional<kFp8, __half, T>::type;  // tensor-core operand type
+  static_assert(!kFp8 || D == 128, "FP8 caches need head_size 128");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* b = reinterpret_cast<Bars*>(sm + L::kBars);
@@ -172,11 +217,14 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
   // ---- set-up: barriers (thread 0), TMEM (warp 1) ----
   if (threadIdx.x == 0) {
     mbar_init(&b->q_full, 1);
+    mbar_init(&b->q_ready, 64);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&b->k_full[i], 1);
+      mbar_init(&b->k_full[i], kFp8 ? 64 : 1);   // FP8: the 64 widening threads arrive
       mbar_init(&b->k_empty[i], 1);
-      mbar_init(&b->v_full[i], 1);
+      mbar_init(&b->v_full[i], kFp8 ? 64 : 1);
       mbar_init(&b->v_empty[i], 1);
+      mbar_init(&b->k_load[i], 1);
+      mbar_init(&b->v_load[i], 1);
     }
     for (int x = 0; x < kTiles; ++x) {
       mbar_init(&b->s_full[x], 1);
@@ -224,12 +272,13 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
         if (!ok) atomicOr(err, PA_DEVERR_BLOCK_ID);
       }
       const unsigned okmask = __ballot_sync(0xffffffffu, ok);
-      const uint32_t bytes = __popc(okmask) * bs * 128 * L::kChunks;
+      const uint32_t bytes = __popc(okmask) * bs * 128 * (kFp8 ? 1 : L::kChunks);
       uint8_t* st = sm + L::kKV + stage * L::kStage;
       bool go = true;
 #pragma unroll
       for (int part = 0; part < 2; ++part) {  // 0: K, 1: V
-        uint64_t* full = part == 0 ? &b->k_full[stage] : &b->v_full[stage];
+        uint64_t* full = kFp8 ? (part == 0 ? &b->k_load[stage] : &b->v_load[stage])
+                              : (part == 0 ? &b->k_full[stage] : &b->v_full[stage]);
         uint64_t* empty = part == 0 ? &b->k_empty[stage] : &b->v_empty[stage];
         if (j >= kStages && !warp_wait_or_abort(b, empty, ((j / kStages) - 1) & 1, err)) {
           go = false;
@@ -237,10 +286,17 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
         }
         if (lane == 0) mbar_arrive_expect_tx(full, bytes);
         __syncwarp();
-        if (ok)
-          for (int c = 0; c < L::kChunks; ++c)
-            tma_load_4d(st + (part == 0 ? L::kK : L::kV) + c * (kKvTile * 128) + lane * bs * 128,
-                        part == 0 ? &tk : &tv, full, c * 64, 0, kvh, blk);
+        if (ok) {
+          if constexpr (kFp8) {
+            // The E4M3 tile (one 128-byte chunk per row) lands in the upper half of the f16 slot.
+            tma_load_4d(st + (part == 0 ? L::kK : L::kV) + (kKvTile * 128) + lane * bs * 128, part == 0 ? &tk : &tv,
+                        full, 0, 0, kvh, blk);
+          } else {
+            for (int c = 0; c < L::kChunks; ++c)
+              tma_load_4d(st + (part == 0 ? L::kK : L::kV) + c * (kKvTile * 128) + lane * bs * 128,
+                          part == 0 ? &tk : &tv, full, c * 64, 0, kvh, blk);
+          }
+        }
         ++issued[part * kStages + stage];
       }
       if (!go) break;
@@ -249,11 +305,62 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
     for (int part = 0; part < 2; ++part)
       for (int i = 0; i < kStages; ++i)
         if (issued[part * kStages + i] > 0)
-          mbar_wait(part == 0 ? &b->k_full[i] : &b->v_full[i], (issued[part * kStages + i] - 1) & 1, err);
+          mbar_wait(kFp8 ? (part == 0 ? &b->k_load[i] : &b->v_load[i]) : (part == 0 ? &b->k_full[i] : &b->v_full[i]),
+                    (issued[part * kStages + i] - 1) & 1, err);
+  } else if (kFp8 && (warp == 2 || warp == 3)) {
+    // ================================ E4M3 widening (FP8 caches) ================================
+    const int ct = threadIdx.x - 64;  // 0..63
+    bool ok = warp_wait_or_abort(b, &b->q_full, 0, err);
+    if (ok && std::is_same<T, __nv_bfloat16>::value) {
+      // The query tiles to f16, in place (same positions; every value of the bf16 range that f16 holds
+      // converts exactly up to f16's precision and range).
+      const int tiles = (nkv_t[1] > 0) ? 2 : 1;
+      uint4* q = reinterpret_cast<uint4*>(sm + L::kQ);
+      for (int i = ct; i < tiles * static_cast<int>(L::kQTile) / 16; i += 64) {
+        uint4 v = q[i];
+        uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
+          const __half2 h = __floats2half2_rn(f.x, f.y);
+          w[k] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        q[i] = v;
+      }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(&b->q_ready);
+    const int32_t* table = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
+    for (int j = 0; ok && j < nkv; ++j) {
+      const int stage = j % kStages;
+      for (int part = 0; part < 2; ++part) {
+        if (!(ok = warp_wait_or_abort(b, part == 0 ? &b->k_load[stage] : &b->v_load[stage], (j / kStages) & 1, err)))
+          break;
+        uint8_t* tile = sm + L::kKV + stage * L::kStage + (part == 0 ? L::kK : L::kV);
+        const float* scales = part == 0 ? a.k_scale : a.v_scale;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int r = ct + 64 * h;
+          __half2 sc = __float2half2_rn(1.f);
+          if constexpr (BS) {
+            const int t = j * kKvTile + r;
+            if (t <= p_max) {
+              const int blk = table[t / a.block_size];
+              sc = __float2half2_rn((blk >= 0 && blk < a.num_blocks)
+                                        ? __ldg(scales + static_cast<size_t>(blk) * a.scale_block_stride + kvh)
+                                        : 0.f);
+            }
+          }
+          widen_row(tile, tile + kKvTile * 128, r, sc, BS);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(part == 0 ? &b->k_full[stage] : &b->v_full[stage]);
+      }
+    }
   } else if (warp == 1) {
     // ================================ MMA issuer ================================
-    constexpr uint32_t idesc_s = mma_idesc_f16<T>(kRows, kKvTile, false);
-    constexpr uint32_t idesc_o = mma_idesc_f16<T>(kRows, D, true);
+    constexpr uint32_t idesc_s = mma_idesc_f16<MT>(kRows, kKvTile, false);
+    constexpr uint32_t idesc_o = mma_idesc_f16<MT>(kRows, D, true);
     auto kv_addr = [&](int j, uint32_t part) { return smem_u32(sm + L::kKV + (j % kStages) * L::kStage + part); };
     auto issue_s = [&](int x, int j) {  // S_x = Q_x K_j^T over d in steps of 16
       const uint32_t q_addr = smem_u32(sm + L::kQ + x * L::kQTile), k_addr = kv_addr(j, L::kK);
@@ -273,7 +380,8 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
         mma_f16_ts(tmem + x * kTmemTile + kTmemO, tmem + x * kTmemTile + 8 * k,
                    smem_desc_sw128(v_addr + k * 16 * 128, kKvTile * 128, 1024), idesc_o, (j > 0 || k > 0) ? 1u : 0u);
     };
-    bool ok = warp_wait_or_abort(b, &b->q_full, 0, err) && warp_wait_or_abort(b, &b->k_full[0], 0, err);
+    bool ok = warp_wait_or_abort(b, kFp8 ? &b->q_ready : &b->q_full, 0, err) &&
+              warp_wait_or_abort(b, &b->k_full[0], 0, err);
     if (ok) {
       tc_fence_after();
       if (lane == 0) {
@@ -341,7 +449,9 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
       const int pos_lane0 = __shfl_sync(0xffffffffu, pos, 0);
       const uint32_t t_s = tmem + x * kTmemTile + (static_cast<uint32_t>(r & ~31) << 16);
       const uint32_t t_o = t_s + kTmemO;
-      const float sl2 = a.scale_log2;
+      // Per-kv-head FP8 scales are exact fp32 factors: K's on the softmax scale, V's on the output.
+      const float sl2 = (kFp8 && !BS) ? a.scale_log2 * __ldg(a.k_scale + kvh) : a.scale_log2;
+      const float out_scale = (kFp8 && !BS) ? __ldg(a.v_scale + kvh) : 1.f;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < nkv_x; ++j) {
@@ -405,7 +515,7 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
             const float2 xy = __ffma2_rn(make_float2(__uint_as_float(v[c][2 * i]), __uint_as_float(v[c][2 * i + 1])),
                                          sl2x2, negm);
             const float2 p = make_float2(ex2(xy.x), ex2(xy.y));
-            w[i] = pack_pair<T>(p.x, p.y);
+            w[i] = pack_pair<MT>(p.x, p.y);
             ls[i & 3] = __fadd2_rn(ls[i & 3], p);
           }
           tmem_st16(t_s + 16 * c, w);
@@ -420,7 +530,7 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
       if (ok) ok = warp_wait_or_abort(b, &b->o_final[x], 0, err);
       if (ok) {
         tc_fence_after();
-        const float inv = 1.f / l;
+        const float inv = out_scale / l;
         T* dst = static_cast<T*>(a.out) + (static_cast<size_t>(q0 + min(tok, n - 1)) * a.num_heads + kvh * G + r % G) * D;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {

@@ -58,8 +58,8 @@ lib.pa_probe_stream_read.argtypes = [_p, _sz, _i, _p, _p]
 lib.pa_probe_paged_read.restype = _i
 lib.pa_probe_paged_read.argtypes = [_p, _p, _i, _p, _i, _p, _i, _i, _i, _i, _i, _p, _p]
 lib.pa_paged_prefill.restype = _i
-lib.pa_paged_prefill.argtypes = [_p, _p, _i, _p, _p, _i, _p, _i, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _sz,
-                                 _p]
+lib.pa_paged_prefill.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f,
+                                 _p, _sz, _p]
 lib.pa_reshape_and_cache.restype = _i
 lib.pa_reshape_and_cache.argtypes = [_p, _p, _i, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 lib.pa_copy_blocks.restype = _i
@@ -213,16 +213,18 @@ def paged_attention(out, query, key_cache, value_cache, block_tables, context_le
 
 
 def paged_prefill(out, query, key_cache, value_cache, block_tables, context_lens, q_start, scale, max_q_len,
-                  workspace, stream=None):
+                  workspace, k_scale=None, v_scale=None, stream=None):
     """Causal prefill: out[T,H,d] for query chunks query[T,H,d] (rows q_start[s]..q_start[s+1]-1 of
-    sequence s, the last rows of its context_lens[s] cached tokens) over key/value_cache[NB,bs,Hkv,d]."""
+    sequence s, the last rows of its context_lens[s] cached tokens) over key/value_cache[NB,bs,Hkv,d].
+    FP8 (uint8 E4M3) caches take k_scale/v_scale: [Hkv] per kv head, or [NB, Hkv] per block."""
     T, H, d = query.shape
     NB, bs, Hkv, _ = key_cache.shape
     _same(out, query, "out/query")
     _same(key_cache, value_cache, "key_cache/value_cache")
     st = lib.pa_paged_prefill(_arg(out, "out"), _arg(query, "query"), dtype_code(query.dtype),
                               _arg(key_cache, "key_cache"), _arg(value_cache, "value_cache"),
-                              dtype_code(key_cache.dtype), _arg(block_tables, "block_tables", _I32, 2),
+                              cache_code(key_cache, k_scale), _arg(k_scale, "k_scale", _F32, (1, 2)),
+                              _arg(v_scale, "v_scale", _F32, (1, 2)), _arg(block_tables, "block_tables", _I32, 2),
                               block_tables.shape[1], _arg(context_lens, "context_lens", _I32, 1),
                               _arg(q_start, "q_start", _I32, 1), context_lens.shape[0], T, H, Hkv, d, bs, NB,
                               int(max_q_len), float(scale), _arg(workspace, "workspace"),

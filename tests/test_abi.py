@@ -243,3 +243,27 @@ def test_probes_reject_bad_arguments(P):
     assert paged(bt=18) == P.PA_ERR_INVALID_ARGUMENT
     assert paged(dt=9) == P.PA_ERR_INVALID_ARGUMENT
     assert paged(Hkv=1, d=4) == P.PA_ERR_UNSUPPORTED            # token row of 8 bytes: not 16-byte vectors
+
+
+def call_prefill(P, **over):
+    args = dict(out=16, query=16, q_dtype=P.PA_BF16, key_cache=16, value_cache=16, kv_dtype=P.PA_BF16, k_scale=None,
+                v_scale=None, block_tables=16, max_blocks_per_seq=4, context_lens=16, q_start=16, num_seqs=2,
+                num_q_tokens=64, num_heads=8, num_kv_heads=2, head_size=128, block_size=16, num_blocks=10, max_q_len=32,
+                scale=0.1, workspace=16, workspace_bytes=256, stream=None)
+    args.update(over)
+    return P.lib.pa_paged_prefill(*args.values())
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(out=None), 1), (dict(q_start=None), 1), (dict(workspace=None), 1), (dict(key_cache=24), 1),
+    (dict(scale=0.0), 1), (dict(scale=float("inf")), 1), (dict(num_heads=6, num_kv_heads=4), 1),
+    (dict(kv_dtype=2), 1),                                                   # FP8 without scales
+    (dict(kv_dtype=3, k_scale=16), 1),                                       # per-block FP8, one scale missing
+    (dict(kv_dtype=2, k_scale=16, v_scale=16, head_size=64), 2),             # FP8: head size 128 only
+    (dict(kv_dtype=0), 2),                                                   # f16 cache with a bf16 query
+    (dict(head_size=96), 2), (dict(block_size=4), 2), (dict(num_heads=24, num_kv_heads=1), 2),
+    (dict(workspace_bytes=128), 3),
+    (dict(num_seqs=0), 0), (dict(max_q_len=0), 0),                           # nothing to compute
+])
+def test_prefill_rejects_bad_arguments_without_cuda(P, over, status):
+    assert call_prefill(P, **over) == status

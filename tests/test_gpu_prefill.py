@@ -14,6 +14,9 @@ takes the same two steps on the same seeded inputs.
   a one-token chunk of the context truncated to p + 1).
 * Contract violations (a chunk longer than its context, a block id outside the pool) set the device
   error word without faulting.
+* FP8-E4M3 caches with per-kv-head and per-block scales: ragged cases compared element by element,
+  and the full-size FP8 chunked workloads on whole sequences and sampled rows; the pools after the
+  step's FP8 reshape_and_cache match the oracle's byte for byte.
 """
 import zlib
 
@@ -196,3 +199,94 @@ def test_contract_violations_are_flagged(P):
                     w.max_q_len, ws)
     torch.cuda.synchronize()
     assert P.get_device_error(ws) & P.PA_DEVERR_BLOCK_ID
+
+
+# ---------------------------------------------------------------------------------------------------
+# FP8-E4M3 caches (one scale per kv head, or per (block, kv head)): the pool is quantised by the oracle's
+# encoder, the step's reshape_and_cache writes the chunk in FP8 (bit-exact against the oracle's), and
+# the prefill reads the codes.
+# ---------------------------------------------------------------------------------------------------
+def fp8_pools(w):
+    """The oracle's E4M3 pools before the step and after it writes the chunk, and the scales."""
+    cfg = w.cfg
+    kd = cfg.cache_dtype
+    ks, vs = w.k_scale.numpy(), w.v_scale.numpy()
+    quant = oracle.quantize_e4m3 if kd == "fp8_e4m3" else oracle.quantize_e4m3_blocks
+    kc0, vc0 = quant(bits16(w.key_values), cfg.dtype, ks), quant(bits16(w.value_values), cfg.dtype, vs)
+    kc, vc = kc0.copy(), vc0.copy()
+    oracle.reshape_and_cache(bits16(w.new_key), bits16(w.new_value), cfg.dtype, kc, vc, kd, w.slot_mapping.numpy(),
+                             ks, vs)
+    return kc0, vc0, kc, vc, ks, vs
+
+
+def fp8_prefill_step(P, w):
+    kc0, vc0, kc, vc, ks, vs = fp8_pools(w)
+    dev = torch.device("cuda")
+    kd, vd = torch.from_numpy(kc0).to(dev), torch.from_numpy(vc0).to(dev)
+    ks_d, vs_d = torch.from_numpy(ks).to(dev), torch.from_numpy(vs).to(dev)
+    P.reshape_and_cache(w.new_key.to(dev), w.new_value.to(dev), kd, vd, w.slot_mapping.to(dev), ks_d, vs_d)
+    q = w.query.to(dev)
+    out = torch.full_like(q, float("nan"))
+    ws = torch.zeros(64, dtype=torch.int32, device=dev)
+    P.paged_prefill(out, q, kd, vd, w.block_tables.to(dev), w.context_lens.to(dev), w.q_start.to(dev),
+                    w.cfg.softmax_scale, w.max_q_len, ws, k_scale=ks_d, v_scale=vs_d)
+    torch.cuda.synchronize()
+    assert P.get_device_error(ws) == 0
+    assert np.array_equal(kd.cpu().numpy(), kc) and np.array_equal(vd.cpu().numpy(), vc), "FP8 pools differ"
+    return out, kc, vc, ks, vs
+
+
+FP8_CASES = [
+    # (H, Hkv, bs, dtype, kv_dtype, lens, chunks)
+    (8, 8, 16, "bf16", "fp8_e4m3", [1, 17, 128, 129, 300], None),
+    (8, 2, 16, "bf16", "fp8_e4m3_block", [200, 64, 513], [200, 1, 130]),
+    (16, 2, 8, "f16", "fp8_e4m3", [255, 256, 257], [100, 256, 0]),
+    (16, 2, 32, "f16", "fp8_e4m3_block", [40, 380], [40, 260]),
+    (8, 4, 128, "bf16", "fp8_e4m3_block", [129, 1000], [129, 333]),
+]
+
+
+@pytest.mark.parametrize("case", FP8_CASES, ids=lambda c: f"H{c[0]}_Hkv{c[1]}_bs{c[2]}_{c[3]}_{c[4]}")
+def test_prefill_fp8_ragged(P, case):
+    H, Hkv, bs, dtype, kvd, lens, chunks = case
+    cfg = W.PrefillConfig(name="fp8", description="", num_seqs=len(lens), num_heads=H, num_kv_heads=Hkv, head_size=128,
+                          block_size=bs, dtype=dtype, seed=zlib.crc32(repr(case).encode()), context_lens=tuple(lens),
+                          kv_dtype=kvd)
+    w = W.make_prefill_workload(cfg, chunk_lens=chunks)
+    out, kc, vc, ks, vs = fp8_prefill_step(P, w)
+    ref = oracle.paged_prefill(bits16(w.query), dtype, kc, vc, kvd, w.block_tables.numpy(), w.context_lens.numpy(),
+                               w.q_start.numpy(), cfg.softmax_scale, ks, vs)
+    got = out.double().cpu().numpy()
+    assert np.all(np.isfinite(got)), "non-finite output"
+    worst = np.max(np.abs(got - ref) - elementwise_bound(ref, kvd, dtype)) if ref.size else -1
+    assert worst <= 0, f"max excess over the bound {worst}"
+
+
+@pytest.mark.parametrize("name", ["chunked_prefill_fp8", "chunked_prefill_fp8_block"])
+def test_prefill_fp8_full_size(P, name):
+    """Full-size FP8 chunked prefill: every row of two adjacent whole sequences and sampled rows of the
+    rest against the oracle, within the FP8 tolerance."""
+    cfg = W.PREFILL_CONFIGS[name]
+    w = W.make_prefill_workload(cfg)
+    out, kc, vc, ks, vs = fp8_prefill_step(P, w)
+    got = out.double().cpu().numpy()
+    assert np.all(np.isfinite(got))
+    lens, q_start = w.context_lens.numpy(), w.q_start.numpy()
+    seqs = whole_sequences("chunked_prefill", lens, q_start)
+    rows = np.concatenate([np.arange(q_start[s], q_start[s + 1]) for s in seqs])
+    sub_start = np.concatenate([[0], np.cumsum([q_start[s + 1] - q_start[s] for s in seqs])]).astype(np.int32)
+    ref = oracle.paged_prefill(bits16(w.query)[rows], cfg.dtype, kc, vc, cfg.cache_dtype, w.block_tables.numpy()[seqs],
+                               lens[seqs], sub_start, cfg.softmax_scale, ks, vs)
+    err = np.max(np.abs(got[rows] - ref))
+    assert err <= TOLERANCE[cfg.cache_dtype], f"{name}: max-abs error {err} over whole sequences {seqs}"
+    rng = np.random.default_rng(zlib.crc32(name.encode()))
+    T = w.query.shape[0]
+    sample = np.unique(np.concatenate([q_start[:-1], q_start[1:] - 1, rng.integers(0, T, 48)]))
+    seq = np.searchsorted(q_start, sample, side="right") - 1
+    n = q_start[seq + 1] - q_start[seq]
+    pos = lens[seq] - n + (sample - q_start[seq])
+    ref_s = oracle.paged_prefill(bits16(w.query)[sample], cfg.dtype, kc, vc, cfg.cache_dtype,
+                                 w.block_tables.numpy()[seq], (pos + 1).astype(np.int32),
+                                 np.arange(len(sample) + 1, dtype=np.int32), cfg.softmax_scale, ks, vs)
+    err_s = np.max(np.abs(got[sample] - ref_s))
+    assert err_s <= TOLERANCE[cfg.cache_dtype], f"{name}: max-abs error {err_s} on sampled rows"

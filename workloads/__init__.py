@@ -326,10 +326,15 @@ class PrefillConfig:
     len_range: Optional[tuple] = None
     chunk: Optional[int] = None                    # None: the whole prompt is the chunk
     scale: Optional[float] = None
+    kv_dtype: Optional[str] = None                 # None: the query dtype; or "fp8_e4m3" / "fp8_e4m3_block"
 
     @property
     def softmax_scale(self) -> float:
         return self.scale if self.scale is not None else 1.0 / math.sqrt(self.head_size)
+
+    @property
+    def cache_dtype(self) -> str:
+        return self.kv_dtype or self.dtype
 
 
 PREFILL_CONFIGS = {
@@ -357,6 +362,20 @@ PREFILL_CONFIGS = {
                     "the chunk, 32 q / 8 kv heads, head_size 128, block_size 16, bf16",
         num_seqs=32, num_heads=32, num_kv_heads=8, head_size=128, block_size=16, dtype="bf16", seed=14,
         len_range=(2048, 8192), chunk=512),
+    "chunked_prefill_fp8": PrefillConfig(
+        name="chunked_prefill_fp8",
+        description="chunked prefill over an FP8-E4M3 cache with one scale per kv head: 32 sequences with "
+                    "contexts U[2048,8192], the last 512 tokens of each as the chunk, 32 q / 8 kv heads, "
+                    "head_size 128, block_size 16, bf16 queries",
+        num_seqs=32, num_heads=32, num_kv_heads=8, head_size=128, block_size=16, dtype="bf16", seed=15,
+        len_range=(2048, 8192), chunk=512, kv_dtype="fp8_e4m3"),
+    "chunked_prefill_fp8_block": PrefillConfig(
+        name="chunked_prefill_fp8_block",
+        description="chunked prefill over an FP8-E4M3 cache with one scale per (block, kv head): 32 sequences "
+                    "with contexts U[2048,8192], the last 512 tokens of each as the chunk, 32 q / 8 kv heads, "
+                    "head_size 128, block_size 16, bf16 queries",
+        num_seqs=32, num_heads=32, num_kv_heads=8, head_size=128, block_size=16, dtype="bf16", seed=16,
+        len_range=(2048, 8192), chunk=512, kv_dtype="fp8_e4m3_block"),
 }
 
 
@@ -373,6 +392,8 @@ class PrefillWorkload:
     new_key: torch.Tensor           # [T, Hkv, d]: the chunks' keys, row order
     new_value: torch.Tensor
     slot_mapping: torch.Tensor      # int64 [T]
+    k_scale: Optional[torch.Tensor] = None   # FP8 caches: float32 [Hkv], or [num_blocks, Hkv] per block
+    v_scale: Optional[torch.Tensor] = None
 
     @property
     def max_q_len(self) -> int:
@@ -442,6 +463,21 @@ def make_prefill_workload(cfg: PrefillConfig, seed: Optional[int] = None, device
         pools.append(pool)
     key_pool, value_pool = pools
 
+    # FP8 calibration scales from the drawn values (the chunk's included), as for decode: max |x| / 448
+    # per kv head, or per (block, kv head) with 1 for blocks without data.
+    k_scale = v_scale = None
+    if cfg.cache_dtype == "fp8_e4m3":
+        k_scale, v_scale = [(pool[used_t].float().abs().amax(dim=(0, 1, 3)) / FP8_MAX).to(torch.float32)
+                            for pool in pools]
+    elif cfg.cache_dtype == "fp8_e4m3_block":
+        scales = []
+        for pool in pools:
+            sc = torch.ones((NB, Hkv), dtype=torch.float32, device=dev)
+            amax = pool[used_t].float().abs().amax(dim=(1, 3))
+            sc[used_t] = torch.where(amax > 0, amax / FP8_MAX, torch.ones_like(amax))
+            scales.append(sc)
+        k_scale, v_scale = scales
+
     # The chunk rows: slots of positions L-n .. L-1, their values taken out of the pool and poisoned there.
     tables_t = torch.from_numpy(tables).to(dev)
     seq_of_row = torch.from_numpy(np.repeat(np.arange(S), n)).to(dev)
@@ -465,4 +501,4 @@ def make_prefill_workload(cfg: PrefillConfig, seed: Optional[int] = None, device
         q_start=torch.from_numpy(q_start.astype(np.int32)).to(dev),
         block_tables=torch.from_numpy(tables.astype(np.int32)).to(dev), num_blocks=NB,
         query=query, key_values=key_pool, value_values=value_pool, new_key=new_key, new_value=new_value,
-        slot_mapping=(blk * bs + off).to(torch.int64))
+        slot_mapping=(blk * bs + off).to(torch.int64), k_scale=k_scale, v_scale=v_scale)
