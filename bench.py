@@ -454,6 +454,13 @@ def measure_decode(args, cfg, P, dev, rank, world, peak, peak_measured, checks):
         rec["ceilings"] = ceil
         rec["roofline"]["frac_of_read_stream"] = round(achieved / ceil["hbm_read_stream_gbs"], 4)
         rec["roofline"]["frac_of_paged_read"] = round(achieved / ceil["paged_read_gbs"], 4)
+        if cfg.shared_prefix_tokens:
+            # Every sequence reads the shared prefix blocks: most logical bytes come from L2 (the unique
+            # bytes are a fifth of them), so the bound for the logical bytes is the L2 read ceiling.
+            rec["roofline"].update({"bound": "l2", "peak": ceil["l2_read_gbs"],
+                                    "frac": round(achieved / ceil["l2_read_gbs"], 4),
+                                    "peak_source": "measured in this run (pa_probe_stream_read, 32 MiB read 64 times)",
+                                    "frac_of_measured_hbm_copy": round(achieved / peak, 4)})
         if checks:
             # L2 flush check: the same attention call with L2 flushed (a write of twice the L2 size)
             # before each step, per-step event timing; against the back-to-back figure above.

@@ -61,7 +61,11 @@ constexpr int kPartitionQuantum = 64;    // partition sizes are multiples of thi
 constexpr int kOrderMaxSeqs = 1024;      // batches up to this size take their items longest first
 constexpr int kOrderMaxRounds = 128;     // ... when the context splits into at most this many partitions
 constexpr int kRemBins = 128;            // partial partitions are ordered by size in this many bins
-constexpr int kClaimAhead = 4;           // the next item is claimed when this many stages remain to issue
+constexpr int kClaimAhead = 6;           // the next item is claimed when this many stages remain to issue
+#ifndef PA_PREFETCH_AHEAD
+#define PA_PREFETCH_AHEAD 4
+#endif
+constexpr int kPrefetchAhead = PA_PREFETCH_AHEAD;  // stages beyond the ring prefetched into L2 (0: none)
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Workspace header words: error bits, work counter, finished-CTA counter.
@@ -503,14 +507,55 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
       }                                                                                                \
     }                                                                                                  \
   } while (0)
-#define PA_CLAIM_NEXT()                                                                                \
+// Prefetch stage KS (tokens TB..TE of the item, kv heads from KVH) into L2: the lanes and coordinates
+// of its TMA loads, block ids from the item's window IDS (boxes beyond the window are skipped).
+#define PA_PREFETCH(IDS, KS, TB, TE, KVH, ROW)                                                         \
   do {                                                                                                 \
-    unsigned int t_ = 0;                                                                               \
-    if (lane == 0) t_ = atomicAdd(args.header + kWsWork, 1u);                                          \
-    nxt_idx = __shfl_sync(0xffffffffu, t_, 0);                                                         \
-    PA_PREPARE(nxt_idx, nxt_c, nxt_L, nxt_ids);                                                        \
-    have_next = true;                                                                                  \
+    const int pt0_ = (TB) + (KS) * S::kTS;                                                             \
+    const int pntok_ = cmin(S::kTS, (TE) - pt0_);                                                      \
+    const int pnbox_ = (pntok_ + kBoxTokens - 1) / kBoxTokens;                                         \
+    const int prel_ = (KS) * S::kGroups + (op_box < S::kGroups ? op_box : 0);                          \
+    int pblk_ = -1;                                                                                    \
+    _Pragma("unroll") for (int j_ = 0; j_ < kIdWindow; ++j_) {                                         \
+      const int v_ = __shfl_sync(0xffffffffu, IDS[j_], prel_ & 31);                                    \
+      if ((prel_ >> 5) == j_) pblk_ = v_;                                                              \
+    }                                                                                                  \
+    if (pntok_ > 0 && op_box < pnbox_ && lane < 2 * S::kChunks * S::kGroups && pblk_ >= 0 &&           \
+        pblk_ < args.num_blocks)                                                                       \
+      tma_prefetch_l2_4d(op_kv ? &tmap_v : &tmap_k, op_ch * S::kChunkElems, (pt0_ + op_box * kBoxTokens) % bs, \
+                         (KVH), pblk_);                                                                \
+    (void)(ROW);                                                                                       \
   } while (0)
+// Claiming the next item takes three steps spread over consecutive stages of the current one, so that
+// no step waits on the one before it: (1) the ticket's atomic, (2) the ticket's decode and the context
+// length's load, (3) the block-id window's loads. Each step is a no-op once done.
+#define PA_CLAIM_STEP()                                                                                \
+  do {                                                                                                 \
+    if (claim_step == 0) {                                                                             \
+      if (lane == 0) pend_t = atomicAdd(args.header + kWsWork, 1u);                                    \
+    } else if (claim_step == 1) {                                                                      \
+      nxt_idx = __shfl_sync(0xffffffffu, pend_t, 0);                                                   \
+      if (nxt_idx < num_tickets) {                                                                     \
+        nxt_c = ordered ? decode_ordered(nxt_idx, args, order) : decode_item(nxt_idx, args);           \
+        nxt_L = __ldg(args.context_lens + nxt_c.s);                                                    \
+      }                                                                                                \
+    } else if (claim_step == 2) {                                                                      \
+      if (nxt_idx < num_tickets) {                                                                     \
+        if (nxt_c.part < 0)                                                                            \
+          nxt_c.part = (nxt_L > 0 && !context_len_invalid(nxt_L, args)) ? (nxt_L - 1) / args.partition_size : 0; \
+        const int need_ = nxt_L <= 0 ? 0 : cmin(args.max_blocks_per_seq, nxt_L / bs + (nxt_L % bs != 0)); \
+        const int32_t* row_ = args.block_tables + static_cast<size_t>(nxt_c.s) * args.max_blocks_per_seq; \
+        _Pragma("unroll") for (int j_ = 0; j_ < kIdWindow; ++j_) {                                     \
+          const int entry_ = ((nxt_c.part * boxes_per_part + j_ * 32 + lane) * kBoxTokens) / bs;       \
+          nxt_ids[j_] = entry_ < need_ ? __ldg(row_ + entry_) : 0;                                     \
+        }                                                                                              \
+      }                                                                                                \
+      have_next = true;                                                                                \
+    }                                                                                                  \
+    if (claim_step < 3) ++claim_step;                                                                  \
+  } while (0)
+    unsigned int pend_t = 0;
+    int claim_step = 0;
 
     {
       unsigned int t0 = 0;
@@ -520,6 +565,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
     }
     while (!aborted && cur_idx < num_tickets) {
       have_next = false;
+      claim_step = 0;
       const ItemCoord c = cur_c;
       const int L = cur_L;
       const bool bad_len = context_len_invalid(L, args);
@@ -586,8 +632,23 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           const int op_kv = (lane / S::kChunks) & 1;
           const int op_ch = lane % S::kChunks;
           const int claim_at = cmax(0, n_stages - kClaimAhead);
+          static_assert(kPrefetchAhead + 2 <= kClaimAhead, "the next item is known before its stages are prefetched");
           for (int k = 0; k < n_stages; ++k) {
-            if (k == claim_at) PA_CLAIM_NEXT();
+            if (k >= claim_at) PA_CLAIM_STEP();
+            {
+              // L2 prefetch of the boxes kPrefetchAhead stages ahead (into the next item near the end of
+              // this one), so that DRAM latency is already under way when the ring slot frees.
+              const int kp = k + kPrefetchAhead;
+              if (kPrefetchAhead == 0) {
+              } else if (kp < n_stages) {
+                PA_PREFETCH(cur_ids, kp, tok_begin, tok_end, kvh0, row);
+              } else if (have_next && nxt_idx < num_tickets && nxt_L > 0 && !context_len_invalid(nxt_L, args)) {
+                const int nb = nxt_c.part * args.partition_size;
+                const int ne = cmin(nxt_L, nb + args.partition_size);
+                const int32_t* nrow = args.block_tables + static_cast<size_t>(nxt_c.s) * args.max_blocks_per_seq;
+                if (nb < ne) PA_PREFETCH(nxt_ids, kp - n_stages, nb, ne, nxt_c.hb * kHeadBlock, nrow);
+              }
+            }
             const int t0 = tok_begin + k * S::kTS;
             const int ntok = cmin(S::kTS, tok_end - t0);
             const int nbox = (ntok + kBoxTokens - 1) / kBoxTokens;
@@ -644,14 +705,15 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         }
       }
       if (aborted) break;
-      if (!have_next) PA_CLAIM_NEXT();  // items without stages (empty, invalid or past the context)
+      while (!have_next) PA_CLAIM_STEP();  // items with few stages (or none: empty, invalid, past the context)
       cur_idx = nxt_idx;
       cur_c = nxt_c;
       cur_L = nxt_L;
 #pragma unroll
       for (int j = 0; j < kIdWindow; ++j) cur_ids[j] = nxt_ids[j];
     }
-#undef PA_CLAIM_NEXT
+#undef PA_CLAIM_STEP
+#undef PA_PREFETCH
 #undef PA_PREPARE
     // No work left: one terminating message.
     if (!aborted) {

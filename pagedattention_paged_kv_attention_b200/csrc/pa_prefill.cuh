@@ -75,15 +75,16 @@ struct Layout {
   static constexpr uint32_t kV = kChunks * kKvTile * 128;
   static constexpr uint32_t kStage = 2 * kChunks * kKvTile * 128;
   static constexpr uint32_t kBars = kKV + kStages * kStage;
-  // Barriers and flags, alignment slack; at least 120 KB so that one CTA holds an SM (and with it
-  // all 512 TMEM columns: a second CTA's allocation would wait for the first to finish).
-  static constexpr uint32_t kBytes = (kBars + 256 + 1024) > 120u * 1024 ? (kBars + 256 + 1024) : 120u * 1024;
+  // Barriers, flags and box scales, alignment slack; at least 120 KB so that one CTA holds an SM (and
+  // with it all 512 TMEM columns: a second CTA's allocation would wait for the first to finish).
+  static constexpr uint32_t kBytes = (kBars + 1024 + 1024) > 120u * 1024 ? (kBars + 1024 + 1024) : 120u * 1024;
 };
 
 struct Bars {
   uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages], s_full[kTiles],
       p_full[kTiles], o_final[kTiles], mma_done;
   uint64_t q_ready, k_load[kStages], v_load[kStages];  // FP8: query in f16, E4M3 tiles landed
+  float box_scale[kStages][2][kKvTile / 8];            // per-block FP8: K and V scale of each box
   uint32_t tmem_base;
   int abort;
 };
@@ -284,6 +285,15 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
           go = false;
           break;
         }
+        if constexpr (kFp8 && BS) {
+          // Scale of each box for the widening warps: the slot's previous tile has been widened (its
+          // MMAs, which waited for that, have released the slot), and the arrive below publishes it.
+          if (lane < nblk)
+            b->box_scale[stage][part][lane] =
+                ok ? __ldg((part == 0 ? a.k_scale : a.v_scale) + static_cast<size_t>(blk) * a.scale_block_stride + kvh)
+                   : 0.f;
+          __syncwarp();
+        }
         if (lane == 0) mbar_arrive_expect_tx(full, bytes);
         __syncwarp();
         if (ok) {
@@ -330,26 +340,18 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
     }
     fence_proxy_async_smem();
     mbar_arrive(&b->q_ready);
-    const int32_t* table = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
     for (int j = 0; ok && j < nkv; ++j) {
       const int stage = j % kStages;
       for (int part = 0; part < 2; ++part) {
         if (!(ok = warp_wait_or_abort(b, part == 0 ? &b->k_load[stage] : &b->v_load[stage], (j / kStages) & 1, err)))
           break;
         uint8_t* tile = sm + L::kKV + stage * L::kStage + (part == 0 ? L::kK : L::kV);
-        const float* scales = part == 0 ? a.k_scale : a.v_scale;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int r = ct + 64 * h;
           __half2 sc = __float2half2_rn(1.f);
           if constexpr (BS) {
-            const int t = j * kKvTile + r;
-            if (t <= p_max) {
-              const int blk = table[t / a.block_size];
-              sc = __float2half2_rn((blk >= 0 && blk < a.num_blocks)
-                                        ? __ldg(scales + static_cast<size_t>(blk) * a.scale_block_stride + kvh)
-                                        : 0.f);
-            }
+            if (j * kKvTile + r <= p_max) sc = __float2half2_rn(b->box_scale[stage][part][r / a.block_size]);
           }
           widen_row(tile, tile + kKvTile * 128, r, sc, BS);
         }
