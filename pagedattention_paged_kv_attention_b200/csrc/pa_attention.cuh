@@ -59,13 +59,12 @@ constexpr int kIdWindow = 4;             // block ids prefetched per item: 32 * 
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kPartitionQuantum = 64;    // partition sizes are multiples of this
 constexpr int kOrderMaxSeqs = 1024;      // batches up to this size take their items longest first
-constexpr int kOrderMaxRounds = 128;     // ... when the context splits into at most this many partitions
+#ifndef PA_ORDER_MAX_ROUNDS
+#define PA_ORDER_MAX_ROUNDS 128
+#endif
+constexpr int kOrderMaxRounds = PA_ORDER_MAX_ROUNDS;  // ... and the context splits into at most this many partitions
 constexpr int kRemBins = 128;            // partial partitions are ordered by size in this many bins
 constexpr int kClaimAhead = 6;           // the next item is claimed when this many stages remain to issue
-#ifndef PA_PREFETCH_AHEAD
-#define PA_PREFETCH_AHEAD 4
-#endif
-constexpr int kPrefetchAhead = PA_PREFETCH_AHEAD;  // stages beyond the ring prefetched into L2 (0: none)
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Workspace header words: error bits, work counter, finished-CTA counter.
@@ -507,25 +506,6 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
       }                                                                                                \
     }                                                                                                  \
   } while (0)
-// Prefetch stage KS (tokens TB..TE of the item, kv heads from KVH) into L2: the lanes and coordinates
-// of its TMA loads, block ids from the item's window IDS (boxes beyond the window are skipped).
-#define PA_PREFETCH(IDS, KS, TB, TE, KVH, ROW)                                                         \
-  do {                                                                                                 \
-    const int pt0_ = (TB) + (KS) * S::kTS;                                                             \
-    const int pntok_ = cmin(S::kTS, (TE) - pt0_);                                                      \
-    const int pnbox_ = (pntok_ + kBoxTokens - 1) / kBoxTokens;                                         \
-    const int prel_ = (KS) * S::kGroups + (op_box < S::kGroups ? op_box : 0);                          \
-    int pblk_ = -1;                                                                                    \
-    _Pragma("unroll") for (int j_ = 0; j_ < kIdWindow; ++j_) {                                         \
-      const int v_ = __shfl_sync(0xffffffffu, IDS[j_], prel_ & 31);                                    \
-      if ((prel_ >> 5) == j_) pblk_ = v_;                                                              \
-    }                                                                                                  \
-    if (pntok_ > 0 && op_box < pnbox_ && lane < 2 * S::kChunks * S::kGroups && pblk_ >= 0 &&           \
-        pblk_ < args.num_blocks)                                                                       \
-      tma_prefetch_l2_4d(op_kv ? &tmap_v : &tmap_k, op_ch * S::kChunkElems, (pt0_ + op_box * kBoxTokens) % bs, \
-                         (KVH), pblk_);                                                                \
-    (void)(ROW);                                                                                       \
-  } while (0)
 // Claiming the next item takes three steps spread over consecutive stages of the current one, so that
 // no step waits on the one before it: (1) the ticket's atomic, (2) the ticket's decode and the context
 // length's load, (3) the block-id window's loads. Each step is a no-op once done.
@@ -632,23 +612,8 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
           const int op_kv = (lane / S::kChunks) & 1;
           const int op_ch = lane % S::kChunks;
           const int claim_at = cmax(0, n_stages - kClaimAhead);
-          static_assert(kPrefetchAhead + 2 <= kClaimAhead, "the next item is known before its stages are prefetched");
           for (int k = 0; k < n_stages; ++k) {
             if (k >= claim_at) PA_CLAIM_STEP();
-            {
-              // L2 prefetch of the boxes kPrefetchAhead stages ahead (into the next item near the end of
-              // this one), so that DRAM latency is already under way when the ring slot frees.
-              const int kp = k + kPrefetchAhead;
-              if (kPrefetchAhead == 0) {
-              } else if (kp < n_stages) {
-                PA_PREFETCH(cur_ids, kp, tok_begin, tok_end, kvh0, row);
-              } else if (have_next && nxt_idx < num_tickets && nxt_L > 0 && !context_len_invalid(nxt_L, args)) {
-                const int nb = nxt_c.part * args.partition_size;
-                const int ne = cmin(nxt_L, nb + args.partition_size);
-                const int32_t* nrow = args.block_tables + static_cast<size_t>(nxt_c.s) * args.max_blocks_per_seq;
-                if (nb < ne) PA_PREFETCH(nxt_ids, kp - n_stages, nb, ne, nxt_c.hb * kHeadBlock, nrow);
-              }
-            }
             const int t0 = tok_begin + k * S::kTS;
             const int ntok = cmin(S::kTS, tok_end - t0);
             const int nbox = (ntok + kBoxTokens - 1) / kBoxTokens;
@@ -713,7 +678,6 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
       for (int j = 0; j < kIdWindow; ++j) cur_ids[j] = nxt_ids[j];
     }
 #undef PA_CLAIM_STEP
-#undef PA_PREFETCH
 #undef PA_PREPARE
     // No work left: one terminating message.
     if (!aborted) {
@@ -834,10 +798,12 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         const uint32_t vbase = kbase + S::kTileBytes;
         const int t4 = lane & 3;
         // ldmatrix row addresses: lane i points at token row i % 8 of this head (in box gr), unit i / 8.
-        float sacc[NG][4];
+        // Two accumulators per box (even and odd k-steps) halve the dependent MMA chain; summed after.
+        float sacc[NG][4], sacc2[NG][4];
 #pragma unroll
         for (int gr = 0; gr < NG; ++gr) {
           sacc[gr][0] = sacc[gr][1] = sacc[gr][2] = sacc[gr][3] = 0.f;
+          sacc2[gr][0] = sacc2[gr][1] = sacc2[gr][2] = sacc2[gr][3] = 0.f;
           const int lrow = tile_row(cw, gr * kBoxTokens + (lane & 7));
           if constexpr (EB == 2) {
 #pragma unroll
@@ -847,7 +813,7 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
               const uint32_t a0[4] = {qa[2 * q4][0], 0u, qa[2 * q4][1], 0u};
               mma_16816<MmaT>(sacc[gr], a0, kb[0], kb[1]);
               const uint32_t a1[4] = {qa[2 * q4 + 1][0], 0u, qa[2 * q4 + 1][1], 0u};
-              mma_16816<MmaT>(sacc[gr], a1, kb[2], kb[3]);
+              mma_16816<MmaT>(sacc2[gr], a1, kb[2], kb[3]);
             }
           } else {
             // FP8 rows are 128 bytes (one swizzle chunk, 16-byte unit u = 16 values of d). ldmatrix
@@ -864,10 +830,12 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
                 const uint32_t b0 = e4m3x2_to_f16x2(static_cast<uint16_t>(kb[j4] & 0xffffu));
                 const uint32_t b1 = e4m3x2_to_f16x2(static_cast<uint16_t>(kb[j4] >> 16));
                 const uint32_t a[4] = {qa[q4 * 4 + j4][0], 0u, qa[q4 * 4 + j4][1], 0u};
-                mma_16816<MmaT>(sacc[gr], a, b0, b1);
+                mma_16816<MmaT>((j4 & 1) ? sacc2[gr] : sacc[gr], a, b0, b1);
               }
             }
           }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sacc[gr][i] += sacc2[gr][i];
         }
         // Scores of query head lane/4 for tokens 8*gr + 2*t4 and 8*gr + 2*t4 + 1. FP8 scales: K's scales
         // the scores of its box, V's the weights that enter P V of its box (per-block scales), or the
