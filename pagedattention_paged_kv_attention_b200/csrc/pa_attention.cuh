@@ -892,43 +892,55 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
         for (int gr = 0; gr < NG; ++gr)
           vmask[gr] = (gr * kBoxTokens + 2 * t4 < nvalid ? 0x0000ffffu : 0u) |
                       (gr * kBoxTokens + 2 * t4 + 1 < nvalid ? 0xffff0000u : 0u);
-        if constexpr (EB == 2) {
-          static_assert(NG == 1, "16-bit caches use one box per stage");
-          const int lrow = tile_row(cw, lane & 7);
+        // A full stage (every stage but an item's last) has no invalid rows: its fragments skip the masks.
+        auto pv = [&](auto masked_tag) {
+          constexpr bool kMasked = decltype(masked_tag)::value;
+          if constexpr (EB == 2) {
+            static_assert(NG == 1, "16-bit caches use one box per stage");
+            const int lrow = tile_row(cw, lane & 7);
 #pragma unroll
-          for (int q4 = 0; q4 < S::kNBlocks / 4; ++q4) {
-            uint32_t vb[4];
-            ldmatrix_x4_trans(vbase + piece_offset<S>(lrow, q4 * 4 + (lane >> 3)), vb);
+            for (int q4 = 0; q4 < S::kNBlocks / 4; ++q4) {
+              uint32_t vb[4];
+              ldmatrix_x4_trans(vbase + piece_offset<S>(lrow, q4 * 4 + (lane >> 3)), vb);
 #pragma unroll
-            for (int j4 = 0; j4 < 4; ++j4) mma_1688<MmaT>(o[q4 * 4 + j4], pfrag[0], 0u, vb[j4] & vmask[0]);
-          }
-        } else {
-          // ldmatrix.trans over the byte rows of box gr gives lane (g, t4) the bytes
-          // [V[2t4][16u+2g], V[2t4][16u+2g+1], V[2t4+1][16u+2g], V[2t4+1][16u+2g+1]]; one byte permute
-          // splits them into the even-d fragment (block 2u: d = 16u + 2g) and the odd-d fragment
-          // (block 2u + 1: d = 16u + 2g + 1). The two boxes are the two k-halves of an m16n8k16 step.
-          static_assert(NG == 2, "FP8 caches use two boxes per stage");
-          const uint32_t a[4] = {pfrag[0], 0u, pfrag[1], 0u};
-          const uint32_t vaddr0 = vbase + tile_row(cw, lane & 7) * 128;
-          const uint32_t vaddr1 = vbase + tile_row(cw, kBoxTokens + (lane & 7)) * 128;
+              for (int j4 = 0; j4 < 4; ++j4)
+                mma_1688<MmaT>(o[q4 * 4 + j4], pfrag[0], 0u, kMasked ? (vb[j4] & vmask[0]) : vb[j4]);
+            }
+          } else {
+            // ldmatrix.trans over the byte rows of box gr gives lane (g, t4) the bytes
+            // [V[2t4][16u+2g], V[2t4][16u+2g+1], V[2t4+1][16u+2g], V[2t4+1][16u+2g+1]]; one byte permute
+            // splits them into the even-d fragment (block 2u: d = 16u + 2g) and the odd-d fragment
+            // (block 2u + 1: d = 16u + 2g + 1). The two boxes are the two k-halves of an m16n8k16 step.
+            static_assert(NG == 2, "FP8 caches use two boxes per stage");
+            const uint32_t a[4] = {pfrag[0], 0u, pfrag[1], 0u};
+            const uint32_t vaddr0 = vbase + tile_row(cw, lane & 7) * 128;
+            const uint32_t vaddr1 = vbase + tile_row(cw, kBoxTokens + (lane & 7)) * 128;
 #pragma unroll
-          for (int q4 = 0; q4 < S::kNBlocks / 8; ++q4) {
-            const uint32_t off = ((q4 * 4 + (lane >> 3)) ^ (lane & 7)) << 4;
-            uint32_t vb0[4], vb1[4];
-            ldmatrix_x4_trans(vaddr0 + off, vb0);
-            ldmatrix_x4_trans(vaddr1 + off, vb1);
+            for (int q4 = 0; q4 < S::kNBlocks / 8; ++q4) {
+              const uint32_t off = ((q4 * 4 + (lane >> 3)) ^ (lane & 7)) << 4;
+              uint32_t vb0[4], vb1[4];
+              ldmatrix_x4_trans(vaddr0 + off, vb0);
+              ldmatrix_x4_trans(vaddr1 + off, vb1);
 #pragma unroll
-            for (int j4 = 0; j4 < 4; ++j4) {
-              const int u = q4 * 4 + j4;
-              const uint32_t ev0 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb0[j4], 0u, 0x4420u))) & vmask[0];
-              const uint32_t ev1 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb1[j4], 0u, 0x4420u))) & vmask[1];
-              const uint32_t od0 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb0[j4], 0u, 0x4431u))) & vmask[0];
-              const uint32_t od1 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb1[j4], 0u, 0x4431u))) & vmask[1];
-              mma_16816<MmaT>(o[2 * u], a, ev0, ev1);
-              mma_16816<MmaT>(o[2 * u + 1], a, od0, od1);
+              for (int j4 = 0; j4 < 4; ++j4) {
+                const int u = q4 * 4 + j4;
+                uint32_t ev0 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb0[j4], 0u, 0x4420u)));
+                uint32_t ev1 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb1[j4], 0u, 0x4420u)));
+                uint32_t od0 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb0[j4], 0u, 0x4431u)));
+                uint32_t od1 = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(vb1[j4], 0u, 0x4431u)));
+                if constexpr (kMasked) {
+                  ev0 &= vmask[0];
+                  ev1 &= vmask[1];
+                  od0 &= vmask[0];
+                  od1 &= vmask[1];
+                }
+                mma_16816<MmaT>(o[2 * u], a, ev0, ev1);
+                mma_16816<MmaT>(o[2 * u + 1], a, od0, od1);
+              }
             }
           }
-        }
+        };
+        if (nvalid == S::kTS) pv(std::false_type{}); else pv(std::true_type{});
        }
       } else if (active) {
         const int nvalid = m.ntok;
