@@ -22,10 +22,15 @@
 
 namespace {
 
+// Automatic partition size. With the kernel's longest-first work order, a sweep on the B200 put the
+// best size where each persistent CTA gets about five items if every context were max_context_len
+// long (fewer, larger items mean fewer split-K partials to write and merge; the order keeps the tail
+// short), and never more than 32 partitions (the merge's cost grows with them): 768 for the 70B-shape
+// batch, 512-768 for 7B, 1024 for 8 x 32768 tokens.
 constexpr int kPlanSMs = 148;            // B200 SM count; planning is a pure function of the sizes
-constexpr int kPlanItemsPerCta = 16;     // work items per persistent CTA the automatic plan aims for
+constexpr int kPlanItemsPerCta = 5;
+constexpr int kPlanMaxPartitions = 32;
 constexpr int kMinAutoPartition = 256;
-constexpr int kMaxAutoPartition = 1024;
 
 using pa_host::aligned;
 using pa_host::ceil_div;
@@ -52,13 +57,18 @@ int plan_partition(int num_seqs, int num_heads, int num_kv_heads, int max_contex
     return -1;
   int g_tile, subgroups;
   group_tiling(num_heads / num_kv_heads, &g_tile, &subgroups);
-  const long items =
-      std::max<long>(1, static_cast<long>(num_seqs) * ceil_div(num_kv_heads, pa::kHeadBlock) * subgroups);
-  const long target = static_cast<long>(kPlanSMs) * kPlanItemsPerCta;
-  const long splits = std::max<long>(1, (target + items - 1) / items);
-  long ps = (std::max(1, max_context_len) + splits - 1) / splits;
-  ps = round_up(static_cast<size_t>(ps), pa::kPartitionQuantum);
-  ps = std::min<long>(std::max<long>(ps, kMinAutoPartition), kMaxAutoPartition);
+  const long long units =
+      std::max<long long>(1, static_cast<long long>(num_seqs) * ceil_div(num_kv_heads, pa::kHeadBlock) * subgroups);
+  const long long ctx = std::max(1, max_context_len);
+  const long long per_cta = static_cast<long long>(kPlanSMs) * kPlanItemsPerCta;
+  const long long balance = (units * ctx + per_cta - 1) / per_cta;              // ~5 items per CTA
+  const long long merge = (ctx + kPlanMaxPartitions - 1) / kPlanMaxPartitions;  // <= 32 partitions
+  long long ps = std::max<long long>({balance, merge, static_cast<long long>(kMinAutoPartition)});
+  ps = (ps + pa::kPartitionQuantum - 1) / pa::kPartitionQuantum * pa::kPartitionQuantum;
+  // No split beyond the context itself (one partition covers it); stays within int.
+  const long long whole = (ctx + pa::kPartitionQuantum - 1) / pa::kPartitionQuantum * pa::kPartitionQuantum;
+  ps = std::min<long long>(ps, std::max<long long>(whole, kMinAutoPartition));
+  ps = std::min<long long>(ps, 0x7fffffffLL / pa::kPartitionQuantum * pa::kPartitionQuantum);
   return static_cast<int>(ps);
 }
 
