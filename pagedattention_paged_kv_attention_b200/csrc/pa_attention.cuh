@@ -1156,7 +1156,41 @@ paged_attention_main(const __grid_constant__ CUtensorMap tmap_k, const __grid_co
 // the partitions; the partition statistics are read once per lane group. Sequences with one
 // partition (or an empty or invalid context) were finished by the main kernel.
 constexpr int kReduceWarps = 4;
-template <typename QT, int D>
+constexpr int kReduceSplitAbove = 16;  // more partitions than this: one CTA per row, its warps split them
+
+// Merges partitions p0 .. p1-1 of one row into (wsum, acc), in partition order: lane i computes the
+// weight of partition q + i once (one load of its m and l per warp instead of per lane) and the weights
+// reach every lane by shuffle.
+template <int D>
+__device__ __forceinline__ void merge_range(const AttnArgs& a, size_t base, int p0, int p1, float M, int lane,
+                                            float& wsum, float (&acc)[D / 32]) {
+  constexpr int kPer = D / 32;
+  const float* po = a.part_o + base * D + lane * kPer;
+  for (int q = p0; q < p1; q += 32) {
+    const int p = q + lane;
+    const float w_lane = p < p1 ? a.part_l[base + p] * fast_exp2(a.part_m[base + p] - M) : 0.f;
+    const int cnt = min(32, p1 - q);
+#pragma unroll 8
+    for (int i = 0; i < cnt; ++i) {
+      const float w = __shfl_sync(0xffffffffu, w_lane, i);
+      wsum += w;
+      if constexpr (kPer == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(po + static_cast<size_t>(q + i) * D);
+        acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(po + static_cast<size_t>(q + i) * D);
+        acc[0] += w * v.x; acc[1] += w * v.y;
+      }
+    }
+  }
+}
+
+// Split-K merge of partitions: out = sum_p w_p o_p / sum_p w_p with w_p = l_p 2^(m_p - max m).
+// SPLIT = false: one warp per (sequence, query head), lanes holding 4 (or 2) consecutive elements of the
+// row, walking the partitions. SPLIT = true (many partitions): one CTA per row; each of its warps
+// merges a quarter of the partitions and warp 0 adds the four results in warp order. Sequences with one
+// partition (or an empty or invalid context) were finished by the main kernel.
+template <typename QT, int D, bool SPLIT>
 __global__ void __launch_bounds__(kReduceWarps * 32)
 paged_attention_reduce(const AttnArgs args) {
   constexpr int kPer = D / 32;  // elements per lane: 4 for d = 128, 2 for d = 64
@@ -1171,8 +1205,8 @@ paged_attention_reduce(const AttnArgs args) {
     }
   } trace_end{args.trace};
 #endif
-  const int lane = threadIdx.x & 31;
-  const long row = static_cast<long>(blockIdx.x) * kReduceWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long row = SPLIT ? static_cast<long>(blockIdx.x) : static_cast<long>(blockIdx.x) * kReduceWarps + warp;
   if (row >= static_cast<long>(args.num_seqs) * args.num_heads) return;
   const int s = static_cast<int>(row / args.num_heads);
   const int L = args.context_lens[s];
@@ -1189,25 +1223,27 @@ paged_attention_reduce(const AttnArgs args) {
   float acc[kPer];
 #pragma unroll
   for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-  const float* po = args.part_o + base * D + lane * kPer;
-  // Partitions in chunks of 32: lane i computes the weight of partition p0 + i once (one load of its
-  // m and l per warp instead of per lane); the weights reach every lane by shuffle, in partition order.
-  for (int p0 = 0; p0 < n_parts; p0 += 32) {
-    const int p = p0 + lane;
-    const float w_lane = p < n_parts ? args.part_l[base + p] * fast_exp2(args.part_m[base + p] - M) : 0.f;
-    const int cnt = min(32, n_parts - p0);
-#pragma unroll 8
-    for (int i = 0; i < cnt; ++i) {
-      const float w = __shfl_sync(0xffffffffu, w_lane, i);
-      wsum += w;
-      if constexpr (kPer == 4) {
-        const float4 v = *reinterpret_cast<const float4*>(po + static_cast<size_t>(p0 + i) * D);
-        acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
-      } else {
-        const float2 v = *reinterpret_cast<const float2*>(po + static_cast<size_t>(p0 + i) * D);
-        acc[0] += w * v.x; acc[1] += w * v.y;
-      }
+  if constexpr (SPLIT) {
+    const int chunk = (n_parts + kReduceWarps - 1) / kReduceWarps;
+    merge_range<D>(args, base, min(n_parts, warp * chunk), min(n_parts, (warp + 1) * chunk), M, lane, wsum, acc);
+    __shared__ float part_acc[kReduceWarps][D];
+    __shared__ float part_wsum[kReduceWarps];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) part_acc[warp][lane * kPer + k] = acc[k];
+    if (lane == 0) part_wsum[warp] = wsum;
+    __syncthreads();
+    if (warp != 0) return;
+    wsum = part_wsum[0];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) acc[k] = part_acc[0][lane * kPer + k];
+#pragma unroll
+    for (int w = 1; w < kReduceWarps; ++w) {
+      wsum += part_wsum[w];
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) acc[k] += part_acc[w][lane * kPer + k];
     }
+  } else {
+    merge_range<D>(args, base, 0, n_parts, M, lane, wsum, acc);
   }
   const float r = 1.0f / wsum;
   QT* out = static_cast<QT*>(args.out) + static_cast<size_t>(row) * D + lane * kPer;

@@ -24,9 +24,13 @@ cudaError_t launch_attention_one(const CUtensorMap& tk, const CUtensorMap& tv, c
   if (e != cudaSuccess) return e;
   if (a.num_partitions > 1) {
     const long rows = static_cast<long>(a.num_heads) * a.num_seqs;
-    e = pa_host::launch_overlapped(paged_attention_reduce<QT, D>,
-                                   dim3(static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps)),
-                                   dim3(kReduceWarps * 32), 0, stream, a);
+    if (a.num_partitions > kReduceSplitAbove)
+      e = pa_host::launch_overlapped(paged_attention_reduce<QT, D, true>, dim3(static_cast<unsigned>(rows)),
+                                     dim3(kReduceWarps * 32), 0, stream, a);
+    else
+      e = pa_host::launch_overlapped(paged_attention_reduce<QT, D, false>,
+                                     dim3(static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps)),
+                                     dim3(kReduceWarps * 32), 0, stream, a);
   }
   return e;
 }
