@@ -30,7 +30,7 @@ import workloads as W  # noqa: E402
 
 METRIC = "paged decode attention: achieved KV-read HBM GB/s & % of peak; tokens/s"
 KERNEL_SOURCES = ("pa_attention.cuh", "pa_device.cuh", "pa_launch.cuh")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "paged_attention_main_7b_traffic.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "paged_attention_main_traffic.json")
 THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
                  0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                  0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
@@ -63,7 +63,8 @@ def recorded_traffic(workload):
         rec = json.load(open(TRAFFIC_FILE))
     except (OSError, ValueError):
         return None
-    if rec.get("kernel_source_hash") != kernel_source_hash() or rec.get("workload") != workload:
+    rec = rec.get(workload)
+    if not rec or rec.get("kernel_source_hash") != kernel_source_hash():
         return None
     return rec.get("dram_bytes_per_launch")
 
