@@ -368,6 +368,7 @@ def measure_decode(args, cfg, P, dev, rank, world, peak, peak_measured, checks):
     max_step_ms = reduce_max(step_ms, world, dev)
     total_kv = reduce_sum(float(ideal["kv"]), world, dev)
     total_seqs = reduce_sum(float(S), world, dev)
+    total_ctx = reduce_sum(float(np.sum(lens)), world, dev)
     value = total_kv / (max_step_ms * 1e-3) / 1e9
 
     # ---- end to end through the API: pinned host inputs in, output back to pinned host ----
@@ -433,6 +434,7 @@ def measure_decode(args, cfg, P, dev, rank, world, peak, peak_measured, checks):
         "value": round(value, 2), "ms_per_step": round(max_step_ms, 4),
         "plan": {"partition_size": ps, "partitions": parts, "num_seqs": S},
         "tokens_per_s": round(total_seqs / (max_step_ms * 1e-3), 1),
+        "context_tokens_per_s": round(total_ctx / (max_step_ms * 1e-3), 1),
         "pct_of_measured_hbm_peak": round(100 * value / peak, 2),
         "pct_of_8tbs": round(100 * value / 8000.0, 2),
         "roofline": {"kernel": "paged_attention (pa_paged_attention call: main kernel%s)" %
