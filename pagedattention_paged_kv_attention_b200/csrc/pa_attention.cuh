@@ -1215,15 +1215,51 @@ paged_attention_reduce(const AttnArgs args) {
   const int n_parts = (L + PS - 1) / PS;
   if (n_parts <= 1) return;
   const size_t base = static_cast<size_t>(row) * args.num_partitions;
-  float M = -INFINITY;
-  for (int p = lane; p < n_parts; p += 32) M = fmaxf(M, args.part_m[base + p]);
-#pragma unroll
-  for (int b = 16; b > 0; b >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, b));
   float wsum = 0.f;
   float acc[kPer];
 #pragma unroll
   for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-  if constexpr (SPLIT) {
+  if constexpr (!SPLIT) {
+    // At most kReduceSplitAbove partitions: every load of the row (lane p's m and l, and each lane's
+    // elements of every partition) is issued before any result is needed, so the row costs one
+    // load round trip. Same order and arithmetic as merge_range.
+    float m_lane = -INFINITY, l_lane = 0.f;
+    if (lane < n_parts) {
+      m_lane = args.part_m[base + lane];
+      l_lane = args.part_l[base + lane];
+    }
+    const float* po = args.part_o + base * D + lane * kPer;
+    float ov[kReduceSplitAbove][kPer];
+#pragma unroll
+    for (int p = 0; p < kReduceSplitAbove; ++p) {
+      if (p < n_parts) {
+        if constexpr (kPer == 4) {
+          const float4 v = *reinterpret_cast<const float4*>(po + static_cast<size_t>(p) * D);
+          ov[p][0] = v.x; ov[p][1] = v.y; ov[p][2] = v.z; ov[p][3] = v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2*>(po + static_cast<size_t>(p) * D);
+          ov[p][0] = v.x; ov[p][1] = v.y;
+        }
+      }
+    }
+    float M = m_lane;
+#pragma unroll
+    for (int b = 16; b > 0; b >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, b));
+    const float w_lane = lane < n_parts ? l_lane * fast_exp2(m_lane - M) : 0.f;
+#pragma unroll
+    for (int p = 0; p < kReduceSplitAbove; ++p) {
+      if (p < n_parts) {
+        const float w = __shfl_sync(0xffffffffu, w_lane, p);
+        wsum += w;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) acc[k] += w * ov[p][k];
+      }
+    }
+  } else {
+    float M = -INFINITY;
+    for (int p = lane; p < n_parts; p += 32) M = fmaxf(M, args.part_m[base + p]);
+#pragma unroll
+    for (int b = 16; b > 0; b >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, b));
     const int chunk = (n_parts + kReduceWarps - 1) / kReduceWarps;
     merge_range<D>(args, base, min(n_parts, warp * chunk), min(n_parts, (warp + 1) * chunk), M, lane, wsum, acc);
     __shared__ float part_acc[kReduceWarps][D];
@@ -1242,8 +1278,6 @@ paged_attention_reduce(const AttnArgs args) {
 #pragma unroll
       for (int k = 0; k < kPer; ++k) acc[k] += part_acc[w][lane * kPer + k];
     }
-  } else {
-    merge_range<D>(args, base, 0, n_parts, M, lane, wsum, acc);
   }
   const float r = 1.0f / wsum;
   QT* out = static_cast<QT*>(args.out) + static_cast<size_t>(row) * D + lane * kPer;
