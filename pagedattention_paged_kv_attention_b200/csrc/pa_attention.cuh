@@ -1188,8 +1188,9 @@ __device__ __forceinline__ void merge_range(const AttnArgs& a, size_t base, int 
 // Split-K merge of partitions: out = sum_p w_p o_p / sum_p w_p with w_p = l_p 2^(m_p - max m).
 // SPLIT = false: one warp per (sequence, query head), lanes holding 4 (or 2) consecutive elements of the
 // row, walking the partitions. SPLIT = true (many partitions): one CTA per row; each of its warps
-// merges a quarter of the partitions and warp 0 adds the four results in warp order. Sequences with one
-// partition (or an empty or invalid context) were finished by the main kernel.
+// merges a quarter of the partitions against their own max, and warp 0 brings the four results to the
+// row's max and adds them in warp order. Sequences with one partition (or an empty or invalid context)
+// were finished by the main kernel.
 template <typename QT, int D, bool SPLIT>
 __global__ void __launch_bounds__(kReduceWarps * 32)
 paged_attention_reduce(const AttnArgs args) {
@@ -1256,27 +1257,75 @@ paged_attention_reduce(const AttnArgs args) {
       }
     }
   } else {
-    float M = -INFINITY;
-    for (int p = lane; p < n_parts; p += 32) M = fmaxf(M, args.part_m[base + p]);
-#pragma unroll
-    for (int b = 16; b > 0; b >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, b));
     const int chunk = (n_parts + kReduceWarps - 1) / kReduceWarps;
-    merge_range<D>(args, base, min(n_parts, warp * chunk), min(n_parts, (warp + 1) * chunk), M, lane, wsum, acc);
+    const int p0 = min(n_parts, warp * chunk), p1 = min(n_parts, (warp + 1) * chunk);
+    float Mw;  // the max this warp's weights are taken against
+    if (chunk <= kReduceSplitAbove) {
+      // One load round trip, as above, over this warp's partitions and against their own max; the
+      // warps' results are brought to the row's max when they are added.
+      float m_lane = -INFINITY, l_lane = 0.f;
+      if (p0 + lane < p1) {
+        m_lane = args.part_m[base + p0 + lane];
+        l_lane = args.part_l[base + p0 + lane];
+      }
+      const float* po = args.part_o + (base + p0) * D + lane * kPer;
+      float ov[kReduceSplitAbove][kPer];
+#pragma unroll
+      for (int p = 0; p < kReduceSplitAbove; ++p) {
+        if (p0 + p < p1) {
+          if constexpr (kPer == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(po + static_cast<size_t>(p) * D);
+            ov[p][0] = v.x; ov[p][1] = v.y; ov[p][2] = v.z; ov[p][3] = v.w;
+          } else {
+            const float2 v = *reinterpret_cast<const float2*>(po + static_cast<size_t>(p) * D);
+            ov[p][0] = v.x; ov[p][1] = v.y;
+          }
+        }
+      }
+      Mw = m_lane;
+#pragma unroll
+      for (int b = 16; b > 0; b >>= 1) Mw = fmaxf(Mw, __shfl_xor_sync(0xffffffffu, Mw, b));
+      const float w_lane = p0 + lane < p1 ? l_lane * fast_exp2(m_lane - Mw) : 0.f;
+#pragma unroll
+      for (int p = 0; p < kReduceSplitAbove; ++p) {
+        if (p0 + p < p1) {
+          const float w = __shfl_sync(0xffffffffu, w_lane, p);
+          wsum += w;
+#pragma unroll
+          for (int k = 0; k < kPer; ++k) acc[k] += w * ov[p][k];
+        }
+      }
+    } else {
+      Mw = -INFINITY;
+      for (int p = lane; p < n_parts; p += 32) Mw = fmaxf(Mw, args.part_m[base + p]);
+#pragma unroll
+      for (int b = 16; b > 0; b >>= 1) Mw = fmaxf(Mw, __shfl_xor_sync(0xffffffffu, Mw, b));
+      merge_range<D>(args, base, p0, p1, Mw, lane, wsum, acc);
+    }
     __shared__ float part_acc[kReduceWarps][D];
     __shared__ float part_wsum[kReduceWarps];
+    __shared__ float part_max[kReduceWarps];
 #pragma unroll
     for (int k = 0; k < kPer; ++k) part_acc[warp][lane * kPer + k] = acc[k];
-    if (lane == 0) part_wsum[warp] = wsum;
+    if (lane == 0) {
+      part_wsum[warp] = wsum;
+      part_max[warp] = Mw;
+    }
     __syncthreads();
     if (warp != 0) return;
-    wsum = part_wsum[0];
+    float M = part_max[0];
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) acc[k] = part_acc[0][lane * kPer + k];
+    for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, part_max[w]);
+    wsum = 0.f;
 #pragma unroll
-    for (int w = 1; w < kReduceWarps; ++w) {
-      wsum += part_wsum[w];
+    for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
 #pragma unroll
-      for (int k = 0; k < kPer; ++k) acc[k] += part_acc[w][lane * kPer + k];
+    for (int w = 0; w < kReduceWarps; ++w) {
+      // A warp without partitions has max -inf and adds nothing (factor 0).
+      const float f = part_wsum[w] > 0.f ? fast_exp2(part_max[w] - M) : 0.f;
+      wsum += f * part_wsum[w];
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) acc[k] += f * part_acc[w][lane * kPer + k];
     }
   }
   const float r = 1.0f / wsum;
