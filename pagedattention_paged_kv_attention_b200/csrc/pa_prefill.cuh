@@ -215,6 +215,19 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
   }
   const int nkv = p_max / kKvTile + 1;  // = nkv_t of the last active tile
 
+  // The TMA warp fetches its tensor maps and the first KV tile's block ids now, so that those loads
+  // overlap the set-up below.
+  int blk_first = 0;
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tq);
+      tma_prefetch_desc(&tk);
+      tma_prefetch_desc(&tv);
+    }
+    if (lane * a.block_size < min(kKvTile, p_max + 1))
+      blk_first = __ldg(a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq + lane);
+  }
+
   // ---- set-up: barriers (thread 0), TMEM (warp 1) ----
   if (threadIdx.x == 0) {
     mbar_init(&b->q_full, 1);
@@ -268,7 +281,7 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
       int blk = 0;
       bool ok = false;
       if (lane < nblk) {
-        blk = table[first / bs + lane];
+        blk = j == 0 ? blk_first : table[first / bs + lane];
         ok = blk >= 0 && blk < a.num_blocks;
         if (!ok) atomicOr(err, PA_DEVERR_BLOCK_ID);
       }
