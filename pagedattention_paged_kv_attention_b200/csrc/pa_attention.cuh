@@ -1191,7 +1191,9 @@ __device__ __forceinline__ void merge_range(const AttnArgs& a, size_t base, int 
 // merges a quarter of the partitions against their own max, and warp 0 brings the four results to the
 // row's max and adds them in warp order. Sequences with one partition (or an empty or invalid context)
 // were finished by the main kernel.
-template <typename QT, int D, bool SPLIT>
+// MAXP (SPLIT = false): a bound on the partition count the launch was sized for (4, 8 or 16), so that a
+// row's preloaded values take no more registers than it needs and more warps stay resident.
+template <typename QT, int D, bool SPLIT, int MAXP = kReduceSplitAbove>
 __global__ void __launch_bounds__(kReduceWarps * 32)
 paged_attention_reduce(const AttnArgs args) {
   constexpr int kPer = D / 32;  // elements per lane: 4 for d = 128, 2 for d = 64
@@ -1221,7 +1223,7 @@ paged_attention_reduce(const AttnArgs args) {
 #pragma unroll
   for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
   if constexpr (!SPLIT) {
-    // At most kReduceSplitAbove partitions: every load of the row (lane p's m and l, and each lane's
+    // At most MAXP partitions: every load of the row (lane p's m and l, and each lane's
     // elements of every partition) is issued before any result is needed, so the row costs one
     // load round trip. Same order and arithmetic as merge_range.
     float m_lane = -INFINITY, l_lane = 0.f;
@@ -1230,9 +1232,9 @@ paged_attention_reduce(const AttnArgs args) {
       l_lane = args.part_l[base + lane];
     }
     const float* po = args.part_o + base * D + lane * kPer;
-    float ov[kReduceSplitAbove][kPer];
+    float ov[MAXP][kPer];
 #pragma unroll
-    for (int p = 0; p < kReduceSplitAbove; ++p) {
+    for (int p = 0; p < MAXP; ++p) {
       if (p < n_parts) {
         if constexpr (kPer == 4) {
           const float4 v = *reinterpret_cast<const float4*>(po + static_cast<size_t>(p) * D);
@@ -1248,7 +1250,7 @@ paged_attention_reduce(const AttnArgs args) {
     for (int b = 16; b > 0; b >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, b));
     const float w_lane = lane < n_parts ? l_lane * fast_exp2(m_lane - M) : 0.f;
 #pragma unroll
-    for (int p = 0; p < kReduceSplitAbove; ++p) {
+    for (int p = 0; p < MAXP; ++p) {
       if (p < n_parts) {
         const float w = __shfl_sync(0xffffffffu, w_lane, p);
         wsum += w;

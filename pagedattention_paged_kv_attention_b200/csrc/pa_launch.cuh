@@ -27,10 +27,18 @@ cudaError_t launch_attention_one(const CUtensorMap& tk, const CUtensorMap& tv, c
     if (a.num_partitions > kReduceSplitAbove)
       e = pa_host::launch_overlapped(paged_attention_reduce<QT, D, true>, dim3(static_cast<unsigned>(rows)),
                                      dim3(kReduceWarps * 32), 0, stream, a);
-    else
-      e = pa_host::launch_overlapped(paged_attention_reduce<QT, D, false>,
-                                     dim3(static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps)),
-                                     dim3(kReduceWarps * 32), 0, stream, a);
+    else {
+      const dim3 grid(static_cast<unsigned>((rows + kReduceWarps - 1) / kReduceWarps));
+      if (a.num_partitions <= 4)
+        e = pa_host::launch_overlapped(paged_attention_reduce<QT, D, false, 4>, grid, dim3(kReduceWarps * 32), 0,
+                                       stream, a);
+      else if (a.num_partitions <= 8)
+        e = pa_host::launch_overlapped(paged_attention_reduce<QT, D, false, 8>, grid, dim3(kReduceWarps * 32), 0,
+                                       stream, a);
+      else
+        e = pa_host::launch_overlapped(paged_attention_reduce<QT, D, false, 16>, grid, dim3(kReduceWarps * 32), 0,
+                                       stream, a);
+    }
   }
   return e;
 }
